@@ -1,0 +1,448 @@
+"""Benchmark of the paged decode step on B200.
+
+A step is one pass of the whole hot path over one batch: copy-on-write block
+copies (when the workload has forks), the append of the step's new tokens,
+and block-table decode attention (partition kernel + split-K reduce).  The
+default workload is MHA decode: batch 64, 32 query = 32 KV heads, head_dim
+128, bf16, block_size 16, context lengths U[128, 2048], pool of 16384 blocks
+placed by a seeded permutation, one new token per sequence.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the fp64 CPU oracle, bounded sample
+
+Prints one JSON line (rank 0).  Under torchrun each rank runs its own batch
+(weak scaling, no data-path collective); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_323_b200 import workload as wl  # noqa: E402
+
+METRIC = "paged decode-attention KV-read HBM GB/s (% of B200 peak) and tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+WORKLOADS = {
+    "mha": ("mha_decode_b64_h32_kv32_d128_bs16_ctxU128-2048_bf16",
+            lambda dev, seed: wl.mha(seed=seed, device=dev)),
+    "gqa_sampling": ("gqa_sampling_b256_g64x4_h32_kv8_d128_bs16_bf16",
+                     lambda dev, seed: wl.gqa_sampling(seed=seed, device=dev)),
+    "long_context": ("long_context_b8_h64_kv8_d128_bs32_ctxU32768-131072_bf16",
+                     lambda dev, seed: wl.long_context(seed=seed, device=dev)),
+    "prefix_bs8": ("prefix_sweep_b1024_prefix2048_h32_kv8_d128_bs8_bf16",
+                   lambda dev, seed: wl.prefix_sweep(8, seed=seed, device=dev)),
+    "prefix_bs16": ("prefix_sweep_b1024_prefix2048_h32_kv8_d128_bs16_bf16",
+                    lambda dev, seed: wl.prefix_sweep(16, seed=seed, device=dev)),
+    "prefix_bs32": ("prefix_sweep_b1024_prefix2048_h32_kv8_d128_bs32_bf16",
+                    lambda dev, seed: wl.prefix_sweep(32, seed=seed, device=dev)),
+    "tiny": ("tiny_b4_ctx35-16-1-50_h4_d64_bs16_f32", lambda dev, seed: wl.tiny(seed=seed, device=dev)),
+}
+DEFAULT_SEED = {"mha": 2, "gqa_sampling": 3, "long_context": 4, "prefix_bs8": 5, "prefix_bs16": 5,
+                "prefix_bs32": 5, "tiny": 1}
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def committed_traffic(kernel: str, workload: str, source_sha: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.traffic.txt")
+    if not os.path.exists(path):
+        return None
+    kv = {}
+    for line in open(path):
+        if "=" in line and not line.startswith("#"):
+            k, v = line.split("=", 1)
+            kv[k.strip()] = v.strip()
+    if kv.get("kernel_source_sha256") != source_sha:
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def kernel_source_sha() -> str:
+    import hashlib
+
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_323_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.startswith("decode") or name in ("common.cuh",):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(world, x: float) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def compact_subset(w: wl.Workload, seqs):
+    """The step restricted to ``seqs`` on a compact host pool (oracle input)."""
+    bs = w.block_size
+    seqs = list(seqs)
+    sel_pairs = [i for i, s in enumerate(w.pair_seq.tolist()) if s in seqs]
+    blocks = set()
+    for s in seqs:
+        nb = -(-int(w.context_lens[s]) // bs)
+        blocks.update(int(x) for x in w.block_tables[s][:nb])
+    for i in sel_pairs:
+        blocks.update(int(x) for x in w.cow_pairs[i])
+    order = sorted(blocks)
+    remap = {b: i for i, b in enumerate(order)}
+    idx = torch.tensor(order, dtype=torch.long, device=w.k_cache.device)
+    kc = wl.to_numpy_bits(w.k_cache.index_select(0, idx))
+    vc = wl.to_numpy_bits(w.v_cache.index_select(0, idx))
+    bt = np.full((len(seqs), w.max_blocks_per_seq), -1, dtype=np.int32)
+    for i, s in enumerate(seqs):
+        nb = -(-int(w.context_lens[s]) // bs)
+        bt[i, :nb] = [remap[int(x)] for x in w.block_tables[s][:nb]]
+    toks = [i for i, s in enumerate(w.token_seq.tolist()) if s in seqs]
+    slots = np.asarray([remap[int(w.slot_mapping[i]) // bs] * bs + int(w.slot_mapping[i]) % bs
+                        for i in toks], dtype=np.int64)
+    tok_idx = torch.tensor(toks, dtype=torch.long, device=w.k_new.device)
+    pairs = np.asarray([[remap[int(w.cow_pairs[i][0])], remap[int(w.cow_pairs[i][1])]]
+                        for i in sel_pairs], dtype=np.int64).reshape(-1, 2)
+    q = wl.to_numpy_bits(w.q.index_select(0, torch.tensor(seqs, device=w.q.device)))
+    return dict(q=q, kc=kc, vc=vc, bt=bt, ctx=w.context_lens[seqs].copy(), slots=slots,
+                k_new=wl.to_numpy_bits(w.k_new.index_select(0, tok_idx)),
+                v_new=wl.to_numpy_bits(w.v_new.index_select(0, tok_idx)), pairs=pairs,
+                kv_bytes=int(w.context_lens[seqs].astype(np.int64).sum()) * w.num_kv_heads
+                * w.head_dim * 2 * w.elt)
+
+
+def oracle_sample_step(sub, scale, threads):
+    import oracle
+
+    kc = sub["kc"].copy()
+    vc = sub["vc"].copy()
+    t0 = time.perf_counter()
+    if len(sub["pairs"]):
+        oracle.copy_blocks(kc, vc, sub["pairs"])
+    oracle.kv_append(kc, vc, sub["k_new"], sub["v_new"], sub["slots"])
+    oracle.paged_attention(sub["q"], kc, vc, sub["bt"], sub["ctx"], scale, nthreads=threads)
+    return time.perf_counter() - t0
+
+
+def pick_sample(w: wl.Workload, target_s: float, threads: int):
+    """Grow a seeded sample of sequences until one oracle step costs about target_s."""
+    rng = np.random.default_rng(1234)
+    order = rng.permutation(w.num_seqs).tolist()
+    n = min(len(order), max(1, threads))
+    while True:
+        sub = compact_subset(w, sorted(order[:n]))
+        dt = oracle_sample_step(sub, w.scale, threads)
+        if dt >= target_s / 4 or n >= len(order):
+            break
+        n = min(len(order), max(n + 1, int(n * min(8.0, target_s / 4 / max(dt, 1e-3)))))
+    return sub, n, dt
+
+
+def cpu_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, world, rank):
+    """The oracle as it stands, timed on host cores, on a bounded sample."""
+    if rank != 0:
+        return
+    name, make = WORKLOADS[args.workload]
+    w = make("cuda", DEFAULT_SEED[args.workload])
+    threads = cpu_threads()
+    sub, n, _ = pick_sample(w, target_s=8.0 / max(1, args.steps), threads=threads)
+    for _ in range(min(args.warmup, 1)):
+        oracle_sample_step(sub, w.scale, threads)
+    times = [oracle_sample_step(sub, w.scale, threads) for _ in range(args.steps)]
+    t = sum(times) / len(times)
+    value = sub["kv_bytes"] / t / 1e9
+    sample = f"{n} of {w.num_seqs} sequences (seeded), all heads, per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": name},
+        "tokens_per_s": n / t,
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_gpu(args, world, rank, local):
+    from paged_kv_cache_323_b200 import pagedkv as pk
+
+    name, make = WORKLOADS[args.workload]
+    seed = DEFAULT_SEED[args.workload] + 1000 * rank  # each rank its own batch (weak scaling)
+    w = make("cuda", seed)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    t = {
+        "q": w.q, "k_cache": w.k_cache, "v_cache": w.v_cache, "k_new": w.k_new, "v_new": w.v_new,
+        "bt": torch.from_numpy(w.block_tables).to(dev),
+        "ctx": torch.from_numpy(w.context_lens).to(dev),
+        "slots": torch.from_numpy(w.slot_mapping).to(dev),
+        "pairs": torch.from_numpy(w.cow_pairs).to(dev),
+    }
+    out = torch.empty_like(w.q)
+    ws_bytes = pk.paged_attention_workspace_size(w.num_seqs, w.num_heads,
+                                                 w.max_blocks_per_seq * w.block_size, w.head_dim,
+                                                 args.partition_tokens)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(q, k_new, v_new, bt, ctx, slots):
+        if len(w.cow_pairs):
+            pk.copy_blocks(t["k_cache"], t["v_cache"], t["pairs"])
+        pk.kv_cache_append(t["k_cache"], t["v_cache"], k_new, v_new, slots)
+        pk.paged_attention_decode_ex(out, q, t["k_cache"], t["v_cache"], bt, ctx, w.scale,
+                                     num_blocks=w.num_blocks,
+                                     partition_tokens=args.partition_tokens,
+                                     workspace=ws if ws_bytes else None)
+
+    dev_args = (t["q"], t["k_new"], t["v_new"], t["bt"], t["ctx"], t["slots"])
+    for _ in range(args.warmup):
+        step(*dev_args)
+    torch.cuda.synchronize()
+    code = pk.get_device_error()
+    if code != 0:
+        raise RuntimeError(f"device error word {code} after warm-up")
+
+    # ------------------------------------------------ device-resident timing
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    phys = vis.split(",")[local] if vis and len(vis.split(",")) > local else str(local)
+    clocks = ClockSampler(int(phys) if phys.isdigit() else local)
+    pk.profile_reset()
+    pk.profile_enable(True)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    launches0 = pk.launch_count()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step(*dev_args)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    launches = pk.launch_count() - launches0
+    clock_info = clocks.stop()
+    pk.profile_enable(False)
+    barrier(world)
+    ms = max_over_ranks(world, ev0.elapsed_time(ev1))
+    per_kernel = {}
+    for kind, kname in ((pk.KERNEL_DECODE_PARTITION, "decode_partition"),
+                        (pk.KERNEL_DECODE_REDUCE, "decode_reduce"), (pk.KERNEL_APPEND, "kv_append"),
+                        (pk.KERNEL_COPY_BLOCKS, "copy_blocks")):
+        n, kms = pk.profile_read(kind)
+        if n:
+            per_kernel[kname] = {"launches": n, "avg_us": kms / n * 1e3}
+    pk.profile_reset()
+
+    # -------------------------------------------- end to end from host memory
+    host = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True).copy_(v)
+            for k, v in zip(("q", "k_new", "v_new", "bt", "ctx", "slots"), dev_args)}
+    staged = {k: torch.empty_like(v) for k, v in zip(("q", "k_new", "v_new", "bt", "ctx", "slots"),
+                                                      dev_args)}
+    out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        for k in staged:
+            staged[k].copy_(host[k], non_blocking=True)
+        step(staged["q"], staged["k_new"], staged["v_new"], staged["bt"], staged["ctx"],
+             staged["slots"])
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_e2e = max_over_ranks(world, ev0.elapsed_time(ev1))
+    code = pk.get_device_error()
+    if code != 0:
+        raise RuntimeError(f"device error word {code} after the timed steps")
+
+    if rank != 0:
+        return
+    kv_bytes = w.kv_bytes_logical()
+    step_s = ms / args.steps / 1e3
+    value = world * kv_bytes / step_s / 1e9
+    peak, peak_src = measured_peak()
+    part = per_kernel.get("decode_partition")
+    roofline = None
+    if part:
+        achieved = kv_bytes / (part["avg_us"] * 1e-6) / 1e9
+        traffic = committed_traffic("decode_partition", args.workload, kernel_source_sha())
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                    "frac": achieved / peak, "traffic": traffic,
+                    "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+                    else "fallback 6650 GB/s"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": name, "num_seqs_per_gpu": w.num_seqs, "num_heads": w.num_heads,
+                   "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
+                   "block_size": w.block_size, "kv_bytes_per_step_per_gpu": kv_bytes,
+                   "partition_tokens": args.partition_tokens or 512,
+                   "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush",
+                   "parallelism": f"{world} independent batches, one per GPU"},
+        "tokens_per_s": world * w.num_seqs / step_s,
+        "pct_of_peak_hbm": 100.0 * value / peak,
+        "per_kernel_us": per_kernel,
+        "roofline": roofline,
+        "gpu_launches": launches,
+        "e2e": {"value": world * kv_bytes / (ms_e2e / args.steps / 1e3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": ms_e2e / args.steps},
+        "clocks": clock_info,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        threads = cpu_threads()
+        sub, n, _ = pick_sample(w, target_s=12.0, threads=threads)
+        dt = oracle_sample_step(sub, w.scale, threads)
+        line["cpu_baseline"] = {"value": sub["kv_bytes"] / dt / 1e9, "unit": "GB/s",
+                                "cores": threads, "kind": "oracle",
+                                "sample": f"{n} of {w.num_seqs} sequences (seeded), all heads, "
+                                          f"one step, {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="pagedkv", choices=["pagedkv", "reference"])
+    ap.add_argument("--workload", default="mha", choices=sorted(WORKLOADS))
+    ap.add_argument("--partition-tokens", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_gpu(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,186 @@
+/*
+ * pagedkv.h -- C ABI of libpagedkv.so, the B200 (sm_100a) paged KV-cache
+ * decode path.
+ *
+ * The method (PagedAttention) keeps each sequence's keys and values in
+ * fixed-size physical blocks that may sit anywhere in a pool, and maps the
+ * sequence's logical blocks to them through a per-sequence block table
+ * ("PagedAttention Explained: Virtual Memory for the KV Cache", section "How
+ * PagedAttention works", items 1-5).  This library provides the three device
+ * operations of that design: the block-aware decode attention that gathers K
+ * and V through the table (item 5), the append of new tokens' K/V into their
+ * slots (section "The problem: the KV cache is big and unpredictable": the
+ * cache grows by one entry per new token), and the block copy of
+ * copy-on-write (section "Sharing blocks between sequences").
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Pools: k_cache and v_cache are separate device arrays, each laid out
+ *    [num_blocks][num_kv_heads][block_size][head_dim], row-major, elements of
+ *    `dtype`.  One (block, kv head) slice is block_size*head_dim contiguous
+ *    elements.  Both base pointers must be 16-byte aligned.
+ *  - Token t of sequence s lives in physical block block_tables[s][t / bs] at
+ *    slot t % bs; the physical slot index is block*bs + slot.
+ *  - q and out are [num_seqs][num_heads][head_dim]; query head h reads kv head
+ *    h / (num_heads / num_kv_heads) (contiguous groups, grouped-query
+ *    attention; "Trade-offs and related techniques").
+ *  - context_lens[s] counts every token the query attends, including tokens
+ *    appended in this step; block_tables entries at index >=
+ *    ceil(context_lens[s] / bs) are never read.
+ *  - Attention is softmax(scale * q K^T) V over those tokens, accumulated in
+ *    fp32, with out rounded to `dtype` (round to nearest even for bf16).  A
+ *    sequence with context length 0 gets a zero output row.
+ *  - All device pointers are owned by the caller; the library never frees
+ *    them.  Every call is asynchronous on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream) and returns a status synchronously after
+ *    host-side validation and the launch.  Nothing is thrown across the ABI.
+ *  - Data-dependent faults found on the device (a table entry outside
+ *    [0, num_blocks), a slot outside the pool, a context length outside
+ *    [0, max_blocks_per_seq*bs], a wait that ran out of time) never trap: the
+ *    kernel skips the affected work (a bad block is left out of the softmax, a
+ *    bad sequence gets a zero row, a bad slot or pair is not written) and
+ *    records the first such status in a per-device error word that
+ *    pkv_get_device_error() returns.
+ *
+ * Supported shapes: head_dim in {64, 128}; block_size in {8, 16, 32};
+ * num_heads / num_kv_heads in {1, 2, 4, 8}; dtype PKV_F32 or PKV_BF16.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PKV_API __attribute__((visibility("default")))
+#else
+#define PKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every entry point. */
+typedef enum {
+    PKV_OK = 0,
+    PKV_ERR_NULL = -1,          /* a required pointer is NULL */
+    PKV_ERR_INVALID = -2,       /* an argument is out of its documented range */
+    PKV_ERR_UNSUPPORTED = -3,   /* a valid shape this build has no kernel for */
+    PKV_ERR_CUDA = -4,          /* the CUDA runtime reported an error */
+    PKV_ERR_WORKSPACE = -5,     /* split-K workspace missing or too small */
+    PKV_ERR_DEVICE_BOUNDS = -6, /* device word: a table entry, slot or length was out of range */
+    PKV_ERR_TIMEOUT = -7        /* device word: a bounded wait in a kernel ran out */
+} pkv_status;
+
+/* Element types of q, out, the pools and the new tokens. */
+typedef enum { PKV_F32 = 0, PKV_BF16 = 1 } pkv_dtype;
+
+/* Kernels reported by the launch profiler. */
+typedef enum {
+    PKV_KERNEL_DECODE_PARTITION = 0, /* block-table walk, gather, QK^T, online softmax, PV */
+    PKV_KERNEL_DECODE_REDUCE = 1,    /* split-K merge of the partitions of one (seq, head) */
+    PKV_KERNEL_APPEND = 2,
+    PKV_KERNEL_COPY_BLOCKS = 3,
+    PKV_KERNEL_KINDS = 4
+} pkv_kernel_kind;
+
+/*
+ * Block-aware decode attention ("How PagedAttention works", item 5): for
+ * every sequence s and query head h, out[s][h] = softmax(scale * q[s][h] .
+ * K_s^T) V_s where K_s, V_s are the first context_lens[s] tokens of the
+ * sequence gathered through block_tables (int32 [num_seqs][max_blocks_per_seq],
+ * row-major).  This form takes bf16 data, does not range-check table entries
+ * against the pool size (only against 0), partitions long contexts
+ * automatically, and uses a workspace the library allocates and keeps per
+ * device (grown with cudaMalloc when needed, so do not call it inside CUDA
+ * graph capture on a new size).  Returns PKV_OK or a pkv_status.
+ */
+PKV_API int paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                           int num_heads, int num_kv_heads, int head_dim, int block_size,
+                           int max_blocks_per_seq, float scale, void* stream);
+
+/*
+ * General form of paged_attention_decode.
+ *   num_blocks        pool size; table entries outside [0, num_blocks) are
+ *                     device faults (the block is skipped, error word set).
+ *   dtype             pkv_dtype of q, out and the pools.
+ *   partition_tokens  context tokens per CTA (split-K); 0 chooses 512.  Must
+ *                     be a multiple of block_size, at most 4096.  Sequences
+ *                     longer than this are split and merged by a second
+ *                     kernel; shorter ones are written in one pass.
+ *   workspace         device memory of at least
+ *                     paged_attention_workspace_size(num_seqs, num_heads,
+ *                     max_blocks_per_seq*block_size, head_dim, partition_tokens)
+ *                     bytes, 256-byte aligned, owned by the caller, not read
+ *                     before it is written; may be NULL when that size is 0.
+ *                     Two calls in flight at once must not share it.
+ */
+PKV_API int paged_attention_decode_ex(void* out, const void* q, const void* k_cache, const void* v_cache,
+                              const int32_t* block_tables, const int32_t* context_lens,
+                              int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                              int block_size, int max_blocks_per_seq, float scale, int num_blocks,
+                              int dtype, int partition_tokens, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/* Bytes of split-K workspace paged_attention_decode_ex needs; 0 when every
+ * sequence fits one partition. */
+PKV_API size_t paged_attention_workspace_size(int num_seqs, int num_heads, int max_context, int head_dim,
+                                      int partition_tokens);
+
+/*
+ * Append new tokens ("The problem: the KV cache is big and unpredictable":
+ * one new entry per token): for i < num_tokens with slot = slot_mapping[i]
+ * >= 0, k_cache[slot / bs][g][slot % bs][:] = k[i][g][:] and likewise for v,
+ * for every kv head g.  k and v are [num_tokens][num_kv_heads][head_dim];
+ * slot_mapping is int64 [num_tokens]; -1 means "skip".  The copy is bit-exact.
+ * Slots >= num_blocks*bs are device faults (not written).  Two tokens must not
+ * name the same slot.
+ */
+PKV_API int kv_cache_append(void* k_cache, void* v_cache, const void* k, const void* v,
+                    const int64_t* slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                    int block_size, int num_blocks, int dtype, void* stream);
+
+/*
+ * Copy-on-write block copy ("Sharing blocks between sequences": the writer's
+ * shared block is copied first, then its table is updated): for each pair i
+ * of src_dst_pairs (int64 [num_pairs][2] = (src, dst)), the whole physical
+ * block src -- every kv head and slot, keys and values -- is copied to dst.
+ * Destinations must be distinct and no destination may also be a source (the
+ * pairs are then independent and run in parallel).  Indices outside
+ * [0, num_blocks) are device faults (pair skipped).  The caller updates its
+ * block tables; the library never touches them.
+ */
+PKV_API int copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_pairs, int num_pairs,
+                int num_kv_heads, int head_dim, int block_size, int num_blocks, int dtype,
+                void* stream);
+
+/* Synchronise `stream`, then return in *code the current device's error word
+ * (PKV_OK, PKV_ERR_DEVICE_BOUNDS or PKV_ERR_TIMEOUT) and clear it. */
+PKV_API int pkv_get_device_error(void* stream, int* code);
+
+/* Static English text of a status code. */
+PKV_API const char* pkv_status_string(int status);
+
+/*
+ * Launch profiler.  When enabled, every kernel launch is bracketed by CUDA
+ * events recorded on its own stream.  pkv_profile_read() waits for the
+ * recorded launches of `kind` and returns their count and summed device time
+ * in milliseconds; pkv_profile_reset() forgets every record.
+ */
+PKV_API int pkv_profile_enable(int on);
+PKV_API int pkv_profile_read(int kind, long long* launches, double* total_ms);
+PKV_API int pkv_profile_reset(void);
+
+/* Kernels launched by this library in this process so far (all kinds). */
+PKV_API unsigned long long pkv_launch_count(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+PKV_API int pkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

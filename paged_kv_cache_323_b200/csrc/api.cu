@@ -1,0 +1,403 @@
+// api.cu -- the C ABI of libpagedkv.so (declared in include/pagedkv.h):
+// argument validation, status codes, launch selection, the library-owned
+// split-K workspace, the per-device error word and the launch profiler.
+// Every compute step runs in the kernels of decode_attn.cuh and kv_ops.cuh.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <climits>
+#include <mutex>
+#include <vector>
+
+#include "../../include/pagedkv.h"
+#include "kv_ops.cuh"
+#include "launch.h"
+
+// One error word per device (a __device__ variable exists once per device
+// context).  Kernels receive its device address; pkv_get_device_error reads
+// and clears it.
+__device__ int g_pkv_device_error;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kAutoPartitionTokens = 512;
+constexpr int kMaxPartitionTokens = 4096;
+
+struct DeviceState {
+    int* err = nullptr;     // device address of g_pkv_device_error
+    void* ws = nullptr;     // library-owned split-K workspace
+    size_t ws_bytes = 0;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+std::atomic<unsigned long long> g_launches{0};
+
+// ---------------------------------------------------------- profiler
+struct ProfRecord {
+    int kind;
+    int device;
+    cudaEvent_t start, stop;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRecord> g_prof;
+std::vector<std::pair<int, cudaEvent_t>> g_free_events;  // (device, event)
+
+cudaEvent_t take_event(int dev) {
+    for (size_t i = 0; i < g_free_events.size(); ++i) {
+        if (g_free_events[i].first == dev) {
+            cudaEvent_t e = g_free_events[i].second;
+            g_free_events[i] = g_free_events.back();
+            g_free_events.pop_back();
+            return e;
+        }
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+int current_device(int* dev) {
+    if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= kMaxDevices) return PKV_ERR_CUDA;
+    return PKV_OK;
+}
+
+int error_word(int dev, int** out) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_dev[dev].err == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_pkv_device_error) != cudaSuccess) return PKV_ERR_CUDA;
+        g_dev[dev].err = static_cast<int*>(p);
+    }
+    *out = g_dev[dev].err;
+    return PKV_OK;
+}
+
+// Launch one kernel through `fn`, counting it and (when profiling) bracketing
+// it with events on its own stream.
+template <class Fn>
+int launch(int kind, cudaStream_t st, Fn&& fn) {
+    cudaEvent_t a = nullptr, b = nullptr;
+    int dev = 0;
+    bool prof = false;
+    {
+        std::lock_guard<std::mutex> lk(g_prof_mu);
+        prof = g_prof_on;
+        if (prof) {
+            cudaGetDevice(&dev);
+            a = take_event(dev);
+            b = take_event(dev);
+            prof = a && b;
+        }
+    }
+    if (prof) cudaEventRecord(a, st);
+    cudaError_t e = fn();
+    if (e == cudaSuccess) e = cudaGetLastError();
+    g_launches.fetch_add(1);
+    if (prof) {
+        cudaEventRecord(b, st);
+        std::lock_guard<std::mutex> lk(g_prof_mu);
+        g_prof.push_back(ProfRecord{kind, dev, a, b});
+    }
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elt_bytes(int dtype) { return dtype == PKV_F32 ? 4 : 2; }
+
+bool decode_shape_supported(int head_dim, int block_size, int group) {
+    const bool d_ok = head_dim == 64 || head_dim == 128;
+    const bool bs_ok = block_size == 8 || block_size == 16 || block_size == 32;
+    const bool g_ok = group == 1 || group == 2 || group == 4 || group == 8;
+    return d_ok && bs_ok && g_ok;
+}
+
+int resolve_partition(int partition_tokens) {
+    return partition_tokens == 0 ? kAutoPartitionTokens : partition_tokens;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t workspace_bytes_for(long long num_seqs, long long num_heads, long long parts, long long D) {
+    if (parts <= 1) return 0;
+    const size_t o_bytes = align256(size_t(num_seqs) * num_heads * parts * D * sizeof(float));
+    return o_bytes + size_t(num_seqs) * num_heads * parts * sizeof(float2);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t paged_attention_workspace_size(int num_seqs, int num_heads, int max_context, int head_dim,
+                                      int partition_tokens) {
+    if (num_seqs <= 0 || num_heads <= 0 || max_context <= 0 || head_dim <= 0 ||
+        partition_tokens < 0)
+        return 0;
+    const long long pt = resolve_partition(partition_tokens);
+    const long long parts = (max_context + pt - 1) / pt;
+    return workspace_bytes_for(num_seqs, num_heads, parts, head_dim);
+}
+
+int paged_attention_decode_ex(void* out, const void* q, const void* k_cache, const void* v_cache,
+                              const int32_t* block_tables, const int32_t* context_lens,
+                              int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                              int block_size, int max_blocks_per_seq, float scale, int num_blocks,
+                              int dtype, int partition_tokens, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+    if (num_seqs < 0) return PKV_ERR_INVALID;
+    if (num_seqs == 0) return PKV_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PKV_ERR_NULL;
+    if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0) return PKV_ERR_INVALID;
+    if (head_dim <= 0 || block_size <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0)
+        return PKV_ERR_INVALID;
+    if (dtype != PKV_F32 && dtype != PKV_BF16) return PKV_ERR_INVALID;
+    if (!isfinite(scale)) return PKV_ERR_INVALID;
+    const int group = num_heads / num_kv_heads;
+    if (!decode_shape_supported(head_dim, block_size, group)) return PKV_ERR_UNSUPPORTED;
+    if (partition_tokens < 0 || partition_tokens > kMaxPartitionTokens ||
+        partition_tokens % block_size != 0)
+        return PKV_ERR_INVALID;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+        return PKV_ERR_INVALID;
+    const long long max_ctx = (long long)max_blocks_per_seq * block_size;
+    if (max_ctx > INT_MAX) return PKV_ERR_INVALID;
+    const int pt = resolve_partition(partition_tokens);
+    const long long parts = (max_ctx + pt - 1) / pt;
+    const long long grid = parts * num_kv_heads * (long long)num_seqs;
+    if (grid > INT_MAX || (long long)num_seqs * num_heads > INT_MAX) return PKV_ERR_INVALID;
+    const size_t need = workspace_bytes_for(num_seqs, num_heads, parts, head_dim);
+    if (need > 0) {
+        if (workspace == nullptr || workspace_bytes < need ||
+            (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+            return PKV_ERR_WORKSPACE;
+    }
+    int dev = 0;
+    if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
+    int* err = nullptr;
+    if (error_word(dev, &err) != PKV_OK) return PKV_ERR_CUDA;
+
+    pkv::DecodeParams p;
+    p.out = out;
+    p.q = q;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.ws_o = static_cast<float*>(workspace);
+    p.ws_ml = need > 0 ? reinterpret_cast<float2*>(static_cast<char*>(workspace) +
+                                                    align256(size_t(num_seqs) * num_heads * parts *
+                                                             head_dim * sizeof(float)))
+                       : nullptr;
+    p.err = err;
+    p.num_seqs = num_seqs;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_blocks = num_blocks;
+    p.partition_tokens = pt;
+    p.num_partitions = (int)parts;
+    p.qscale = scale * 1.4426950408889634f;  // log2(e): softmax runs in base 2
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int rc = launch(PKV_KERNEL_DECODE_PARTITION, st, [&] {
+        return dtype == PKV_F32 ? pkv::launch_decode_partition_f32(p, head_dim, block_size, group, grid, st)
+                                : pkv::launch_decode_partition_bf16(p, head_dim, block_size, group, grid, st);
+    });
+    if (rc != PKV_OK || parts <= 1) return rc;
+
+    pkv::ReduceParams r;
+    r.out = out;
+    r.ws_o = p.ws_o;
+    r.ws_ml = p.ws_ml;
+    r.context_lens = context_lens;
+    r.num_heads = num_heads;
+    r.max_ctx = (int)max_ctx;
+    r.partition_tokens = pt;
+    r.num_partitions = (int)parts;
+    const long long rgrid = (long long)num_seqs * num_heads;
+    return launch(PKV_KERNEL_DECODE_REDUCE, st, [&] {
+        return dtype == PKV_F32 ? pkv::launch_decode_reduce_f32(r, head_dim, rgrid, st)
+                                : pkv::launch_decode_reduce_bf16(r, head_dim, rgrid, st);
+    });
+}
+
+int paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                           int num_heads, int num_kv_heads, int head_dim, int block_size,
+                           int max_blocks_per_seq, float scale, void* stream) {
+    if (num_seqs < 0) return PKV_ERR_INVALID;
+    if (num_seqs == 0) return PKV_OK;
+    if (num_heads <= 0 || head_dim <= 0 || block_size <= 0 || max_blocks_per_seq <= 0)
+        return PKV_ERR_INVALID;
+    const long long max_ctx = (long long)max_blocks_per_seq * block_size;
+    if (max_ctx > INT_MAX) return PKV_ERR_INVALID;
+    const size_t need = paged_attention_workspace_size(num_seqs, num_heads, (int)max_ctx, head_dim, 0);
+    void* ws = nullptr;
+    if (need > 0) {
+        int dev = 0;
+        if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
+        std::lock_guard<std::mutex> lk(g_mu);
+        DeviceState& d = g_dev[dev];
+        if (d.ws_bytes < need) {
+            if (d.ws) cudaFree(d.ws);  // synchronises: no launch still reads the old buffer
+            d.ws = nullptr;
+            d.ws_bytes = 0;
+            if (cudaMalloc(&d.ws, need) != cudaSuccess) return PKV_ERR_CUDA;
+            d.ws_bytes = need;
+        }
+        ws = d.ws;
+    }
+    return paged_attention_decode_ex(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                                     num_heads, num_kv_heads, head_dim, block_size,
+                                     max_blocks_per_seq, scale, INT_MAX, PKV_BF16, 0, ws, need,
+                                     stream);
+}
+
+int kv_cache_append(void* k_cache, void* v_cache, const void* k, const void* v,
+                    const int64_t* slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                    int block_size, int num_blocks, int dtype, void* stream) {
+    if (num_tokens < 0) return PKV_ERR_INVALID;
+    if (num_tokens == 0) return PKV_OK;
+    if (!k_cache || !v_cache || !k || !v || !slot_mapping) return PKV_ERR_NULL;
+    if (num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+        return PKV_ERR_INVALID;
+    if (dtype != PKV_F32 && dtype != PKV_BF16) return PKV_ERR_INVALID;
+    const int row_bytes = head_dim * elt_bytes(dtype);
+    if (row_bytes % 16 != 0) return PKV_ERR_UNSUPPORTED;
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k) || !aligned16(v))
+        return PKV_ERR_INVALID;
+    int dev = 0;
+    if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
+    int* err = nullptr;
+    if (error_word(dev, &err) != PKV_OK) return PKV_ERR_CUDA;
+    pkv::AppendParams p;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.k = k;
+    p.v = v;
+    p.slot_mapping = slot_mapping;
+    p.err = err;
+    p.num_slots = (long long)num_blocks * block_size;
+    p.num_tokens = num_tokens;
+    p.num_kv_heads = num_kv_heads;
+    p.block_size = block_size;
+    p.chunks_per_row = row_bytes / 16;
+    const long long total = (long long)num_tokens * num_kv_heads * p.chunks_per_row;
+    long long blocks = (total + 255) / 256;
+    if (blocks > 148LL * 32) blocks = 148LL * 32;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return launch(PKV_KERNEL_APPEND, st, [&] {
+        pkv::kv_append_kernel<<<(unsigned)blocks, 256, 0, st>>>(p);
+        return cudaGetLastError();
+    });
+}
+
+int copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_pairs, int num_pairs,
+                int num_kv_heads, int head_dim, int block_size, int num_blocks, int dtype,
+                void* stream) {
+    if (num_pairs < 0) return PKV_ERR_INVALID;
+    if (num_pairs == 0) return PKV_OK;
+    if (!k_cache || !v_cache || !src_dst_pairs) return PKV_ERR_NULL;
+    if (num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+        return PKV_ERR_INVALID;
+    if (dtype != PKV_F32 && dtype != PKV_BF16) return PKV_ERR_INVALID;
+    const long long block_bytes = (long long)num_kv_heads * block_size * head_dim * elt_bytes(dtype);
+    if (block_bytes % 16 != 0) return PKV_ERR_UNSUPPORTED;
+    if (!aligned16(k_cache) || !aligned16(v_cache)) return PKV_ERR_INVALID;
+    int dev = 0;
+    if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
+    int* err = nullptr;
+    if (error_word(dev, &err) != PKV_OK) return PKV_ERR_CUDA;
+    pkv::CopyParams p;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.pairs = src_dst_pairs;
+    p.err = err;
+    p.chunks_per_block = block_bytes / 16;
+    p.num_pairs = num_pairs;
+    p.num_blocks = num_blocks;
+    long long per_pair = (p.chunks_per_block + 1023) / 1024;  // 256 threads x 4 chunks
+    if (per_pair > 64) per_pair = 64;
+    if (num_pairs > 65535) return PKV_ERR_INVALID;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return launch(PKV_KERNEL_COPY_BLOCKS, st, [&] {
+        pkv::copy_blocks_kernel<<<dim3((unsigned)per_pair, (unsigned)num_pairs), 256, 0, st>>>(p);
+        return cudaGetLastError();
+    });
+}
+
+int pkv_get_device_error(void* stream, int* code) {
+    if (!code) return PKV_ERR_NULL;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PKV_ERR_CUDA;
+    int dev = 0;
+    if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
+    int* err = nullptr;
+    if (error_word(dev, &err) != PKV_OK) return PKV_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, err, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return PKV_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpy(err, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return PKV_ERR_CUDA;
+    *code = v;
+    return PKV_OK;
+}
+
+const char* pkv_status_string(int status) {
+    switch (status) {
+        case PKV_OK: return "ok";
+        case PKV_ERR_NULL: return "a required pointer is NULL";
+        case PKV_ERR_INVALID: return "an argument is out of range";
+        case PKV_ERR_UNSUPPORTED: return "no kernel for this shape or type";
+        case PKV_ERR_CUDA: return "CUDA runtime error";
+        case PKV_ERR_WORKSPACE: return "split-K workspace missing or too small";
+        case PKV_ERR_DEVICE_BOUNDS: return "device: table entry, slot or context length out of range";
+        case PKV_ERR_TIMEOUT: return "device: a bounded wait ran out of time";
+        default: return "unknown status";
+    }
+}
+
+int pkv_profile_enable(int on) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_on = on != 0;
+    return PKV_OK;
+}
+
+int pkv_profile_read(int kind, long long* launches, double* total_ms) {
+    if (!launches || !total_ms) return PKV_ERR_NULL;
+    if (kind < 0 || kind >= PKV_KERNEL_KINDS) return PKV_ERR_INVALID;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    long long n = 0;
+    double ms = 0.0;
+    for (const ProfRecord& r : g_prof) {
+        if (r.kind != kind) continue;
+        if (cudaEventSynchronize(r.stop) != cudaSuccess) return PKV_ERR_CUDA;
+        float t = 0.f;
+        if (cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess) return PKV_ERR_CUDA;
+        ms += t;
+        ++n;
+    }
+    *launches = n;
+    *total_ms = ms;
+    return PKV_OK;
+}
+
+int pkv_profile_reset(void) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    for (const ProfRecord& r : g_prof) {
+        cudaEventSynchronize(r.stop);
+        g_free_events.emplace_back(r.device, r.start);
+        g_free_events.emplace_back(r.device, r.stop);
+    }
+    g_prof.clear();
+    return PKV_OK;
+}
+
+unsigned long long pkv_launch_count(void) { return g_launches.load(); }
+
+int pkv_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,202 @@
+"""Thin ctypes binding of libpagedkv.so (the C ABI in include/pagedkv.h).
+
+Argument marshalling only: each function takes torch tensors that already
+live on the GPU, reads their shapes and device pointers, and calls the C
+entry point of the same name on the current torch stream.  Every step of the
+decode path runs in the library's CUDA kernels; there is no fallback, and
+importing this module fails when the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpagedkv.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_323_b200.build` "
+        "(nvcc, sm_100a); the decode path has no other implementation")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+PKV_OK = 0
+PKV_ERR_NULL = -1
+PKV_ERR_INVALID = -2
+PKV_ERR_UNSUPPORTED = -3
+PKV_ERR_CUDA = -4
+PKV_ERR_WORKSPACE = -5
+PKV_ERR_DEVICE_BOUNDS = -6
+PKV_ERR_TIMEOUT = -7
+PKV_F32 = 0
+PKV_BF16 = 1
+KERNEL_DECODE_PARTITION = 0
+KERNEL_DECODE_REDUCE = 1
+KERNEL_APPEND = 2
+KERNEL_COPY_BLOCKS = 3
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+
+# name -> (restype, argtypes); the order mirrors include/pagedkv.h
+SIGNATURES = {
+    "paged_attention_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P]),
+    "paged_attention_decode_ex": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float,
+                                       _I, _I, _I, _P, _SZ, _P]),
+    "paged_attention_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "kv_cache_append": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
+    "copy_blocks": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
+    "pkv_get_device_error": (_I, [_P, ctypes.POINTER(_I)]),
+    "pkv_status_string": (ctypes.c_char_p, [_I]),
+    "pkv_profile_enable": (_I, [_I]),
+    "pkv_profile_read": (_I, [_I, ctypes.POINTER(ctypes.c_longlong), ctypes.POINTER(ctypes.c_double)]),
+    "pkv_profile_reset": (_I, []),
+    "pkv_launch_count": (ctypes.c_ulonglong, []),
+    "pkv_version": (_I, []),
+}
+for _name, (_res, _args) in SIGNATURES.items():
+    _fn = getattr(lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+class PagedKVError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+def status_string(status: int) -> str:
+    return lib.pkv_status_string(int(status)).decode()
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != PKV_OK:
+        raise PagedKVError(rc, where)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return PKV_F32
+    if t.dtype == torch.bfloat16:
+        return PKV_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def paged_attention_workspace_size(num_seqs: int, num_heads: int, max_context: int, head_dim: int,
+                                   partition_tokens: int = 0) -> int:
+    return int(lib.paged_attention_workspace_size(num_seqs, num_heads, max_context, head_dim,
+                                                  partition_tokens))
+
+
+def paged_attention_decode_ex(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                              *, num_blocks: int | None = None, partition_tokens: int = 0,
+                              workspace: torch.Tensor | None = None, stream=None) -> None:
+    """out, q: [B][H][D]; caches: [N][Hkv][bs][D]; block_tables int32 [B][maxb];
+    context_lens int32 [B].  ``workspace`` is a uint8 CUDA tensor of at least
+    :func:`paged_attention_workspace_size` bytes (allocated here when None)."""
+    B, H, D = q.shape
+    N, Hkv, bs, D2 = k_cache.shape
+    if D2 != D or tuple(out.shape) != (B, H, D) or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("shape mismatch between q, out and the caches")
+    maxb = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    if num_blocks is None:
+        num_blocks = N
+    need = paged_attention_workspace_size(B, H, maxb * bs, D, partition_tokens)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    code = _dtype_code(q)
+    rc = lib.paged_attention_decode_ex(
+        _dev(out, "out", q.dtype), _dev(q, "q"), _dev(k_cache, "k_cache", q.dtype),
+        _dev(v_cache, "v_cache", q.dtype), _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32), B, H, Hkv, D, bs, maxb, float(scale),
+        int(num_blocks), code, int(partition_tokens), ws_ptr, ws_bytes, _stream(stream))
+    _check(rc, "paged_attention_decode_ex")
+
+
+def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                           stream=None) -> None:
+    """bf16 form with the library-owned workspace (see include/pagedkv.h)."""
+    B, H, D = q.shape
+    N, Hkv, bs, _ = k_cache.shape
+    rc = lib.paged_attention_decode(
+        _dev(out, "out", torch.bfloat16), _dev(q, "q", torch.bfloat16),
+        _dev(k_cache, "k_cache", torch.bfloat16), _dev(v_cache, "v_cache", torch.bfloat16),
+        _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32), B, H, Hkv, D, bs, block_tables.shape[1],
+        float(scale), _stream(stream))
+    _check(rc, "paged_attention_decode")
+
+
+def kv_cache_append(k_cache, v_cache, k, v, slot_mapping, stream=None) -> None:
+    """k, v: [T][Hkv][D]; slot_mapping int64 [T] (-1 = skip)."""
+    T = slot_mapping.shape[0]
+    N, Hkv, bs, D = k_cache.shape
+    if T and (tuple(k.shape) != (T, Hkv, D) or tuple(v.shape) != (T, Hkv, D)):
+        raise ValueError("k / v must be [num_tokens][num_kv_heads][head_dim]")
+    rc = lib.kv_cache_append(
+        _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache", k_cache.dtype),
+        _dev(k, "k", k_cache.dtype) if T else None, _dev(v, "v", k_cache.dtype) if T else None,
+        _dev(slot_mapping, "slot_mapping", torch.int64) if T else None, T, Hkv, D, bs, N,
+        _dtype_code(k_cache), _stream(stream))
+    _check(rc, "kv_cache_append")
+
+
+def copy_blocks(k_cache, v_cache, src_dst_pairs, stream=None) -> None:
+    """src_dst_pairs: int64 [n][2] of (src, dst) physical blocks."""
+    n = src_dst_pairs.shape[0]
+    N, Hkv, bs, D = k_cache.shape
+    rc = lib.copy_blocks(
+        _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache", k_cache.dtype),
+        _dev(src_dst_pairs, "src_dst_pairs", torch.int64) if n else None, n, Hkv, D, bs, N,
+        _dtype_code(k_cache), _stream(stream))
+    _check(rc, "copy_blocks")
+
+
+def get_device_error(stream=None) -> int:
+    code = ctypes.c_int(0)
+    _check(lib.pkv_get_device_error(_stream(stream), ctypes.byref(code)), "pkv_get_device_error")
+    return code.value
+
+
+def profile_enable(on: bool = True) -> None:
+    _check(lib.pkv_profile_enable(1 if on else 0), "pkv_profile_enable")
+
+
+def profile_read(kind: int) -> tuple[int, float]:
+    n = ctypes.c_longlong(0)
+    ms = ctypes.c_double(0.0)
+    _check(lib.pkv_profile_read(kind, ctypes.byref(n), ctypes.byref(ms)), "pkv_profile_read")
+    return n.value, ms.value
+
+
+def profile_reset() -> None:
+    _check(lib.pkv_profile_reset(), "pkv_profile_reset")
+
+
+def launch_count() -> int:
+    return int(lib.pkv_launch_count())

@@ -52,6 +52,8 @@ class Workload:
     block_tables: np.ndarray  # int32 [B][max_blocks_per_seq], -1 where unallocated
     cow_pairs: np.ndarray  # int64 [n][2] (src, dst)
     slot_mapping: np.ndarray  # int64 [T]
+    token_seq: np.ndarray  # int32 [T]: the sequence each new token belongs to
+    pair_seq: np.ndarray  # int32 [n]: the writer each copy-on-write pair serves
     q: torch.Tensor  # [B][H][D]
     k_cache: torch.Tensor  # [N][Hkv][bs][D], state BEFORE the step
     v_cache: torch.Tensor
@@ -100,13 +102,14 @@ def _normal(shape, rng: np.random.Generator, tgen, device, dtype: str, mult: flo
 
 
 def _finish(name, dtype, rng, seed, device, *, lens, tables, cow_pairs, new_pos, num_blocks,
-            H, Hkv, D, bs, maxb, q_mult=1.0, meta=None) -> Workload:
+            H, Hkv, D, bs, maxb, q_mult=1.0, meta=None, pair_seq=()) -> Workload:
     """Shared tail of every generator: slots of the new tokens, then tensors."""
     B = len(lens)
-    slots = []
+    slots, owners = [], []
     for s, positions in enumerate(new_pos):
         for t in positions:
             slots.append(int(tables[s][t // bs]) * bs + t % bs)
+            owners.append(s)
     slot_mapping = np.asarray(slots, dtype=np.int64)
     tgen = None
     if device not in (None, "cpu"):
@@ -126,7 +129,8 @@ def _finish(name, dtype, rng, seed, device, *, lens, tables, cow_pairs, new_pos,
         block_size=bs, num_blocks=num_blocks, max_blocks_per_seq=maxb,
         scale=float(np.float32(1.0 / math.sqrt(D))), context_lens=np.asarray(lens, dtype=np.int32),
         block_tables=bt, cow_pairs=np.asarray(cow_pairs, dtype=np.int64).reshape(-1, 2),
-        slot_mapping=slot_mapping, q=q, k_cache=k_cache, v_cache=v_cache, k_new=k_new,
+        slot_mapping=slot_mapping, token_seq=np.asarray(owners, dtype=np.int32),
+        pair_seq=np.asarray(pair_seq, dtype=np.int32), q=q, k_cache=k_cache, v_cache=v_cache, k_new=k_new,
         v_new=v_new, meta=meta or {})
 
 
@@ -186,7 +190,7 @@ def gqa_sampling(seed: int = 3, device="cpu", groups: int = 64, samples: int = 4
         need += sum(-(-int(P + g) // bs) - -(-int(P) // bs) for g in gs)
     num_blocks = int(math.ceil(need * (1.0 + slack)))
     pool = _Pool(rng, num_blocks)
-    tables, new_pos, lens, cow = [], [], [], []
+    tables, new_pos, lens, cow, cow_seq = [], [], [], [], []
     for P, gs in zip(prompts, gens):
         P = int(P)
         shared = [pool.take() for _ in range(-(-P // bs))]
@@ -201,6 +205,7 @@ def gqa_sampling(seed: int = 3, device="cpu", groups: int = 64, samples: int = 4
                 dst = pool.take()
                 pool.ref[src] -= 1
                 cow.append((src, dst))
+                cow_seq.append(len(tables))
                 table[first] = dst
             while len(table) < -(-L // bs):
                 table.append(pool.take())
@@ -210,7 +215,7 @@ def gqa_sampling(seed: int = 3, device="cpu", groups: int = 64, samples: int = 4
     maxb = max(len(t) for t in tables)
     return _finish("gqa_sampling", dtype, rng, seed, device, lens=lens, tables=tables,
                    cow_pairs=cow, new_pos=new_pos, num_blocks=num_blocks, H=heads, Hkv=kv_heads,
-                   D=head_dim, bs=bs, maxb=maxb,
+                   D=head_dim, bs=bs, maxb=maxb, pair_seq=cow_seq,
                    meta={"prompts": prompts.tolist(), "gens": gens.tolist(), "samples": samples})
 
 
