@@ -17,12 +17,9 @@ from __future__ import annotations
 
 import argparse
 import json
-import math
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 import numpy as np
@@ -50,9 +47,12 @@ WORKLOADS = {
     "prefix_bs32": ("prefix_sweep_b1024_prefix2048_h32_kv8_d128_bs32_bf16",
                     lambda dev, seed: wl.prefix_sweep(32, seed=seed, device=dev)),
     "tiny": ("tiny_b4_ctx35-16-1-50_h4_d64_bs16_f32", lambda dev, seed: wl.tiny(seed=seed, device=dev)),
+    # a smaller MHA batch for profiler captures: 16 sequences, 4096-block pool (1 GB), ~0.3 GB KV per step
+    "mha_small": ("mha_decode_b16_h32_kv32_d128_bs16_ctxU128-2048_bf16_pool4096",
+                  lambda dev, seed: wl.mha(seed=seed, device=dev, num_seqs=16, num_blocks=4096)),
 }
 DEFAULT_SEED = {"mha": 2, "gqa_sampling": 3, "long_context": 4, "prefix_bs8": 5, "prefix_bs16": 5,
-                "prefix_bs32": 5, "tiny": 1}
+                "prefix_bs32": 5, "tiny": 1, "mha_small": 2}
 
 
 def measured_peak():
@@ -98,50 +98,71 @@ def kernel_source_sha() -> str:
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    """SM clocks and clock-event (throttle) reasons of this process's GPU,
+    sampled by NVML (read-only queries) every ~2 ms in a background thread
+    while the timed region runs."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.path = None
+    def __init__(self, device: int):
+        self.device = device
+        self.samples = []
+        self.max_mhz = None
+        self._stop = None
+        self._thread = None
+        self._nvml = None
 
     def start(self):
+        import threading
+
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            import pynvml as nv
+
+            nv.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(self.device).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self._h = nv.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self._h, nv.NVML_CLOCK_SM)
+            self._nvml = nv
+        except Exception as e:  # no NVML: report no clocks rather than guess
+            self._err = repr(e)
+            return
+        self._stop = threading.Event()
+
+        def loop():
+            nv = self._nvml
+            while not self._stop.is_set():
+                try:
+                    mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                    self.samples.append((mhz, rs))
+                except Exception:
+                    pass
+                self._stop.wait(0.002)
+
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
+        if self._nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                    "note": "NVML unavailable: " + getattr(self, "_err", "")}
+        self._stop.set()
+        self._thread.join()
+        nv = self._nvml
+        mhz = [m for m, _ in self.samples]
+        reasons = sorted({name for _, rs in self.samples for name, attr in self.REASONS
+                          if rs & getattr(nv, attr, 0)})
         try:
-            self.proc.wait(timeout=5)
+            nv.nvmlShutdown()
         except Exception:
-            self.proc.kill()
-        rows = []
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) >= 9:
-                rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+            pass
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(mhz)}
 
 
 def dist_setup(n_gpus: int):
@@ -312,9 +333,7 @@ def run_gpu(args, world, rank, local):
         raise RuntimeError(f"device error word {code} after warm-up")
 
     # ------------------------------------------------ device-resident timing
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
-    phys = vis.split(",")[local] if vis and len(vis.split(",")) > local else str(local)
-    clocks = ClockSampler(int(phys) if phys.isdigit() else local)
+    clocks = ClockSampler(torch.cuda.current_device())
     pk.profile_reset()
     pk.profile_enable(True)
     barrier(world)
@@ -422,8 +441,8 @@ def run_gpu(args, world, rank, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="pagedkv", choices=["pagedkv", "reference"])
     ap.add_argument("--workload", default="mha", choices=sorted(WORKLOADS))
     ap.add_argument("--partition-tokens", type=int, default=0)
