@@ -78,11 +78,10 @@ typedef enum { PKV_F32 = 0, PKV_BF16 = 1 } pkv_dtype;
 
 /* Kernels reported by the launch profiler. */
 typedef enum {
-    PKV_KERNEL_DECODE_PARTITION = 0, /* block-table walk, gather, QK^T, online softmax, PV */
-    PKV_KERNEL_DECODE_REDUCE = 1,    /* split-K merge of the partitions of one (seq, head) */
-    PKV_KERNEL_APPEND = 2,
-    PKV_KERNEL_COPY_BLOCKS = 3,
-    PKV_KERNEL_KINDS = 4
+    PKV_KERNEL_DECODE = 0, /* table walk, gather, QK^T, online softmax, PV, fused split-K merge */
+    PKV_KERNEL_APPEND = 1,
+    PKV_KERNEL_COPY_BLOCKS = 2,
+    PKV_KERNEL_KINDS = 3
 } pkv_kernel_kind;
 
 /*
@@ -106,16 +105,23 @@ PKV_API int paged_attention_decode(void* out, const void* q, const void* k_cache
  *   num_blocks        pool size; table entries outside [0, num_blocks) are
  *                     device faults (the block is skipped, error word set).
  *   dtype             pkv_dtype of q, out and the pools.
- *   partition_tokens  context tokens per CTA (split-K); 0 chooses 512.  Must
- *                     be a multiple of block_size, at most 4096.  Sequences
- *                     longer than this are split and merged by a second
- *                     kernel; shorter ones are written in one pass.
+ *   partition_tokens  context tokens per CTA (split-K); a multiple of
+ *                     block_size, at most 4096, or 0 for automatic (512,
+ *                     doubled for very long tables while the grid stays
+ *                     large).  A sequence longer than one partition is split;
+ *                     the last of its partitions to finish merges them all in
+ *                     partition order, inside the same kernel.  Shorter ones
+ *                     are written in one pass.
  *   workspace         device memory of at least
  *                     paged_attention_workspace_size(num_seqs, num_heads,
  *                     max_blocks_per_seq*block_size, head_dim, partition_tokens)
- *                     bytes, 256-byte aligned, owned by the caller, not read
- *                     before it is written; may be NULL when that size is 0.
- *                     Two calls in flight at once must not share it.
+ *                     bytes, 256-byte aligned, owned by the caller; may be
+ *                     NULL when that size is 0.  It holds the partial results
+ *                     and one merge counter per (sequence, kv head): it must
+ *                     be zero-filled (e.g. cudaMemset) before its first use,
+ *                     and every completed call leaves the counters at zero
+ *                     again, so it can be reused without clearing.  Two calls
+ *                     in flight at once must not share it.
  */
 PKV_API int paged_attention_decode_ex(void* out, const void* q, const void* k_cache, const void* v_cache,
                               const int32_t* block_tables, const int32_t* context_lens,

@@ -117,16 +117,40 @@ bool decode_shape_supported(int head_dim, int block_size, int group) {
     return d_ok && bs_ok && g_ok;
 }
 
-int resolve_partition(int partition_tokens) {
-    return partition_tokens == 0 ? kAutoPartitionTokens : partition_tokens;
-}
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Split-K workspace: [B][H][P][D] fp32 partial outputs, [B][H][P] (m, l)
+// pairs, then one int counter per (sequence, head) slot (used per kv head).
+struct WorkspaceLayout {
+    size_t o_off, ml_off, cnt_off, total;
+};
+
+WorkspaceLayout workspace_layout(long long num_seqs, long long num_heads, long long parts, long long D) {
+    WorkspaceLayout w{0, 0, 0, 0};
+    if (parts <= 1) return w;
+    w.o_off = 0;
+    w.ml_off = align256(size_t(num_seqs) * num_heads * parts * D * sizeof(float));
+    w.cnt_off = w.ml_off + align256(size_t(num_seqs) * num_heads * parts * sizeof(float2));
+    w.total = w.cnt_off + align256(size_t(num_seqs) * num_heads * sizeof(int));
+    return w;
+}
+
 size_t workspace_bytes_for(long long num_seqs, long long num_heads, long long parts, long long D) {
-    if (parts <= 1) return 0;
-    const size_t o_bytes = align256(size_t(num_seqs) * num_heads * parts * D * sizeof(float));
-    return o_bytes + size_t(num_seqs) * num_heads * parts * sizeof(float2);
+    return workspace_layout(num_seqs, num_heads, parts, D).total;
+}
+
+// Partition size when the caller passes 0: 512 tokens, doubled (up to 4096)
+// while a sequence of the maximum length would still be split into more than
+// 64 partitions and the grid keeps at least four waves of 3 CTAs per SM.  Long
+// contexts then merge fewer partials in the fused split-K merge.
+int auto_partition_tokens(long long num_seqs, long long num_kv_heads, long long max_ctx) {
+    long long pt = kAutoPartitionTokens;
+    const long long min_ctas = 4LL * 148 * 3;
+    while (pt < kMaxPartitionTokens && (max_ctx + pt - 1) / pt > 64 &&
+           num_seqs * num_kv_heads * ((max_ctx + 2 * pt - 1) / (2 * pt)) >= min_ctas)
+        pt *= 2;
+    return (int)pt;
 }
 
 }  // namespace
@@ -138,7 +162,8 @@ size_t paged_attention_workspace_size(int num_seqs, int num_heads, int max_conte
     if (num_seqs <= 0 || num_heads <= 0 || max_context <= 0 || head_dim <= 0 ||
         partition_tokens < 0)
         return 0;
-    const long long pt = resolve_partition(partition_tokens);
+    // the automatic size is never below 512 tokens, so 512 bounds its workspace
+    const long long pt = partition_tokens == 0 ? kAutoPartitionTokens : partition_tokens;
     const long long parts = (max_context + pt - 1) / pt;
     return workspace_bytes_for(num_seqs, num_heads, parts, head_dim);
 }
@@ -166,7 +191,8 @@ int paged_attention_decode_ex(void* out, const void* q, const void* k_cache, con
         return PKV_ERR_INVALID;
     const long long max_ctx = (long long)max_blocks_per_seq * block_size;
     if (max_ctx > INT_MAX) return PKV_ERR_INVALID;
-    const int pt = resolve_partition(partition_tokens);
+    const int pt = partition_tokens == 0 ? auto_partition_tokens(num_seqs, num_kv_heads, max_ctx)
+                                         : partition_tokens;
     const long long parts = (max_ctx + pt - 1) / pt;
     const long long grid = parts * num_kv_heads * (long long)num_seqs;
     if (grid > INT_MAX || (long long)num_seqs * num_heads > INT_MAX) return PKV_ERR_INVALID;
@@ -188,11 +214,11 @@ int paged_attention_decode_ex(void* out, const void* q, const void* k_cache, con
     p.v_cache = v_cache;
     p.block_tables = block_tables;
     p.context_lens = context_lens;
-    p.ws_o = static_cast<float*>(workspace);
-    p.ws_ml = need > 0 ? reinterpret_cast<float2*>(static_cast<char*>(workspace) +
-                                                    align256(size_t(num_seqs) * num_heads * parts *
-                                                             head_dim * sizeof(float)))
-                       : nullptr;
+    const WorkspaceLayout wl = workspace_layout(num_seqs, num_heads, parts, head_dim);
+    char* wsb = static_cast<char*>(workspace);
+    p.ws_o = need > 0 ? reinterpret_cast<float*>(wsb + wl.o_off) : nullptr;
+    p.ws_ml = need > 0 ? reinterpret_cast<float2*>(wsb + wl.ml_off) : nullptr;
+    p.counters = need > 0 ? reinterpret_cast<int*>(wsb + wl.cnt_off) : nullptr;
     p.err = err;
     p.num_seqs = num_seqs;
     p.num_heads = num_heads;
@@ -204,25 +230,9 @@ int paged_attention_decode_ex(void* out, const void* q, const void* k_cache, con
     p.qscale = scale * 1.4426950408889634f;  // log2(e): softmax runs in base 2
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    int rc = launch(PKV_KERNEL_DECODE_PARTITION, st, [&] {
+    return launch(PKV_KERNEL_DECODE, st, [&] {
         return dtype == PKV_F32 ? pkv::launch_decode_partition_f32(p, head_dim, block_size, group, grid, st)
                                 : pkv::launch_decode_partition_bf16(p, head_dim, block_size, group, grid, st);
-    });
-    if (rc != PKV_OK || parts <= 1) return rc;
-
-    pkv::ReduceParams r;
-    r.out = out;
-    r.ws_o = p.ws_o;
-    r.ws_ml = p.ws_ml;
-    r.context_lens = context_lens;
-    r.num_heads = num_heads;
-    r.max_ctx = (int)max_ctx;
-    r.partition_tokens = pt;
-    r.num_partitions = (int)parts;
-    const long long rgrid = (long long)num_seqs * num_heads;
-    return launch(PKV_KERNEL_DECODE_REDUCE, st, [&] {
-        return dtype == PKV_F32 ? pkv::launch_decode_reduce_f32(r, head_dim, rgrid, st)
-                                : pkv::launch_decode_reduce_bf16(r, head_dim, rgrid, st);
     });
 }
 
@@ -248,6 +258,7 @@ int paged_attention_decode(void* out, const void* q, const void* k_cache, const 
             d.ws = nullptr;
             d.ws_bytes = 0;
             if (cudaMalloc(&d.ws, need) != cudaSuccess) return PKV_ERR_CUDA;
+            if (cudaMemset(d.ws, 0, need) != cudaSuccess) return PKV_ERR_CUDA;  // merge counters start at 0
             d.ws_bytes = need;
         }
         ws = d.ws;
@@ -268,7 +279,7 @@ int kv_cache_append(void* k_cache, void* v_cache, const void* k, const void* v,
         return PKV_ERR_INVALID;
     if (dtype != PKV_F32 && dtype != PKV_BF16) return PKV_ERR_INVALID;
     const int row_bytes = head_dim * elt_bytes(dtype);
-    if (row_bytes % 16 != 0) return PKV_ERR_UNSUPPORTED;
+    if (row_bytes % 16 != 0 || row_bytes > 256 * 16) return PKV_ERR_UNSUPPORTED;
     if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k) || !aligned16(v))
         return PKV_ERR_INVALID;
     int dev = 0;
@@ -287,9 +298,10 @@ int kv_cache_append(void* k_cache, void* v_cache, const void* k, const void* v,
     p.num_kv_heads = num_kv_heads;
     p.block_size = block_size;
     p.chunks_per_row = row_bytes / 16;
-    const long long total = (long long)num_tokens * num_kv_heads * p.chunks_per_row;
-    long long blocks = (total + 255) / 256;
-    if (blocks > 148LL * 32) blocks = 148LL * 32;
+    const long long rows = (long long)num_tokens * num_kv_heads;
+    const long long rows_per_cta = 256 / p.chunks_per_row;
+    long long blocks = (rows + rows_per_cta - 1) / rows_per_cta;
+    if (blocks > 148LL * 16) blocks = 148LL * 16;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return launch(PKV_KERNEL_APPEND, st, [&] {
         pkv::kv_append_kernel<<<(unsigned)blocks, 256, 0, st>>>(p);

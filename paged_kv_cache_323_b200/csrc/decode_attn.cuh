@@ -30,10 +30,13 @@
 //    fp32 running max / sum, then PV into fp32 registers.
 //  * Warps merge their (m, l, o) states through shared memory; a sequence
 //    that fits one partition is normalised and written directly, otherwise
-//    the partition's (m, l, o) go to the workspace and the reduce kernel
-//    merges them in partition order.  No atomics: the arithmetic order
-//    depends only on logical token positions, so outputs are bit-identical
-//    under any physical placement of the blocks.
+//    the partition's (m, l, o) go to the workspace and the last partition CTA
+//    of the (sequence, kv head) to finish -- found with one atomicInc on a
+//    per-group counter that wraps back to zero -- merges all of them in
+//    partition order.  Which CTA merges never changes the arithmetic order,
+//    which depends only on logical token positions, so outputs are
+//    bit-identical under any physical placement of the blocks and across
+//    runs.
 //  * Faults never trap: a bad table entry or context length sets the device
 //    error word and is skipped or zero-filled; every mbarrier wait is bounded.
 #pragma once
@@ -53,6 +56,7 @@ struct DecodeParams {
     const int32_t* context_lens;
     float* ws_o;    // [B][H][P][D] unnormalised partial outputs
     float2* ws_ml;  // [B][H][P] (running max in log2 units, running sum)
+    int* counters;  // [B][Hkv] partitions finished, zero between launches
     int* err;
     int num_seqs;
     int num_heads;
@@ -94,12 +98,16 @@ struct DecodeCfg {
     static constexpr int PSCR_OFF = PHYS_OFF + MAX_PART_BLOCKS * 4;
     static constexpr int FLAG_OFF = PSCR_OFF + PSCR_FLOATS * 4;
     static constexpr int SMEM_BYTES = FLAG_OFF + 16;
+    // fused merge scratch after the merge area: [G][2] + [groups][G*D/4] float4
+    static constexpr int MERGE_SCRATCH_BYTES =
+        (MERGE_FLOATS + 2 * G + 4) * 4 + THREADS * 16 + (G * D / 4) * 16;
 
     static_assert(D % EPC == 0 && CPR <= 32 && 32 % CPR == 0, "head_dim chunking");
     static_assert(TR % RPI == 0 && RPL >= 1, "rows per lane");
     static_assert(NST % NBL == 0, "a stage always feeds the same block lane");
     static_assert(GW <= CPR, "a lane's logits after the butterfly belong to one head");
     static_assert(MERGE_FLOATS * 4 <= STAGES_BYTES, "merge area reuses the stages");
+    static_assert(MERGE_SCRATCH_BYTES <= STAGES_BYTES, "fused merge scratch reuses the stages");
     static_assert(SLICE % 16 == 0, "bulk copies move multiples of 16 bytes");
 };
 
@@ -416,24 +424,24 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, BS, G>::THREADS, 2)
     __syncthreads();
 
     const int H = p.num_heads;
-    const float* mrg_c = mrg;
+    const long long sh0 = (long long)s * H + (long long)g * G;  // first query head of the group
     for (int t = tid; t < G * D; t += blockDim.x) {
         const int hg = t / D;
         const int d = t % D;
         float M = -INFINITY;
 #pragma unroll
-        for (int b = 0; b < C::NBL; ++b) M = fmaxf(M, mrg_c[(b * G + hg) * (D + 2) + D]);
+        for (int b = 0; b < C::NBL; ++b) M = fmaxf(M, mrg[(b * G + hg) * (D + 2) + D]);
         float L = 0.f, O = 0.f;
         if (M != -INFINITY) {
 #pragma unroll
             for (int b = 0; b < C::NBL; ++b) {
-                const float* row = mrg_c + (b * G + hg) * (D + 2);
+                const float* row = mrg + (b * G + hg) * (D + 2);
                 const float w = exp2f(row[D] - M);
                 L = fmaf(w, row[D + 1], L);
                 O = fmaf(w, row[d], O);
             }
         }
-        const long long sh = (long long)s * H + (long long)g * G + hg;
+        const long long sh = sh0 + hg;
         if (nparts == 1) {
             Elem<T>::store(static_cast<T*>(p.out) + sh * D + d, L > 0.f ? O / L : 0.f);
         } else {
@@ -441,86 +449,89 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, BS, G>::THREADS, 2)
             if (d == 0) p.ws_ml[sh * P + part] = make_float2(M, L);
         }
     }
-}
+    if (nparts == 1) return;
 
-// Split-K merge for one (sequence, query head) per CTA of 128 threads:
-//     M = max_i m_i,  L = sum_i 2^(m_i - M) l_i,  out = sum_i 2^(m_i - M) o_i / L
-// in partition order (deterministic).  Sequences that fit one partition were
-// written by the partition kernel and are skipped.
-struct ReduceParams {
-    void* out;
-    const float* ws_o;
-    const float2* ws_ml;
-    const int32_t* context_lens;
-    int num_heads;
-    int max_ctx;
-    int partition_tokens;
-    int num_partitions;
-};
-
-template <typename T, int D>
-__global__ void __launch_bounds__(128) decode_reduce_kernel(const ReduceParams p) {
-    constexpr int COLS = D / 4;          // float4 columns of one partial row
-    constexpr int GROUPS = 128 / COLS;   // partitions processed side by side
-    __shared__ float red[4];
-    __shared__ float4 part_acc[GROUPS][COLS];
-
-    const long long u = blockIdx.x;
-    const int s = (int)(u / p.num_heads);
-    const int ctx = p.context_lens[s];
-    if (ctx < 0 || ctx > p.max_ctx) return;
-    const int nparts = (ctx + p.partition_tokens - 1) / p.partition_tokens;
-    if (nparts <= 1) return;
-    const float2* ml = p.ws_ml + u * p.num_partitions;
-    const float* o = p.ws_o + u * p.num_partitions * D;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
-    float M = -INFINITY;
-    for (int i = tid; i < nparts; i += 128) M = fmaxf(M, ml[i].x);
-#pragma unroll
-    for (int msk = 16; msk; msk >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, msk));
-    if (lane == 0) red[warp] = M;
+    // ---- split-K merge, fused: the last partition CTA of (s, g) to finish
+    // merges every partition of the group's heads.  atomicInc wraps the
+    // counter back to 0 on that last arrival, so the counters are zero again
+    // after every complete launch.
+    int* last_flag = reinterpret_cast<int*>(smem + C::FLAG_OFF) + 1;
+    __threadfence();
     __syncthreads();
-    M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-    __syncthreads();
-    float L = 0.f;
-    if (M != -INFINITY) {
-        for (int i = tid; i < nparts; i += 128) L = fmaf(exp2f(ml[i].x - M), ml[i].y, L);
+    if (tid == 0) {
+        const unsigned old = atomicInc(reinterpret_cast<unsigned*>(p.counters) + (long long)s * Hkv + g,
+                                       (unsigned)(nparts - 1));
+        *last_flag = old == (unsigned)(nparts - 1);
     }
-#pragma unroll
-    for (int msk = 16; msk; msk >>= 1) L += __shfl_xor_sync(0xffffffffu, L, msk);
-    if (lane == 0) red[warp] = L;
     __syncthreads();
-    L = (red[0] + red[1]) + (red[2] + red[3]);
+    if (!*last_flag) return;
+    __threadfence();
 
-    const int col = tid % COLS;
-    const int grp = tid / COLS;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (M != -INFINITY) {
-#pragma unroll 4
-        for (int i = grp; i < nparts; i += GROUPS) {
-            const float w = exp2f(ml[i].x - M);
-            const float4 v = reinterpret_cast<const float4*>(o + (long long)i * D)[col];
-            acc.x = fmaf(w, v.x, acc.x);
-            acc.y = fmaf(w, v.y, acc.y);
-            acc.z = fmaf(w, v.z, acc.z);
-            acc.w = fmaf(w, v.w, acc.w);
+    // per head: M = max_i m_i, L = sum_i 2^(m_i - M) l_i (one warp per head)
+    float* red = reinterpret_cast<float*>(smem) + C::MERGE_FLOATS;  // [G][2], then [threads][4]
+    for (int hg = warp; hg < G; hg += C::NCW + 1) {
+        const float2* ml = p.ws_ml + (sh0 + hg) * P;
+        float M = -INFINITY;
+        for (int i = lane; i < nparts; i += 32) M = fmaxf(M, __ldcg(&ml[i]).x);
+#pragma unroll
+        for (int msk = 16; msk; msk >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, msk));
+        float L = 0.f;
+        if (M != -INFINITY) {
+            for (int i = lane; i < nparts; i += 32) {
+                const float2 v = __ldcg(&ml[i]);
+                L = fmaf(exp2f(v.x - M), v.y, L);
+            }
+        }
+#pragma unroll
+        for (int msk = 16; msk; msk >>= 1) L += __shfl_xor_sync(0xffffffffu, L, msk);
+        if (lane == 0) {
+            red[2 * hg] = M;
+            red[2 * hg + 1] = L;
         }
     }
-    part_acc[grp][col] = acc;
     __syncthreads();
-    if (tid < COLS) {
-        float4 t = part_acc[0][tid];
-#pragma unroll
-        for (int gidx = 1; gidx < GROUPS; ++gidx) {
-            const float4 v = part_acc[gidx][tid];
+    // out = sum_i 2^(m_i - M) o_i / L, partitions split over thread groups
+    constexpr int COLS = D / 4;
+    constexpr int UNITS = G * COLS;
+    constexpr int GROUPS = C::THREADS / UNITS > 0 ? C::THREADS / UNITS : 1;
+    float4* acc_s = reinterpret_cast<float4*>(red + ((2 * G + 3) / 4) * 4);  // [GROUPS][UNITS]
+    for (int u = tid; u < GROUPS * UNITS; u += blockDim.x) {
+        const int unit = u % UNITS;
+        const int grp = u / UNITS;
+        const int hg = unit / COLS;
+        const int col = unit % COLS;
+        const float M = red[2 * hg];
+        const float2* ml = p.ws_ml + (sh0 + hg) * P;
+        const float4* o = reinterpret_cast<const float4*>(p.ws_o + (sh0 + hg) * P * D) + col;
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (M != -INFINITY) {
+#pragma unroll 4
+            for (int i = grp; i < nparts; i += GROUPS) {
+                const float w = exp2f(__ldcg(&ml[i]).x - M);
+                const float4 v = __ldcg(o + (long long)i * COLS);
+                a.x = fmaf(w, v.x, a.x);
+                a.y = fmaf(w, v.y, a.y);
+                a.z = fmaf(w, v.z, a.z);
+                a.w = fmaf(w, v.w, a.w);
+            }
+        }
+        acc_s[grp * UNITS + unit] = a;
+    }
+    __syncthreads();
+    for (int unit = tid; unit < UNITS; unit += blockDim.x) {
+        const int hg = unit / COLS;
+        const int col = unit % COLS;
+        float4 t = acc_s[unit];
+        for (int grp = 1; grp < GROUPS; ++grp) {
+            const float4 v = acc_s[grp * UNITS + unit];
             t.x += v.x;
             t.y += v.y;
             t.z += v.z;
             t.w += v.w;
         }
+        const float L = red[2 * hg + 1];
         const float inv = L > 0.f ? 1.f / L : 0.f;
-        T* dst = static_cast<T*>(p.out) + u * D + tid * 4;
+        T* dst = static_cast<T*>(p.out) + (sh0 + hg) * D + col * 4;
         Elem<T>::store(dst + 0, t.x * inv);
         Elem<T>::store(dst + 1, t.y * inv);
         Elem<T>::store(dst + 2, t.z * inv);

@@ -9,9 +9,4 @@ cudaError_t launch_decode_partition_bf16(const DecodeParams& p, int D, int BS, i
     return dispatch_partition<__nv_bfloat16>(p, D, BS, G, grid, st);
 }
 
-cudaError_t launch_decode_reduce_bf16(const ReduceParams& p, int D, long long grid,
-                                      cudaStream_t st) {
-    return dispatch_reduce<__nv_bfloat16>(p, D, grid, st);
-}
-
 }  // namespace pkv

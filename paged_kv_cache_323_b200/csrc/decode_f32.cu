@@ -9,8 +9,4 @@ cudaError_t launch_decode_partition_f32(const DecodeParams& p, int D, int BS, in
     return dispatch_partition<float>(p, D, BS, G, grid, st);
 }
 
-cudaError_t launch_decode_reduce_f32(const ReduceParams& p, int D, long long grid, cudaStream_t st) {
-    return dispatch_reduce<float>(p, D, grid, st);
-}
-
 }  // namespace pkv

@@ -61,17 +61,4 @@ cudaError_t dispatch_partition(const DecodeParams& p, int D, int BS, int G, long
     }
 }
 
-template <typename T>
-cudaError_t dispatch_reduce(const ReduceParams& p, int D, long long grid, cudaStream_t st) {
-    switch (D) {
-        case 64:
-            decode_reduce_kernel<T, 64><<<static_cast<unsigned>(grid), 128, 0, st>>>(p);
-            return cudaGetLastError();
-        case 128:
-            decode_reduce_kernel<T, 128><<<static_cast<unsigned>(grid), 128, 0, st>>>(p);
-            return cudaGetLastError();
-        default: return cudaErrorInvalidValue;
-    }
-}
-
 }  // namespace pkv

@@ -32,31 +32,38 @@ struct AppendParams {
     int chunks_per_row;  // head_dim * elt / 16
 };
 
-// One thread per 16-byte chunk of one (token, kv head) row, K and V.
+// A CTA of 256 threads covers 256 / chunks_per_row whole (token, kv head)
+// rows, one thread per 16-byte chunk.  The new token's K and V chunks are
+// loaded before the slot is known, so the only dependent step is the store.
 __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
-    const long long per_token = (long long)p.num_kv_heads * p.chunks_per_row;
-    const long long total = (long long)p.num_tokens * per_token;
+    const int cpr = p.chunks_per_row;
+    const int rows_per_cta = blockDim.x / cpr;
+    const int r_in = threadIdx.x / cpr;
+    const int ch = threadIdx.x - r_in * cpr;
+    if (r_in >= rows_per_cta) return;
+    const long long nrows = (long long)p.num_tokens * p.num_kv_heads;
     uint4* kc = static_cast<uint4*>(p.k_cache);
     uint4* vc = static_cast<uint4*>(p.v_cache);
     const uint4* kn = static_cast<const uint4*>(p.k);
     const uint4* vn = static_cast<const uint4*>(p.v);
-    for (long long x = blockIdx.x * (long long)blockDim.x + threadIdx.x; x < total;
-         x += (long long)gridDim.x * blockDim.x) {
-        const long long i = x / per_token;
-        const long long rem = x - i * per_token;  // g * chunks_per_row + chunk
+    for (long long row = (long long)blockIdx.x * rows_per_cta + r_in; row < nrows;
+         row += (long long)gridDim.x * rows_per_cta) {
+        const long long x = row * cpr + ch;
+        const uint4 kv = kn[x];
+        const uint4 vv = vn[x];
+        const long long i = row / p.num_kv_heads;
+        const long long g = row - i * p.num_kv_heads;
         const long long slot = p.slot_mapping[i];
         if (slot < 0) continue;  // -1: nothing to write for this token
         if (slot >= p.num_slots) {
-            if (rem == 0) set_error(p.err, PKV_ERR_DEVICE_BOUNDS);
+            if (ch == 0 && g == 0) set_error(p.err, PKV_ERR_DEVICE_BOUNDS);
             continue;
         }
         const long long blk = slot / p.block_size;
         const long long off = slot - blk * p.block_size;
-        const long long g = rem / p.chunks_per_row;
-        const long long ch = rem - g * p.chunks_per_row;
-        const long long dst = ((blk * p.num_kv_heads + g) * p.block_size + off) * p.chunks_per_row + ch;
-        kc[dst] = kn[x];
-        vc[dst] = vn[x];
+        const long long dst = ((blk * p.num_kv_heads + g) * p.block_size + off) * cpr + ch;
+        kc[dst] = kv;
+        vc[dst] = vv;
     }
 }
 

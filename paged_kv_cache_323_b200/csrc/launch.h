@@ -11,8 +11,5 @@ cudaError_t launch_decode_partition_f32(const DecodeParams& p, int D, int BS, in
                                         cudaStream_t st);
 cudaError_t launch_decode_partition_bf16(const DecodeParams& p, int D, int BS, int G,
                                          long long grid, cudaStream_t st);
-cudaError_t launch_decode_reduce_f32(const ReduceParams& p, int D, long long grid, cudaStream_t st);
-cudaError_t launch_decode_reduce_bf16(const ReduceParams& p, int D, long long grid,
-                                      cudaStream_t st);
 
 }  // namespace pkv

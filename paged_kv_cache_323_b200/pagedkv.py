@@ -33,10 +33,9 @@ PKV_ERR_DEVICE_BOUNDS = -6
 PKV_ERR_TIMEOUT = -7
 PKV_F32 = 0
 PKV_BF16 = 1
-KERNEL_DECODE_PARTITION = 0
-KERNEL_DECODE_REDUCE = 1
-KERNEL_APPEND = 2
-KERNEL_COPY_BLOCKS = 3
+KERNEL_DECODE = 0
+KERNEL_APPEND = 1
+KERNEL_COPY_BLOCKS = 2
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -115,8 +114,9 @@ def paged_attention_decode_ex(out, q, k_cache, v_cache, block_tables, context_le
                               *, num_blocks: int | None = None, partition_tokens: int = 0,
                               workspace: torch.Tensor | None = None, stream=None) -> None:
     """out, q: [B][H][D]; caches: [N][Hkv][bs][D]; block_tables int32 [B][maxb];
-    context_lens int32 [B].  ``workspace`` is a uint8 CUDA tensor of at least
-    :func:`paged_attention_workspace_size` bytes (allocated here when None)."""
+    context_lens int32 [B].  ``workspace`` is a zero-initialised uint8 CUDA
+    tensor of at least :func:`paged_attention_workspace_size` bytes, reusable
+    across calls (a fresh zeroed one is allocated here when None)."""
     B, H, D = q.shape
     N, Hkv, bs, D2 = k_cache.shape
     if D2 != D or tuple(out.shape) != (B, H, D) or tuple(v_cache.shape) != tuple(k_cache.shape):
@@ -126,7 +126,7 @@ def paged_attention_decode_ex(out, q, k_cache, v_cache, block_tables, context_le
         num_blocks = N
     need = paged_attention_workspace_size(B, H, maxb * bs, D, partition_tokens)
     if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     code = _dtype_code(q)

@@ -286,8 +286,8 @@ def test_launch_count_and_profiler():
     n0 = pk.launch_count()
     gpu_step(w, t)
     pk.profile_enable(False)
-    assert pk.launch_count() - n0 == 3  # append, partition, reduce
-    n, ms = pk.profile_read(pk.KERNEL_DECODE_PARTITION)
+    assert pk.launch_count() - n0 == 2  # append, decode (split-K merge fused)
+    n, ms = pk.profile_read(pk.KERNEL_DECODE)
     assert n == 1 and ms > 0
     n, _ = pk.profile_read(pk.KERNEL_APPEND)
     assert n == 1
