@@ -162,6 +162,40 @@ PKV_API int copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_pai
                 int num_kv_heads, int head_dim, int block_size, int num_blocks, int dtype,
                 void* stream);
 
+/*
+ * Decode attention for callers that cannot allocate device memory.  The pages
+ * have no counterpart of this call: it is a property of this library, not of
+ * the method.
+ *
+ * A serving engine usually gives its KV-block pool all the device memory left
+ * after the weights, some host frameworks forbid allocations outside their own
+ * allocator, and cudaMalloc / cudaFree may synchronise the device; such
+ * callers cannot provide or let the library allocate the split-K workspace.
+ * This call computes exactly what paged_attention_decode_ex computes (same
+ * arguments without the workspace, same kernel, same results) and keeps the
+ * split-K scratch in a fixed array of PKV_NOALLOC_SCRATCH_BYTES that is part
+ * of the library's device image: every GPU that loads the library holds that
+ * memory until the process exits.  It calls no allocating routine.
+ *   - A batch whose scratch (paged_attention_workspace_size for the partition
+ *     size chosen) exceeds PKV_NOALLOC_SCRATCH_BYTES returns
+ *     PKV_ERR_WORKSPACE without launching anything; a larger partition_tokens
+ *     lowers the need.
+ *   - The first call on a device looks up the array's device address there
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls share the array and it keeps the last call's contents; each
+ *     call clears the merge counters on its stream before its kernel.  Calls
+ *     whose kernels overlap on the GPU (other streams, other threads) race on
+ *     the array: order them.
+ */
+#define PKV_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+PKV_API int paged_attention_decode_noalloc(void* out, const void* q, const void* k_cache,
+                                           const void* v_cache, const int32_t* block_tables,
+                                           const int32_t* context_lens, int num_seqs,
+                                           int num_heads, int num_kv_heads, int head_dim,
+                                           int block_size, int max_blocks_per_seq, float scale,
+                                           int num_blocks, int dtype, int partition_tokens,
+                                           void* stream);
+
 /* Synchronise `stream`, then return in *code the current device's error word
  * (PKV_OK, PKV_ERR_DEVICE_BOUNDS or PKV_ERR_TIMEOUT) and clear it. */
 PKV_API int pkv_get_device_error(void* stream, int* code);

@@ -155,6 +155,28 @@ int auto_partition_tokens(long long num_seqs, long long num_kv_heads, long long 
 
 }  // namespace
 
+// Not exported: the workspace paged_attention_decode_ex needs for the
+// partition size it would pick, and where the merge counters sit in it.
+extern "C" void pkv_internal_decode_scratch(int num_seqs, int num_heads, int num_kv_heads,
+                                            int head_dim, int block_size, int max_blocks_per_seq,
+                                            int partition_tokens, size_t* total, size_t* cnt_off,
+                                            size_t* cnt_bytes) {
+    *total = *cnt_off = *cnt_bytes = 0;
+    if (num_seqs <= 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        max_blocks_per_seq <= 0 || partition_tokens < 0)
+        return;
+    const long long max_ctx = (long long)max_blocks_per_seq * block_size;
+    const long long pt = partition_tokens == 0 ? auto_partition_tokens(num_seqs, num_kv_heads, max_ctx)
+                                               : partition_tokens;
+    const long long parts = (max_ctx + pt - 1) / pt;
+    const WorkspaceLayout w = workspace_layout(num_seqs, num_heads, parts, head_dim);
+    *total = w.total;
+    if (w.total > 0) {
+        *cnt_off = w.cnt_off;
+        *cnt_bytes = size_t(num_seqs) * num_heads * sizeof(int);
+    }
+}
+
 extern "C" {
 
 size_t paged_attention_workspace_size(int num_seqs, int num_heads, int max_context, int head_dim,

@@ -47,6 +47,8 @@ SIGNATURES = {
     "paged_attention_decode_ex": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float,
                                        _I, _I, _I, _P, _SZ, _P]),
     "paged_attention_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "paged_attention_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
+                                            ctypes.c_float, _I, _I, _I, _P]),
     "kv_cache_append": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     "copy_blocks": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     "pkv_get_device_error": (_I, [_P, ctypes.POINTER(_I)]),
@@ -136,6 +138,34 @@ def paged_attention_decode_ex(out, q, k_cache, v_cache, block_tables, context_le
         _dev(context_lens, "context_lens", torch.int32), B, H, Hkv, D, bs, maxb, float(scale),
         int(num_blocks), code, int(partition_tokens), ws_ptr, ws_bytes, _stream(stream))
     _check(rc, "paged_attention_decode_ex")
+
+
+# Size of the fixed device scratch of paged_attention_decode_noalloc.
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
+
+
+def paged_attention_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens,
+                                   scale: float, *, num_blocks: int | None = None,
+                                   partition_tokens: int = 0, stream=None) -> None:
+    """Same result as :func:`paged_attention_decode_ex`, for callers that
+    cannot allocate device memory (a KV pool that fills the GPU, a host
+    allocator that must account for every byte, or a loop that cannot afford
+    cudaMalloc's synchronisation): the split-K scratch lives in a fixed
+    NOALLOC_SCRATCH_BYTES device array inside the library, shared by every
+    call, so calls must not overlap on the GPU.  Batches that need more
+    scratch raise PagedKVError (PKV_ERR_WORKSPACE).  Nothing is allocated."""
+    B, H, D = q.shape
+    N, Hkv, bs, D2 = k_cache.shape
+    if D2 != D or tuple(out.shape) != (B, H, D) or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("shape mismatch between q, out and the caches")
+    maxb = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    rc = lib.paged_attention_decode_noalloc(
+        _dev(out, "out", q.dtype), _dev(q, "q"), _dev(k_cache, "k_cache", q.dtype),
+        _dev(v_cache, "v_cache", q.dtype), _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32), B, H, Hkv, D, bs, maxb, float(scale),
+        N if num_blocks is None else int(num_blocks), _dtype_code(q), int(partition_tokens),
+        _stream(stream))
+    _check(rc, "paged_attention_decode_noalloc")
 
 
 def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,

@@ -110,3 +110,14 @@ def test_status_strings_and_version(pk):
     assert pk.status_string(-99) == "unknown status"
     assert pk.lib.pkv_version() == 100
     assert pk.lib.pkv_get_device_error(None, None) == pk.PKV_ERR_NULL
+
+
+def test_noalloc_validation(pk):
+    """The fixed-scratch entry point refuses oversize batches before touching the GPU."""
+    L = pk.lib
+    args = [FAKE] * 6
+    assert L.paged_attention_decode_noalloc(*args, 0, 8, 2, 128, 16, 8, 0.1, 64, 1, 0, None) == pk.PKV_OK
+    assert L.paged_attention_decode_noalloc(*args, -1, 8, 2, 128, 16, 8, 0.1, 64, 1, 0, None) == pk.PKV_ERR_INVALID
+    # 64 sequences x 64 heads x 128 partitions x 128 dims of fp32 partials >> 16 MiB
+    assert L.paged_attention_decode_noalloc(*args, 64, 64, 8, 128, 16, 4096, 0.1, 64, 1, 512,
+                                            None) == pk.PKV_ERR_WORKSPACE
