@@ -189,13 +189,25 @@ def barrier(world):
 
 
 def max_over_ranks(world, x: float) -> float:
+    """The slowest rank's time: every rank's number goes through one MAX all-reduce."""
     if world == 1:
         return x
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(workload: str, rank: int) -> int:
+    """Each rank draws its own batch (weak scaling): seed offset by rank."""
+    return DEFAULT_SEED[workload] + 1000 * rank
+
+
+def job_value(world: int, kv_bytes_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job KV GB/s: the bytes all ranks read per step over the slowest rank's step time."""
+    return world * kv_bytes_per_rank / (ms_per_step / 1e3) / 1e9
 
 
 def compact_subset(w: wl.Workload, seqs):
@@ -297,8 +309,7 @@ def run_gpu(args, world, rank, local):
     from paged_kv_cache_323_b200 import pagedkv as pk
 
     name, make = WORKLOADS[args.workload]
-    seed = DEFAULT_SEED[args.workload] + 1000 * rank  # each rank its own batch (weak scaling)
-    w = make("cuda", seed)
+    w = make("cuda", rank_seed(args.workload, rank))
     dev = torch.device("cuda", torch.cuda.current_device())
     t = {
         "q": w.q, "k_cache": w.k_cache, "v_cache": w.v_cache, "k_new": w.k_new, "v_new": w.v_new,
@@ -394,7 +405,7 @@ def run_gpu(args, world, rank, local):
         return
     kv_bytes = w.kv_bytes_logical()
     step_s = ms / args.steps / 1e3
-    value = world * kv_bytes / step_s / 1e9
+    value = job_value(world, kv_bytes, ms / args.steps)
     peak, peak_src = measured_peak()
     part = per_kernel.get("decode")
     roofline = None
@@ -412,7 +423,9 @@ def run_gpu(args, world, rank, local):
         "config": {"workload": name, "num_seqs_per_gpu": w.num_seqs, "num_heads": w.num_heads,
                    "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
                    "block_size": w.block_size, "kv_bytes_per_step_per_gpu": kv_bytes,
-                   "partition_tokens": args.partition_tokens or 512,
+                   "partition_tokens": pk.paged_attention_partition_tokens(
+                       w.num_seqs, w.num_kv_heads, w.max_blocks_per_seq * w.block_size,
+                       args.partition_tokens),
                    "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush",
                    "parallelism": f"{world} independent batches, one per GPU"},
         "tokens_per_s": world * w.num_seqs / step_s,
@@ -420,7 +433,7 @@ def run_gpu(args, world, rank, local):
         "per_kernel_us": per_kernel,
         "roofline": roofline,
         "gpu_launches": launches,
-        "e2e": {"value": world * kv_bytes / (ms_e2e / args.steps / 1e3) / 1e9, "unit": "GB/s",
+        "e2e": {"value": job_value(world, kv_bytes, ms_e2e / args.steps), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": ms_e2e / args.steps},
         "clocks": clock_info,

@@ -106,9 +106,9 @@ PKV_API int paged_attention_decode(void* out, const void* q, const void* k_cache
  *                     device faults (the block is skipped, error word set).
  *   dtype             pkv_dtype of q, out and the pools.
  *   partition_tokens  context tokens per CTA (split-K); a multiple of
- *                     block_size, at most 4096, or 0 for automatic (512,
+ *                     block_size, at most 4096, or 0 for automatic (1024,
  *                     doubled for very long tables while the grid stays
- *                     large).  A sequence longer than one partition is split;
+ *                     large; see paged_attention_partition_tokens).  A sequence longer than one partition is split;
  *                     the last of its partitions to finish merges them all in
  *                     partition order, inside the same kernel.  Shorter ones
  *                     are written in one pass.
@@ -130,8 +130,14 @@ PKV_API int paged_attention_decode_ex(void* out, const void* q, const void* k_ca
                               int dtype, int partition_tokens, void* workspace,
                               size_t workspace_bytes, void* stream);
 
+/* Partition size (tokens per CTA) paged_attention_decode_ex uses for these
+ * sizes: partition_tokens itself, or the automatic choice when it is 0. */
+PKV_API int paged_attention_partition_tokens(int num_seqs, int num_kv_heads, int max_context,
+                                             int partition_tokens);
+
 /* Bytes of split-K workspace paged_attention_decode_ex needs; 0 when every
- * sequence fits one partition. */
+ * sequence fits one partition.  With partition_tokens 0 the result covers
+ * any automatic choice. */
 PKV_API size_t paged_attention_workspace_size(int num_seqs, int num_heads, int max_context, int head_dim,
                                       int partition_tokens);
 

@@ -23,7 +23,8 @@ __device__ int g_pkv_device_error;
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kAutoPartitionTokens = 512;
+constexpr int kAutoPartitionTokens = 1024;
+constexpr int kMinPartitionTokens = 512;  // bounds the automatic choice from below
 constexpr int kMaxPartitionTokens = 4096;
 
 struct DeviceState {
@@ -140,10 +141,11 @@ size_t workspace_bytes_for(long long num_seqs, long long num_heads, long long pa
     return workspace_layout(num_seqs, num_heads, parts, D).total;
 }
 
-// Partition size when the caller passes 0: 512 tokens, doubled (up to 4096)
-// while a sequence of the maximum length would still be split into more than
-// 64 partitions and the grid keeps at least four waves of 3 CTAs per SM.  Long
-// contexts then merge fewer partials in the fused split-K merge.
+// Partition size when the caller passes 0: 1024 tokens (fewer split-K
+// merges than 512 at no loss of parallelism on batch-64 MHA), doubled (up to
+// 4096) while a sequence of the maximum length would still be split into more
+// than 64 partitions and the grid keeps at least four waves of 3 CTAs per SM.
+// Long contexts then merge fewer partials in the fused split-K merge.
 int auto_partition_tokens(long long num_seqs, long long num_kv_heads, long long max_ctx) {
     long long pt = kAutoPartitionTokens;
     const long long min_ctas = 4LL * 148 * 3;
@@ -184,10 +186,17 @@ size_t paged_attention_workspace_size(int num_seqs, int num_heads, int max_conte
     if (num_seqs <= 0 || num_heads <= 0 || max_context <= 0 || head_dim <= 0 ||
         partition_tokens < 0)
         return 0;
-    // the automatic size is never below 512 tokens, so 512 bounds its workspace
-    const long long pt = partition_tokens == 0 ? kAutoPartitionTokens : partition_tokens;
+    // the automatic size is never below kMinPartitionTokens, which bounds its workspace
+    const long long pt = partition_tokens == 0 ? kMinPartitionTokens : partition_tokens;
     const long long parts = (max_context + pt - 1) / pt;
     return workspace_bytes_for(num_seqs, num_heads, parts, head_dim);
+}
+
+int paged_attention_partition_tokens(int num_seqs, int num_kv_heads, int max_context,
+                                     int partition_tokens) {
+    if (num_seqs <= 0 || num_kv_heads <= 0 || max_context <= 0 || partition_tokens < 0) return 0;
+    return partition_tokens == 0 ? auto_partition_tokens(num_seqs, num_kv_heads, max_context)
+                                 : partition_tokens;
 }
 
 int paged_attention_decode_ex(void* out, const void* q, const void* k_cache, const void* v_cache,

@@ -505,7 +505,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, BS, G>::THREADS, 2)
         const float4* o = reinterpret_cast<const float4*>(p.ws_o + (sh0 + hg) * P * D) + col;
         float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
         if (M != -INFINITY) {
-#pragma unroll 4
+#pragma unroll 8
             for (int i = grp; i < nparts; i += GROUPS) {
                 const float w = exp2f(__ldcg(&ml[i]).x - M);
                 const float4 v = __ldcg(o + (long long)i * COLS);

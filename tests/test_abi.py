@@ -121,3 +121,12 @@ def test_noalloc_validation(pk):
     # 64 sequences x 64 heads x 128 partitions x 128 dims of fp32 partials >> 16 MiB
     assert L.paged_attention_decode_noalloc(*args, 64, 64, 8, 128, 16, 4096, 0.1, 64, 1, 512,
                                             None) == pk.PKV_ERR_WORKSPACE
+
+
+def test_partition_tokens(pk):
+    pt = pk.paged_attention_partition_tokens
+    assert pt(64, 32, 2048, 0) == 1024  # batch-64 MHA: automatic 1024
+    assert pt(64, 32, 2048, 256) == 256  # explicit sizes pass through
+    big = pt(8, 8, 131072, 0)  # long context: fewer, larger partitions
+    assert big > 1024 and big <= 4096 and 131072 // big <= 64
+    assert pt(0, 8, 1024, 0) == 0
