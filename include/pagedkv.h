@@ -219,6 +219,13 @@ PKV_API int pkv_profile_enable(int on);
 PKV_API int pkv_profile_read(int kind, long long* launches, double* total_ms);
 PKV_API int pkv_profile_reset(void);
 
+/* Choose the decode kernel for grouped-query heads (2, 4 or 8 query heads
+ * per kv head, bf16, head_dim 128, partitions a multiple of 128 tokens):
+ * 1 (default) runs the tensor-core kernel (tcgen05 MMAs into tensor memory),
+ * 0 the CUDA-core kernel that serves every other shape.  Both compute the
+ * same attention; returns the previous setting.  Process-wide. */
+PKV_API int pkv_set_tensor_core_gqa(int enable);
+
 /* Kernels launched by this library in this process so far (all kinds). */
 PKV_API unsigned long long pkv_launch_count(void);
 

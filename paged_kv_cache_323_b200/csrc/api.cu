@@ -35,6 +35,7 @@ struct DeviceState {
 
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
+std::atomic<int> g_tc_gqa{1};  // tensor-core kernel for grouped-query heads where it applies
 std::atomic<unsigned long long> g_launches{0};
 
 // ---------------------------------------------------------- profiler
@@ -261,7 +262,10 @@ int paged_attention_decode_ex(void* out, const void* q, const void* k_cache, con
     p.qscale = scale * 1.4426950408889634f;  // log2(e): softmax runs in base 2
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool use_tc = g_tc_gqa.load() != 0 &&
+                        pkv::decode_tc_supported(dtype, head_dim, block_size, group, pt);
     return launch(PKV_KERNEL_DECODE, st, [&] {
+        if (use_tc) return pkv::launch_decode_tc(p, block_size, group, grid, st);
         return dtype == PKV_F32 ? pkv::launch_decode_partition_f32(p, head_dim, block_size, group, grid, st)
                                 : pkv::launch_decode_partition_bf16(p, head_dim, block_size, group, grid, st);
     });
@@ -440,6 +444,10 @@ int pkv_profile_reset(void) {
 }
 
 unsigned long long pkv_launch_count(void) { return g_launches.load(); }
+
+int pkv_set_tensor_core_gqa(int enable) {
+    return g_tc_gqa.exchange(enable != 0 ? 1 : 0);
+}
 
 int pkv_version(void) { return 100; }
 

@@ -1,0 +1,100 @@
+// decode_tc.cu -- host side of the tensor-core GQA decode kernel: TMA tensor
+// maps over the K and V pools, and dispatch over (block_size, group size).
+#include <atomic>
+#include <mutex>
+
+#include "decode_tc.cuh"
+#include "launch.h"
+
+namespace pkv {
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encoder() {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+// The pool [num_blocks][Hkv][bs][128] bf16 as a 4-D tensor (dims innermost
+// first: dim, slot, kv head, block); boxes of 64 dims x bs slots of one
+// (block, kv head), 128-byte swizzle.
+cudaError_t make_pool_map(CUtensorMap* map, const void* pool, int Hkv, int BS, int num_blocks) {
+    EncodeTiledFn fn = encoder();
+    if (fn == nullptr) return cudaErrorNotSupported;
+    const cuuint64_t dims[4] = {128, (cuuint64_t)BS, (cuuint64_t)Hkv, (cuuint64_t)num_blocks};
+    const cuuint64_t strides[3] = {128 * 2, (cuuint64_t)BS * 128 * 2, (cuuint64_t)Hkv * BS * 128 * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)BS, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(pool), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int BS, int G>
+cudaError_t launch_inst(const DecodeParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
+                        long long grid, cudaStream_t st) {
+    using C = tc::TcCfg<BS, G>;
+    auto kern = tc::decode_tc_kernel<BS, G>;
+    static std::atomic<unsigned long long> configured{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(configured.load() & bit)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        configured.fetch_or(bit);
+    }
+    kern<<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, st>>>(p, mk, mv);
+    return cudaGetLastError();
+}
+
+template <int BS>
+cudaError_t launch_group(const DecodeParams& p, int G, const CUtensorMap& mk, const CUtensorMap& mv,
+                         long long grid, cudaStream_t st) {
+    switch (G) {
+        case 2: return launch_inst<BS, 2>(p, mk, mv, grid, st);
+        case 4: return launch_inst<BS, 4>(p, mk, mv, grid, st);
+        case 8: return launch_inst<BS, 8>(p, mk, mv, grid, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+bool decode_tc_supported(int dtype, int D, int BS, int G, int partition_tokens) {
+    return dtype == PKV_BF16 && D == 128 && (BS == 8 || BS == 16 || BS == 32) &&
+           (G == 2 || G == 4 || G == 8) && partition_tokens % 128 == 0;
+}
+
+cudaError_t launch_decode_tc(const DecodeParams& p, int BS, int G, long long grid,
+                             cudaStream_t st) {
+    CUtensorMap mk, mv;
+    cudaError_t e = make_pool_map(&mk, p.k_cache, p.num_kv_heads, BS, p.num_blocks);
+    if (e != cudaSuccess) return e;
+    e = make_pool_map(&mv, p.v_cache, p.num_kv_heads, BS, p.num_blocks);
+    if (e != cudaSuccess) return e;
+    switch (BS) {
+        case 8: return launch_group<8>(p, G, mk, mv, grid, st);
+        case 16: return launch_group<16>(p, G, mk, mv, grid, st);
+        case 32: return launch_group<32>(p, G, mk, mv, grid, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace pkv

@@ -58,6 +58,7 @@ SIGNATURES = {
     "pkv_profile_read": (_I, [_I, ctypes.POINTER(ctypes.c_longlong), ctypes.POINTER(ctypes.c_double)]),
     "pkv_profile_reset": (_I, []),
     "pkv_launch_count": (ctypes.c_ulonglong, []),
+    "pkv_set_tensor_core_gqa": (_I, [_I]),
     "pkv_version": (_I, []),
 }
 for _name, (_res, _args) in SIGNATURES.items():
@@ -237,3 +238,9 @@ def profile_reset() -> None:
 
 def launch_count() -> int:
     return int(lib.pkv_launch_count())
+
+
+def set_tensor_core_gqa(enable: bool) -> bool:
+    """Select the tensor-core (True) or CUDA-core (False) decode kernel for
+    grouped-query heads; returns the previous setting."""
+    return bool(lib.pkv_set_tensor_core_gqa(1 if enable else 0))

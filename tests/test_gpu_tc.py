@@ -1,0 +1,99 @@
+"""The tensor-core (tcgen05) decode kernel for grouped-query heads against the
+oracle, and against the CUDA-core kernel on the same inputs.
+
+It serves bf16 caches with head_dim 128, groups of 2/4/8 query heads and
+partitions that are multiples of 128 tokens; the cases below span partial
+128-token chunks, partial blocks, several partitions (fused split-K merge),
+NaN in unused slots, and bad table entries.
+"""
+import numpy as np
+import pytest
+import torch
+
+from paged_kv_cache_323_b200 import workload as wl
+from steps import assert_close, assert_pool_equal, gpu_step, oracle_step, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture
+def tc_mode():
+    from paged_kv_cache_323_b200 import pagedkv as pk
+
+    prev = pk.set_tensor_core_gqa(True)
+    yield pk
+    pk.set_tensor_core_gqa(prev)
+
+
+@pytest.mark.parametrize("bs", [8, 16, 32])
+@pytest.mark.parametrize("G", [2, 4, 8])
+def test_tc_small(tc_mode, bs, G):
+    lens = [1, 5, 127, 128, 129, 300, 640]
+    w = wl.custom(200 + G + bs, lens, heads=2 * G, kv_heads=2, head_dim=128, block_size=bs,
+                  dtype="bf16", maxb=-(-640 // bs) + 1)
+    ref, kref, vref = oracle_step(w)
+    out, kc, vc = gpu_step(w, partition_tokens=256)
+    assert_pool_equal(kc, kref, "k pool")
+    assert_close(out, ref, w.dtype)
+
+
+@pytest.mark.parametrize("pt", [128, 512, 1024, 0])
+def test_tc_partitions(tc_mode, pt):
+    w = wl.gqa_sampling(groups=4, prompt_median=600, prompt_max=3000)
+    ref, _, _ = oracle_step(w)
+    out, _, _ = gpu_step(w, partition_tokens=pt)
+    assert_close(out, ref, w.dtype)
+
+
+def test_tc_matches_cuda_core(tc_mode):
+    pk = tc_mode
+    w = wl.prefix_sweep(16, num_seqs=16, prefix=512, suffix_range=(16, 300))
+    ref, _, _ = oracle_step(w)
+    out_tc, _, _ = gpu_step(w)
+    pk.set_tensor_core_gqa(False)
+    out_cc, _, _ = gpu_step(w)
+    pk.set_tensor_core_gqa(True)
+    assert_close(out_tc, ref, w.dtype, "tensor-core kernel")
+    assert_close(out_cc, ref, w.dtype, "CUDA-core kernel")
+    d = (out_tc.float() - out_cc.float()).abs().max().item()
+    assert d <= 2e-2, d
+
+
+def test_tc_nan_poisoned_and_bad_entry(tc_mode):
+    pk = tc_mode
+    w = wl.custom(77, [200, 333, 50], heads=16, kv_heads=2, head_dim=128, block_size=16,
+                  dtype="bf16", num_blocks=60, maxb=24)
+    bs = w.block_size
+    used = np.zeros((w.num_blocks, bs), dtype=bool)
+    for s in range(w.num_seqs):
+        for t in range(int(w.context_lens[s])):
+            used[w.block_tables[s][t // bs], t % bs] = True
+    mask = torch.from_numpy(~used)[:, None, :, None].expand_as(w.k_cache)
+    w.k_cache = w.k_cache.masked_fill(mask, float("nan"))
+    w.v_cache = w.v_cache.masked_fill(mask, float("nan"))
+    ref, _, _ = oracle_step(w)
+    out, _, _ = gpu_step(w, partition_tokens=128)
+    assert_close(out, ref, w.dtype)
+    # a table entry outside the pool: error word set, output finite
+    w.block_tables[1, 3] = w.num_blocks + 5
+    t = to_device(w)
+    out, _, _ = gpu_step(w, t, partition_tokens=128, check_error=False)
+    assert pk.get_device_error() == pk.PKV_ERR_DEVICE_BOUNDS
+    assert torch.isfinite(out.float()).all()
+
+
+def test_tc_permutation_bit_identical(tc_mode):
+    w = wl.custom(91, [700, 1000, 257], heads=32, kv_heads=8, head_dim=128, block_size=16,
+                  dtype="bf16")
+    out1, _, _ = gpu_step(w)
+    perm = np.random.default_rng(3).permutation(w.num_blocks)
+    w2 = wl.Workload(**{**w.__dict__})
+    w2.k_cache = torch.empty_like(w.k_cache)
+    w2.v_cache = torch.empty_like(w.v_cache)
+    w2.k_cache[torch.from_numpy(perm)] = w.k_cache
+    w2.v_cache[torch.from_numpy(perm)] = w.v_cache
+    w2.block_tables = np.where(w.block_tables >= 0, perm[np.maximum(w.block_tables, 0)], -1).astype(np.int32)
+    bs = w.block_size
+    w2.slot_mapping = np.asarray([perm[s // bs] * bs + s % bs for s in w.slot_mapping], dtype=np.int64)
+    out2, _, _ = gpu_step(w2)
+    assert torch.equal(out1, out2)
