@@ -106,9 +106,8 @@ PKV_API int paged_attention_decode(void* out, const void* q, const void* k_cache
  *                     device faults (the block is skipped, error word set).
  *   dtype             pkv_dtype of q, out and the pools.
  *   partition_tokens  context tokens per CTA (split-K); a multiple of
- *                     block_size, at most 4096, or 0 for automatic (1024,
- *                     doubled for very long tables while the grid stays
- *                     large; see paged_attention_partition_tokens).  A sequence longer than one partition is split;
+ *                     block_size, at most 4096, or 0 for automatic (see
+ *                     paged_attention_partition_tokens).  A sequence longer than one partition is split;
  *                     the last of its partitions to finish merges them all in
  *                     partition order, inside the same kernel.  Shorter ones
  *                     are written in one pass.
@@ -131,9 +130,11 @@ PKV_API int paged_attention_decode_ex(void* out, const void* q, const void* k_ca
                               size_t workspace_bytes, void* stream);
 
 /* Partition size (tokens per CTA) paged_attention_decode_ex uses for these
- * sizes: partition_tokens itself, or the automatic choice when it is 0. */
-PKV_API int paged_attention_partition_tokens(int num_seqs, int num_kv_heads, int max_context,
-                                             int partition_tokens);
+ * arguments: partition_tokens itself, or the automatic choice when it is 0
+ * (which depends on the kernel that serves the shape).  0 on bad sizes. */
+PKV_API int paged_attention_partition_tokens(int num_seqs, int num_heads, int num_kv_heads,
+                                             int head_dim, int block_size, int max_context,
+                                             int dtype, int partition_tokens);
 
 /* Bytes of split-K workspace paged_attention_decode_ex needs; 0 when every
  * sequence fits one partition.  With partition_tokens 0 the result covers

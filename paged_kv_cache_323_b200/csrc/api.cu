@@ -142,12 +142,24 @@ size_t workspace_bytes_for(long long num_seqs, long long num_heads, long long pa
     return workspace_layout(num_seqs, num_heads, parts, D).total;
 }
 
-// Partition size when the caller passes 0: 1024 tokens (fewer split-K
-// merges than 512 at no loss of parallelism on batch-64 MHA), doubled (up to
-// 4096) while a sequence of the maximum length would still be split into more
-// than 64 partitions and the grid keeps at least four waves of 3 CTAs per SM.
-// Long contexts then merge fewer partials in the fused split-K merge.
-int auto_partition_tokens(long long num_seqs, long long num_kv_heads, long long max_ctx) {
+// Partition size when the caller passes 0.
+//  * CUDA-core kernel: 1024 tokens (fewer split-K merges than 512 at no loss
+//    of parallelism on batch-64 MHA), doubled (up to 4096) while a sequence
+//    of the maximum length would still be split into more than 64 partitions
+//    and the grid keeps at least four waves of 3 CTAs per SM.
+//  * Tensor-core kernel: 4096 tokens, halved (down to 512) while the grid
+//    would have fewer than eight waves of 2 CTAs per SM.  Its CTAs carry a
+//    fixed set-up and drain cost, so long partitions pay: on B200 the
+//    parallel-sampling GQA batch ran at 0.55 / 0.75 / 0.88 / 0.97 of peak
+//    with 512 / 1024 / 2048 / 4096-token partitions.
+int auto_partition_tokens(long long num_seqs, long long num_kv_heads, long long max_ctx, bool tc) {
+    if (tc) {
+        long long pt = kMaxPartitionTokens;
+        const long long min_ctas = 8LL * 148 * 2;
+        while (pt > kMinPartitionTokens && num_seqs * num_kv_heads * ((max_ctx + pt - 1) / pt) < min_ctas)
+            pt /= 2;
+        return (int)pt;
+    }
     long long pt = kAutoPartitionTokens;
     const long long min_ctas = 4LL * 148 * 3;
     while (pt < kMaxPartitionTokens && (max_ctx + pt - 1) / pt > 64 &&
@@ -156,21 +168,35 @@ int auto_partition_tokens(long long num_seqs, long long num_kv_heads, long long 
     return (int)pt;
 }
 
+// Whether the tensor-core kernel serves this shape (any partition size that
+// is a multiple of 128 tokens).
+bool tc_shape(int dtype, int head_dim, int block_size, int group) {
+    return g_tc_gqa.load() != 0 && pkv::decode_tc_supported(dtype, head_dim, block_size, group, 128);
+}
+
+int resolve_partition_tokens(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                             int block_size, long long max_ctx, int dtype, int partition_tokens) {
+    if (partition_tokens != 0) return partition_tokens;
+    const int group = num_kv_heads > 0 ? num_heads / num_kv_heads : 1;
+    return auto_partition_tokens(num_seqs, num_kv_heads, max_ctx,
+                                 tc_shape(dtype, head_dim, block_size, group));
+}
+
 }  // namespace
 
 // Not exported: the workspace paged_attention_decode_ex needs for the
 // partition size it would pick, and where the merge counters sit in it.
 extern "C" void pkv_internal_decode_scratch(int num_seqs, int num_heads, int num_kv_heads,
                                             int head_dim, int block_size, int max_blocks_per_seq,
-                                            int partition_tokens, size_t* total, size_t* cnt_off,
-                                            size_t* cnt_bytes) {
+                                            int dtype, int partition_tokens, size_t* total,
+                                            size_t* cnt_off, size_t* cnt_bytes) {
     *total = *cnt_off = *cnt_bytes = 0;
     if (num_seqs <= 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
         max_blocks_per_seq <= 0 || partition_tokens < 0)
         return;
     const long long max_ctx = (long long)max_blocks_per_seq * block_size;
-    const long long pt = partition_tokens == 0 ? auto_partition_tokens(num_seqs, num_kv_heads, max_ctx)
-                                               : partition_tokens;
+    const long long pt = resolve_partition_tokens(num_seqs, num_heads, num_kv_heads, head_dim,
+                                                  block_size, max_ctx, dtype, partition_tokens);
     const long long parts = (max_ctx + pt - 1) / pt;
     const WorkspaceLayout w = workspace_layout(num_seqs, num_heads, parts, head_dim);
     *total = w.total;
@@ -193,11 +219,14 @@ size_t paged_attention_workspace_size(int num_seqs, int num_heads, int max_conte
     return workspace_bytes_for(num_seqs, num_heads, parts, head_dim);
 }
 
-int paged_attention_partition_tokens(int num_seqs, int num_kv_heads, int max_context,
+int paged_attention_partition_tokens(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                     int block_size, int max_context, int dtype,
                                      int partition_tokens) {
-    if (num_seqs <= 0 || num_kv_heads <= 0 || max_context <= 0 || partition_tokens < 0) return 0;
-    return partition_tokens == 0 ? auto_partition_tokens(num_seqs, num_kv_heads, max_context)
-                                 : partition_tokens;
+    if (num_seqs <= 0 || num_heads <= 0 || num_kv_heads <= 0 || max_context <= 0 ||
+        partition_tokens < 0)
+        return 0;
+    return resolve_partition_tokens(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                    max_context, dtype, partition_tokens);
 }
 
 int paged_attention_decode_ex(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -223,8 +252,8 @@ int paged_attention_decode_ex(void* out, const void* q, const void* k_cache, con
         return PKV_ERR_INVALID;
     const long long max_ctx = (long long)max_blocks_per_seq * block_size;
     if (max_ctx > INT_MAX) return PKV_ERR_INVALID;
-    const int pt = partition_tokens == 0 ? auto_partition_tokens(num_seqs, num_kv_heads, max_ctx)
-                                         : partition_tokens;
+    const int pt = resolve_partition_tokens(num_seqs, num_heads, num_kv_heads, head_dim,
+                                            block_size, max_ctx, dtype, partition_tokens);
     const long long parts = (max_ctx + pt - 1) / pt;
     const long long grid = parts * num_kv_heads * (long long)num_seqs;
     if (grid > INT_MAX || (long long)num_seqs * num_heads > INT_MAX) return PKV_ERR_INVALID;

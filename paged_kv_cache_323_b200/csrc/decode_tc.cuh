@@ -303,36 +303,39 @@ __global__ void __launch_bounds__(192, 2)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            for (int li = 0; li < 2 * nchunks; ++li) {
-                const int c = li >> 1;
-                const CUtensorMap* map = (li & 1) ? &tmv : &tmk;
-                const int st = li % C::NSLOT;
-                if (li >= C::NSLOT &&
-                    !mbar_wait_bounded(&empty[st], ((li / C::NSLOT) - 1) & 1, abort_flag)) {
-                    set_error(p.err, PKV_ERR_TIMEOUT);
-                    *abort_flag = 1;
+        // The whole warp: lane j issues the copies of block j of the chunk, so
+        // the (up to 16) TMA issues of a chunk do not serialise on one thread.
+        for (int li = 0; li < 2 * nchunks; ++li) {
+            const int c = li >> 1;
+            const CUtensorMap* map = (li & 1) ? &tmv : &tmk;
+            const int st = li % C::NSLOT;
+            if (li >= C::NSLOT) {
+                const bool ready = mbar_wait_bounded(&empty[st], ((li / C::NSLOT) - 1) & 1, abort_flag);
+                if (!__all_sync(0xffffffffu, ready)) {
+                    if (lane == 0) {
+                        set_error(p.err, PKV_ERR_TIMEOUT);
+                        *abort_flag = 1;
+                    }
                     break;
                 }
-                const int jb0 = c * C::BPT;
-                const int jb1 = min(jb0 + C::BPT, nblk);
-                int nload = 0;
-                for (int j = jb0; j < jb1; ++j) nload += phys[j] >= 0;
-                unsigned char* slot = smem + st * C::SLOT;
-                if (nload > 0) {
-                    mbar_arrive_expect_tx(&full[st], (uint32_t)(nload * BS * 2 * C::ROW));
-                    for (int j = jb0; j < jb1; ++j) {
-                        const int e = phys[j];
-                        if (e < 0) continue;
-                        unsigned char* dst = slot + (j - jb0) * BS * C::ROW;
-                        tma_load_4d(dst, map, 0, 0, g, e, &full[st]);
-                        tma_load_4d(dst + C::HALF, map, 64, 0, g, e, &full[st]);
-                    }
-                } else {
-                    mbar_arrive(&full[st]);
-                }
-                issued = li + 1;
             }
+            const int jb0 = c * C::BPT;
+            const int j = jb0 + lane;
+            const int e = (lane < C::BPT && j < nblk) ? phys[j] : -1;
+            const int nload = __popc(__ballot_sync(0xffffffffu, e >= 0));
+            if (lane == 0) {
+                if (nload > 0)
+                    mbar_arrive_expect_tx(&full[st], (uint32_t)(nload * BS * 2 * C::ROW));
+                else
+                    mbar_arrive(&full[st]);
+            }
+            __syncwarp();  // the expected byte count is registered before any copy lands
+            if (e >= 0) {
+                unsigned char* dst = smem + st * C::SLOT + lane * BS * C::ROW;
+                tma_load_4d(dst, map, 0, 0, g, e, &full[st]);
+                tma_load_4d(dst + C::HALF, map, 64, 0, g, e, &full[st]);
+            }
+            issued = li + 1;
         }
     } else if (warp == 1) {
         // --------------------------------------------------------- MMA issuer

@@ -59,8 +59,8 @@ int scratch_address(void** out) {
 // merge counters for the partition size paged_attention_decode_ex picks.
 extern "C" void pkv_internal_decode_scratch(int num_seqs, int num_heads, int num_kv_heads,
                                             int head_dim, int block_size, int max_blocks_per_seq,
-                                            int partition_tokens, size_t* total, size_t* cnt_off,
-                                            size_t* cnt_bytes);
+                                            int dtype, int partition_tokens, size_t* total,
+                                            size_t* cnt_off, size_t* cnt_bytes);
 
 extern "C" PKV_API int paged_attention_decode_noalloc(
     void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -76,7 +76,8 @@ extern "C" PKV_API int paged_attention_decode_noalloc(
     if (max_ctx > INT_MAX) return PKV_ERR_INVALID;
     size_t need = 0, cnt_off = 0, cnt_bytes = 0;
     pkv_internal_decode_scratch(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
-                                max_blocks_per_seq, partition_tokens, &need, &cnt_off, &cnt_bytes);
+                                max_blocks_per_seq, dtype, partition_tokens, &need, &cnt_off,
+                                &cnt_bytes);
     // a batch whose split-K scratch exceeds the fixed array is refused, never truncated
     if (need > (size_t)PKV_NOALLOC_SCRATCH_BYTES) return PKV_ERR_WORKSPACE;
     void* scratch = nullptr;

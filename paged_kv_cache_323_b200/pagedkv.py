@@ -47,7 +47,7 @@ SIGNATURES = {
     "paged_attention_decode_ex": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float,
                                        _I, _I, _I, _P, _SZ, _P]),
     "paged_attention_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
-    "paged_attention_partition_tokens": (_I, [_I, _I, _I, _I]),
+    "paged_attention_partition_tokens": (_I, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "paged_attention_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
                                             ctypes.c_float, _I, _I, _I, _P]),
     "kv_cache_append": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
@@ -114,9 +114,11 @@ def paged_attention_workspace_size(num_seqs: int, num_heads: int, max_context: i
                                                   partition_tokens))
 
 
-def paged_attention_partition_tokens(num_seqs: int, num_kv_heads: int, max_context: int,
-                                     partition_tokens: int = 0) -> int:
-    return int(lib.paged_attention_partition_tokens(num_seqs, num_kv_heads, max_context,
+def paged_attention_partition_tokens(num_seqs: int, num_heads: int, num_kv_heads: int,
+                                     head_dim: int, block_size: int, max_context: int,
+                                     dtype: int = PKV_BF16, partition_tokens: int = 0) -> int:
+    return int(lib.paged_attention_partition_tokens(num_seqs, num_heads, num_kv_heads, head_dim,
+                                                    block_size, max_context, dtype,
                                                     partition_tokens))
 
 

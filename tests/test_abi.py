@@ -125,8 +125,17 @@ def test_noalloc_validation(pk):
 
 def test_partition_tokens(pk):
     pt = pk.paged_attention_partition_tokens
-    assert pt(64, 32, 2048, 0) == 1024  # batch-64 MHA: automatic 1024
-    assert pt(64, 32, 2048, 256) == 256  # explicit sizes pass through
-    big = pt(8, 8, 131072, 0)  # long context: fewer, larger partitions
-    assert big > 1024 and big <= 4096 and 131072 // big <= 64
-    assert pt(0, 8, 1024, 0) == 0
+    bf = pk.PKV_BF16
+    assert pt(64, 32, 32, 128, 16, 2048, bf, 0) == 1024  # batch-64 MHA, CUDA-core kernel
+    assert pt(64, 32, 32, 128, 16, 2048, bf, 256) == 256  # explicit sizes pass through
+    # grouped-query heads on the tensor-core kernel: long partitions unless the grid gets small
+    assert pt(256, 32, 8, 128, 16, 8256, bf, 0) == 4096
+    assert pt(8, 64, 8, 128, 32, 131072, bf, 0) == 2048
+    assert pt(1, 32, 8, 128, 16, 1024, bf, 0) == 512
+    prev = pk.set_tensor_core_gqa(False)
+    try:
+        big = pt(8, 64, 8, 128, 32, 131072, bf, 0)  # CUDA-core kernel: fewer, larger partitions
+        assert 1024 < big <= 4096 and 131072 // big <= 64
+    finally:
+        pk.set_tensor_core_gqa(prev)
+    assert pt(0, 8, 8, 128, 16, 1024, bf, 0) == 0
