@@ -89,7 +89,8 @@ def kernel_source_sha() -> str:
 
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_323_b200", "csrc")
-    for name in ("common.cuh", "decode_attn.cuh", "decode_launch.cuh"):  # the decode kernel's source
+    for name in ("common.cuh", "decode_attn.cuh", "decode_launch.cuh", "decode_tc.cuh",
+                 "decode_tc.cu"):  # the decode kernels' source
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -371,32 +372,67 @@ def run_gpu(args, world, rank, local):
     pk.profile_reset()
 
     # -------------------------------------------- end to end from host memory
+    # Every step uploads its inputs (q, new K/V, slots, tables, lengths) from
+    # pinned host memory and reads its output back.  Uploads and read-backs
+    # run on a copy stream with double-buffered device staging, so step i+1's
+    # upload and step i-1's read-back overlap step i's kernels; the KV pool
+    # stays resident (it is the cache itself).
+    names = ("q", "k_new", "v_new", "bt", "ctx", "slots")
     host = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True).copy_(v)
-            for k, v in zip(("q", "k_new", "v_new", "bt", "ctx", "slots"), dev_args)}
-    staged = {k: torch.empty_like(v) for k, v in zip(("q", "k_new", "v_new", "bt", "ctx", "slots"),
-                                                      dev_args)}
-    out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+            for k, v in zip(names, dev_args)}
+    staged = [{k: torch.empty_like(v) for k, v in zip(names, dev_args)} for _ in range(2)]
+    outs = [torch.empty_like(out) for _ in range(2)]
+    out_host = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = out_host.numel() * out_host.element_size()
+    d2h = out_host[0].numel() * out_host[0].element_size()
+    up_stream = torch.cuda.Stream()    # host -> device
+    down_stream = torch.cuda.Stream()  # device -> host
+    ev_up = [torch.cuda.Event() for _ in range(2)]     # inputs of buffer b uploaded
+    ev_used = [torch.cuda.Event() for _ in range(2)]   # step on buffer b finished
+    ev_back = [torch.cuda.Event() for _ in range(2)]   # output of buffer b read back
 
-    def e2e_step():
-        for k in staged:
-            staged[k].copy_(host[k], non_blocking=True)
-        step(staged["q"], staged["k_new"], staged["v_new"], staged["bt"], staged["ctx"],
-             staged["slots"])
-        out_host.copy_(out, non_blocking=True)
+    def upload(b):
+        with torch.cuda.stream(up_stream):
+            for k in names:
+                staged[b][k].copy_(host[k], non_blocking=True)
+            ev_up[b].record(up_stream)
 
-    for _ in range(args.warmup):
-        e2e_step()
+    def e2e_run(n):
+        nonlocal out
+        keep = out
+        upload(0)
+        for i in range(n):
+            b = i % 2
+            if i + 1 < n:
+                if i >= 1:
+                    up_stream.wait_event(ev_used[1 - b])  # step i-1 is done with buffer 1-b
+                upload(1 - b)
+            stream.wait_event(ev_up[b])
+            if i >= 2:
+                stream.wait_event(ev_back[b])  # outs[b] was read back
+            out = outs[b]
+            sb = staged[b]
+            step(sb["q"], sb["k_new"], sb["v_new"], sb["bt"], sb["ctx"], sb["slots"])
+            ev_used[b].record(stream)
+            down_stream.wait_event(ev_used[b])
+            with torch.cuda.stream(down_stream):
+                out_host[b].copy_(outs[b], non_blocking=True)
+                ev_back[b].record(down_stream)
+        stream.wait_stream(up_stream)
+        stream.wait_stream(down_stream)
+        out = keep
+
+    e2e_run(args.warmup)
     barrier(world)
     torch.cuda.synchronize()
     ev0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    e2e_run(args.steps)
     ev1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     ms_e2e = max_over_ranks(world, ev0.elapsed_time(ev1))
+    if not torch.equal(out_host[(args.steps - 1) % 2], out.cpu()):
+        raise RuntimeError("end-to-end output differs from the device-resident run")
     code = pk.get_device_error()
     if code != 0:
         raise RuntimeError(f"device error word {code} after the timed steps")
