@@ -47,12 +47,25 @@ WORKLOADS = {
     "prefix_bs32": ("prefix_sweep_b1024_prefix2048_h32_kv8_d128_bs32_bf16",
                     lambda dev, seed: wl.prefix_sweep(32, seed=seed, device=dev)),
     "tiny": ("tiny_b4_ctx35-16-1-50_h4_d64_bs16_f32", lambda dev, seed: wl.tiny(seed=seed, device=dev)),
+    # the gather's cost: the same MHA batch at block sizes 8 / 16 / 32, blocks placed at random
+    # (paged) or consecutively per sequence (the layout of a contiguous per-request cache)
+    "mha_bs8": ("mha_decode_b64_h32_kv32_d128_bs8_ctxU128-2048_bf16",
+                lambda dev, seed: wl.mha(seed=seed, device=dev, block_size=8)),
+    "mha_bs32": ("mha_decode_b64_h32_kv32_d128_bs32_ctxU128-2048_bf16",
+                 lambda dev, seed: wl.mha(seed=seed, device=dev, block_size=32)),
+    "mha_contig_bs8": ("mha_decode_b64_h32_kv32_d128_bs8_contiguous_bf16",
+                       lambda dev, seed: wl.mha(seed=seed, device=dev, block_size=8, contiguous=True)),
+    "mha_contig_bs16": ("mha_decode_b64_h32_kv32_d128_bs16_contiguous_bf16",
+                        lambda dev, seed: wl.mha(seed=seed, device=dev, contiguous=True)),
+    "mha_contig_bs32": ("mha_decode_b64_h32_kv32_d128_bs32_contiguous_bf16",
+                        lambda dev, seed: wl.mha(seed=seed, device=dev, block_size=32, contiguous=True)),
     # a smaller MHA batch for profiler captures: 16 sequences, 4096-block pool (1 GB), ~0.3 GB KV per step
     "mha_small": ("mha_decode_b16_h32_kv32_d128_bs16_ctxU128-2048_bf16_pool4096",
                   lambda dev, seed: wl.mha(seed=seed, device=dev, num_seqs=16, num_blocks=4096)),
 }
 DEFAULT_SEED = {"mha": 2, "gqa_sampling": 3, "long_context": 4, "prefix_bs8": 5, "prefix_bs16": 5,
-                "prefix_bs32": 5, "tiny": 1, "mha_small": 2}
+                "prefix_bs32": 5, "tiny": 1, "mha_small": 2, "mha_bs8": 2, "mha_bs32": 2,
+                "mha_contig_bs8": 2, "mha_contig_bs16": 2, "mha_contig_bs32": 2}
 
 
 def measured_peak():
@@ -272,6 +285,36 @@ def pick_sample(w: wl.Workload, target_s: float, threads: int):
     return sub, n, dt
 
 
+def measure_swap(pk, w, stream, nblocks: int = 1024, reps: int = 5) -> dict:
+    """Preemption by swapping: host-link bandwidth of swap_blocks moving
+    `nblocks` whole blocks of the pool to a pinned host pool and back (CUDA
+    events on the launch stream, best of `reps`)."""
+    nblocks = min(nblocks, w.num_blocks)
+    shape = (nblocks,) + tuple(w.k_cache.shape[1:])
+    hk = torch.empty(shape, dtype=w.k_cache.dtype, pin_memory=True)
+    hv = torch.empty(shape, dtype=w.k_cache.dtype, pin_memory=True)
+    rng = np.random.default_rng(99)
+    dev_blocks = torch.from_numpy(rng.choice(w.num_blocks, nblocks, replace=False).astype(np.int64))
+    host_blocks = torch.arange(nblocks, dtype=torch.int64)
+    out_pairs = torch.stack([dev_blocks, host_blocks], 1).cuda()
+    in_pairs = torch.stack([host_blocks, dev_blocks], 1).cuda()
+    nbytes = 2 * nblocks * w.k_cache[0].numel() * w.k_cache.element_size()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    res = {}
+    for name, args in (("device_to_host", (hk, hv, w.k_cache, w.v_cache, out_pairs)),
+                       ("host_to_device", (w.k_cache, w.v_cache, hk, hv, in_pairs))):
+        best = float("inf")
+        for _ in range(reps):
+            e0.record(stream)
+            pk.swap_blocks(*args)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        res[name + "_gbs"] = nbytes / (best * 1e-3) / 1e9
+    res.update({"blocks": nblocks, "bytes": nbytes, "unit": "GB/s"})
+    return res
+
+
 def cpu_threads() -> int:
     try:
         return len(os.sched_getaffinity(0))
@@ -344,9 +387,11 @@ def run_gpu(args, world, rank, local):
         raise RuntimeError(f"device error word {code} after warm-up")
 
     # ------------------------------------------------ device-resident timing
+    # The headline region runs the steps bare.  Per-kernel durations come from
+    # a second region of the same steps in which the library brackets every
+    # launch with CUDA events on its stream (those events cost a few percent
+    # of the step, so they stay out of the headline).
     clocks = ClockSampler(torch.cuda.current_device())
-    pk.profile_reset()
-    pk.profile_enable(True)
     barrier(world)
     torch.cuda.synchronize()
     clocks.start()
@@ -359,10 +404,20 @@ def run_gpu(args, world, rank, local):
     ev1.record(stream)
     torch.cuda.synchronize()
     launches = pk.launch_count() - launches0
-    clock_info = clocks.stop()
-    pk.profile_enable(False)
     barrier(world)
     ms = max_over_ranks(world, ev0.elapsed_time(ev1))
+
+    pk.profile_reset()
+    pk.profile_enable(True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step(*dev_args)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    pk.profile_enable(False)
+    clock_info = clocks.stop()
+    barrier(world)
+    ms_profiled = max_over_ranks(world, ev0.elapsed_time(ev1))
     per_kernel = {}
     for kind, kname in ((pk.KERNEL_DECODE, "decode"), (pk.KERNEL_APPEND, "kv_append"),
                         (pk.KERNEL_COPY_BLOCKS, "copy_blocks")):
@@ -468,6 +523,7 @@ def run_gpu(args, world, rank, local):
         "tokens_per_s": world * w.num_seqs / step_s,
         "pct_of_peak_hbm": 100.0 * value / peak,
         "per_kernel_us": per_kernel,
+        "ms_per_step_profiled": ms_profiled / args.steps,
         "roofline": roofline,
         "gpu_launches": launches,
         "e2e": {"value": job_value(world, kv_bytes, ms_e2e / args.steps), "unit": "GB/s",
@@ -475,6 +531,8 @@ def run_gpu(args, world, rank, local):
                 "ms_per_step": ms_e2e / args.steps},
         "clocks": clock_info,
     }
+    if world == 1:
+        line["swap"] = measure_swap(pk, w, stream)
     if world == 1 and not args.no_cpu_baseline:
         # the oracle as it stands, on this host's cores: a seeded sample of the
         # batch, stepped repeatedly for about 10 s of CPU time

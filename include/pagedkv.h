@@ -70,7 +70,8 @@ typedef enum {
     PKV_ERR_CUDA = -4,          /* the CUDA runtime reported an error */
     PKV_ERR_WORKSPACE = -5,     /* split-K workspace missing or too small */
     PKV_ERR_DEVICE_BOUNDS = -6, /* device word: a table entry, slot or length was out of range */
-    PKV_ERR_TIMEOUT = -7        /* device word: a bounded wait in a kernel ran out */
+    PKV_ERR_TIMEOUT = -7,       /* device word: a bounded wait in a kernel ran out */
+    PKV_ERR_OUT_OF_BLOCKS = -8  /* block manager: the free list cannot cover the request */
 } pkv_status;
 
 /* Element types of q, out, the pools and the new tokens. */
@@ -81,7 +82,8 @@ typedef enum {
     PKV_KERNEL_DECODE = 0, /* table walk, gather, QK^T, online softmax, PV, fused split-K merge */
     PKV_KERNEL_APPEND = 1,
     PKV_KERNEL_COPY_BLOCKS = 2,
-    PKV_KERNEL_KINDS = 3
+    PKV_KERNEL_SWAP_BLOCKS = 3,
+    PKV_KERNEL_KINDS = 4
 } pkv_kernel_kind;
 
 /*
@@ -202,6 +204,24 @@ PKV_API int paged_attention_decode_noalloc(void* out, const void* q, const void*
                                            int block_size, int max_blocks_per_seq, float scale,
                                            int num_blocks, int dtype, int partition_tokens,
                                            void* stream);
+
+/*
+ * Preemption by swapping ("Preemption and scheduling": move a sequence's
+ * blocks to CPU memory and bring them back later): for each pair (src, dst)
+ * of src_dst_pairs (int64 [num_pairs][2]), block src of the source pools
+ * (src_k, src_v: [num_src_blocks][num_kv_heads][block_size][head_dim]) is
+ * copied whole to block dst of the destination pools (same layout,
+ * num_dst_blocks blocks).  Any pool and the pairs may be device memory or
+ * page-locked (pinned) host memory; the copy is one kernel on `stream` that
+ * reads or writes host pools over the host link through their device
+ * mapping.  Pageable host memory is PKV_ERR_INVALID.  Bit-exact.  Indices
+ * outside the pools are device faults (pair skipped).  Destinations must be
+ * distinct and no destination may also be a source.
+ */
+PKV_API int swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                        const int64_t* src_dst_pairs, int num_pairs, int num_kv_heads,
+                        int head_dim, int block_size, int num_src_blocks, int num_dst_blocks,
+                        int dtype, void* stream);
 
 /* Synchronise `stream`, then return in *code the current device's error word
  * (PKV_OK, PKV_ERR_DEVICE_BOUNDS or PKV_ERR_TIMEOUT) and clear it. */

@@ -22,6 +22,7 @@ from .binding import (  # noqa: F401
     library_path,
     open_library,
     paged_attention,
+    swap_blocks,
     use_library,
     waste_per_sequence,
     waste_physical,

@@ -58,6 +58,7 @@ def open_library(path: str):
     lib.oracle_paged_attention.restype = i32
     lib.oracle_kv_append.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32]
     lib.oracle_copy_blocks.argtypes = [P, P, P, i32, i32, i32, i32, i32]
+    lib.oracle_swap_blocks.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32]
     return lib
 
 
@@ -178,3 +179,15 @@ def copy_blocks(k_cache: np.ndarray, v_cache: np.ndarray, pairs) -> None:
     _, hkv, bs, d = k_cache.shape
     _load().oracle_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(pairs), pairs.shape[0], hkv, d,
                                bs, code)
+
+
+def swap_blocks(dst_k: np.ndarray, dst_v: np.ndarray, src_k: np.ndarray, src_v: np.ndarray,
+                pairs) -> None:
+    """In place on the destination pools."""
+    pairs = np.ascontiguousarray(pairs, dtype=np.int64).reshape(-1, 2)
+    code = _dtype_code(src_k)
+    assert dst_k.dtype == src_k.dtype and dst_k.shape[1:] == src_k.shape[1:]
+    _, hkv, bs, d = src_k.shape
+    _load().oracle_swap_blocks(_ptr(dst_k), _ptr(dst_v), _ptr(np.ascontiguousarray(src_k)),
+                               _ptr(np.ascontiguousarray(src_v)), _ptr(pairs), pairs.shape[0], hkv,
+                               d, bs, code)

@@ -314,3 +314,22 @@ void oracle_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs,
                 (size_t)block_bytes);
     }
 }
+
+/* Preemption by swapping ("PagedAttention Explained: Virtual Memory for the
+ * KV Cache", section "Preemption and scheduling": a sequence's blocks move to
+ * CPU memory and come back later): for each (src, dst) pair, the whole block
+ * src of the source pools is copied to block dst of the destination pools. */
+void oracle_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                        const int64_t* pairs, int num_pairs, int num_kv_heads, int head_dim,
+                        int block_size, int dtype) {
+    /* one block: every kv head, every slot, every dimension */
+    const int64_t block_bytes = (int64_t)elem_bytes(dtype) * head_dim * block_size * num_kv_heads;
+    for (int i = 0; i < num_pairs; ++i) {
+        const int64_t src = pairs[2 * i];     /* block in the source pools */
+        const int64_t dst = pairs[2 * i + 1]; /* block in the destination pools */
+        memcpy((char*)dst_k + dst * block_bytes, (const char*)src_k + src * block_bytes,
+               (size_t)block_bytes);
+        memcpy((char*)dst_v + dst * block_bytes, (const char*)src_v + src * block_bytes,
+               (size_t)block_bytes);
+    }
+}

@@ -17,7 +17,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpagedkv.so")
-SOURCES = ["api.cu", "decode_f32.cu", "decode_bf16.cu", "decode_tc.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "decode_f32.cu", "decode_bf16.cu", "decode_tc.cu", "noalloc.cu",
+           "block_manager.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + [
     "-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
@@ -51,8 +52,12 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     extra = ["-Xptxas", "-v"] if verbose_ptxas else []
 
     def compile_one(src: str) -> str:
-        obj = os.path.join(BUILD, src.replace(".cu", ".o"))
-        cmd = [nvcc()] + NVCC_FLAGS + extra + ["-c", os.path.join(CSRC, src), "-o", obj]
+        obj = os.path.join(BUILD, os.path.splitext(src)[0] + ".o")
+        if src.endswith(".cpp"):  # host-only C++: the host compiler through nvcc's flags
+            cmd = [nvcc(), "-x", "c++", "-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler",
+                   "-fvisibility=hidden", "-c", os.path.join(CSRC, src), "-o", obj]
+        else:
+            cmd = [nvcc()] + NVCC_FLAGS + extra + ["-c", os.path.join(CSRC, src), "-o", obj]
         p = subprocess.run(cmd, capture_output=True, text=True)
         log = os.path.join(BUILD, src + ".log")
         with open(log, "w") as f:

@@ -390,18 +390,77 @@ int copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_pairs, int 
     int* err = nullptr;
     if (error_word(dev, &err) != PKV_OK) return PKV_ERR_CUDA;
     pkv::CopyParams p;
-    p.k_cache = k_cache;
-    p.v_cache = v_cache;
+    p.dst_k = k_cache;
+    p.dst_v = v_cache;
+    p.src_k = k_cache;
+    p.src_v = v_cache;
     p.pairs = src_dst_pairs;
     p.err = err;
     p.chunks_per_block = block_bytes / 16;
     p.num_pairs = num_pairs;
-    p.num_blocks = num_blocks;
+    p.num_src_blocks = num_blocks;
+    p.num_dst_blocks = num_blocks;
     long long per_pair = (p.chunks_per_block + 1023) / 1024;  // 256 threads x 4 chunks
     if (per_pair > 64) per_pair = 64;
     if (num_pairs > 65535) return PKV_ERR_INVALID;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return launch(PKV_KERNEL_COPY_BLOCKS, st, [&] {
+        pkv::copy_blocks_kernel<<<dim3((unsigned)per_pair, (unsigned)num_pairs), 256, 0, st>>>(p);
+        return cudaGetLastError();
+    });
+}
+
+int swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                const int64_t* src_dst_pairs, int num_pairs, int num_kv_heads, int head_dim,
+                int block_size, int num_src_blocks, int num_dst_blocks, int dtype, void* stream) {
+    if (num_pairs < 0) return PKV_ERR_INVALID;
+    if (num_pairs == 0) return PKV_OK;
+    if (!dst_k || !dst_v || !src_k || !src_v || !src_dst_pairs) return PKV_ERR_NULL;
+    if (num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_src_blocks <= 0 ||
+        num_dst_blocks <= 0 || num_pairs > 65535)
+        return PKV_ERR_INVALID;
+    if (dtype != PKV_F32 && dtype != PKV_BF16) return PKV_ERR_INVALID;
+    const long long block_bytes = (long long)num_kv_heads * block_size * head_dim * elt_bytes(dtype);
+    if (block_bytes % 16 != 0) return PKV_ERR_UNSUPPORTED;
+    // every pointer must be device memory or page-locked host memory the
+    // device can reach; host pointers are replaced by their device mapping
+    const void* ptrs[5] = {dst_k, dst_v, src_k, src_v, src_dst_pairs};
+    void* mapped[5];
+    for (int i = 0; i < 5; ++i) {
+        cudaPointerAttributes a;
+        if (cudaPointerGetAttributes(&a, ptrs[i]) != cudaSuccess) {
+            cudaGetLastError();
+            return PKV_ERR_INVALID;
+        }
+        if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) {
+            mapped[i] = const_cast<void*>(ptrs[i]);
+        } else if (a.type == cudaMemoryTypeHost && a.devicePointer != nullptr) {
+            mapped[i] = static_cast<char*>(a.devicePointer) +
+                        (static_cast<const char*>(ptrs[i]) - static_cast<const char*>(a.hostPointer));
+        } else {
+            return PKV_ERR_INVALID;  // pageable host memory: pin it first
+        }
+        if (i < 4 && (reinterpret_cast<uintptr_t>(mapped[i]) & 15u) != 0) return PKV_ERR_INVALID;
+    }
+    int dev = 0;
+    if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
+    int* err = nullptr;
+    if (error_word(dev, &err) != PKV_OK) return PKV_ERR_CUDA;
+    pkv::CopyParams p;
+    p.dst_k = mapped[0];
+    p.dst_v = mapped[1];
+    p.src_k = mapped[2];
+    p.src_v = mapped[3];
+    p.pairs = static_cast<const int64_t*>(mapped[4]);
+    p.err = err;
+    p.chunks_per_block = block_bytes / 16;
+    p.num_pairs = num_pairs;
+    p.num_src_blocks = num_src_blocks;
+    p.num_dst_blocks = num_dst_blocks;
+    long long per_pair = (p.chunks_per_block + 1023) / 1024;
+    if (per_pair > 64) per_pair = 64;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return launch(PKV_KERNEL_SWAP_BLOCKS, st, [&] {
         pkv::copy_blocks_kernel<<<dim3((unsigned)per_pair, (unsigned)num_pairs), 256, 0, st>>>(p);
         return cudaGetLastError();
     });
@@ -432,6 +491,7 @@ const char* pkv_status_string(int status) {
         case PKV_ERR_WORKSPACE: return "split-K workspace missing or too small";
         case PKV_ERR_DEVICE_BOUNDS: return "device: table entry, slot or context length out of range";
         case PKV_ERR_TIMEOUT: return "device: a bounded wait ran out of time";
+        case PKV_ERR_OUT_OF_BLOCKS: return "no free block left in the pool (preempt and retry)";
         default: return "unknown status";
     }
 }

@@ -68,29 +68,34 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
 }
 
 struct CopyParams {
-    void* k_cache;
-    void* v_cache;
+    void* dst_k;
+    void* dst_v;
+    const void* src_k;
+    const void* src_v;
     const int64_t* pairs;
     int* err;
     long long chunks_per_block;  // num_kv_heads * block_size * head_dim * elt / 16
     int num_pairs;
-    int num_blocks;
+    int num_src_blocks;
+    int num_dst_blocks;
 };
 
-// gridDim.y = pairs; gridDim.x CTAs share one pair's block, 4 chunks per
-// thread in flight for K and for V.
+// One pair per gridDim.y row; gridDim.x CTAs share one pair's block, 4
+// chunks per thread in flight for K and for V.  Serves copy-on-write (source
+// and destination in the same device pool) and swapping (one side in a
+// pinned host pool, reached through its device-mapped address).
 __global__ void __launch_bounds__(256) copy_blocks_kernel(const CopyParams p) {
     const int pair = blockIdx.y;
     const long long src = p.pairs[2 * pair];
     const long long dst = p.pairs[2 * pair + 1];
-    if (src < 0 || src >= p.num_blocks || dst < 0 || dst >= p.num_blocks) {
+    if (src < 0 || src >= p.num_src_blocks || dst < 0 || dst >= p.num_dst_blocks) {
         if (blockIdx.x == 0 && threadIdx.x == 0) set_error(p.err, PKV_ERR_DEVICE_BOUNDS);
         return;
     }
-    const uint4* ks = static_cast<const uint4*>(p.k_cache) + src * p.chunks_per_block;
-    const uint4* vs = static_cast<const uint4*>(p.v_cache) + src * p.chunks_per_block;
-    uint4* kd = static_cast<uint4*>(p.k_cache) + dst * p.chunks_per_block;
-    uint4* vd = static_cast<uint4*>(p.v_cache) + dst * p.chunks_per_block;
+    const uint4* ks = static_cast<const uint4*>(p.src_k) + src * p.chunks_per_block;
+    const uint4* vs = static_cast<const uint4*>(p.src_v) + src * p.chunks_per_block;
+    uint4* kd = static_cast<uint4*>(p.dst_k) + dst * p.chunks_per_block;
+    uint4* vd = static_cast<uint4*>(p.dst_v) + dst * p.chunks_per_block;
     constexpr int U = 4;
     const long long stride = (long long)gridDim.x * blockDim.x;
     for (long long base = blockIdx.x * (long long)blockDim.x + threadIdx.x; base < p.chunks_per_block;

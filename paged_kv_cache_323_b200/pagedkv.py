@@ -31,11 +31,13 @@ PKV_ERR_CUDA = -4
 PKV_ERR_WORKSPACE = -5
 PKV_ERR_DEVICE_BOUNDS = -6
 PKV_ERR_TIMEOUT = -7
+PKV_ERR_OUT_OF_BLOCKS = -8
 PKV_F32 = 0
 PKV_BF16 = 1
 KERNEL_DECODE = 0
 KERNEL_APPEND = 1
 KERNEL_COPY_BLOCKS = 2
+KERNEL_SWAP_BLOCKS = 3
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -52,6 +54,19 @@ SIGNATURES = {
                                             ctypes.c_float, _I, _I, _I, _P]),
     "kv_cache_append": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     "copy_blocks": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
+    "swap_blocks": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
+    "pkv_bm_create": (_P, [_I, _I, _I, _P]),
+    "pkv_bm_destroy": (None, [_P]),
+    "pkv_bm_add_sequence": (_I, [_P]),
+    "pkv_bm_fork": (_I, [_P, _I]),
+    "pkv_bm_append": (_I, [_P, _I, _I, _P, _P, _I, ctypes.POINTER(_I)]),
+    "pkv_bm_free": (_I, [_P, _I]),
+    "pkv_bm_tables": (_I, [_P, _P, _I, _I, _P, _P]),
+    "pkv_bm_length": (_I, [_P, _I]),
+    "pkv_bm_pick_victim": (_I, [_P]),
+    "pkv_bm_swap_out": (_I, [_P, _I, _P, _I, ctypes.POINTER(_I)]),
+    "pkv_bm_swap_in": (_I, [_P, _I, _P, _I, ctypes.POINTER(_I)]),
+    "pkv_bm_get_stats": (_I, [_P, _P]),
     "pkv_get_device_error": (_I, [_P, ctypes.POINTER(_I)]),
     "pkv_status_string": (ctypes.c_char_p, [_I]),
     "pkv_profile_enable": (_I, [_I]),
@@ -215,6 +230,126 @@ def copy_blocks(k_cache, v_cache, src_dst_pairs, stream=None) -> None:
         _dev(src_dst_pairs, "src_dst_pairs", torch.int64) if n else None, n, Hkv, D, bs, N,
         _dtype_code(k_cache), _stream(stream))
     _check(rc, "copy_blocks")
+
+
+def _reachable(t: torch.Tensor, name: str, dtype=None) -> int:
+    """Pointer of a device tensor or of a pinned host tensor (swap pools)."""
+    if not (t.is_cuda or t.is_pinned()):
+        raise ValueError(f"{name} must be a CUDA tensor or pinned host memory")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def swap_blocks(dst_k, dst_v, src_k, src_v, src_dst_pairs, stream=None) -> None:
+    """Copy whole blocks between pools, either of which may be pinned host
+    memory (preemption by swapping); src_dst_pairs int64 [n][2]."""
+    n = src_dst_pairs.shape[0]
+    Ns, Hkv, bs, D = src_k.shape
+    Nd = dst_k.shape[0]
+    if tuple(dst_k.shape[1:]) != (Hkv, bs, D):
+        raise ValueError("source and destination pools must share the block layout")
+    rc = lib.swap_blocks(
+        _reachable(dst_k, "dst_k"), _reachable(dst_v, "dst_v", dst_k.dtype),
+        _reachable(src_k, "src_k", dst_k.dtype), _reachable(src_v, "src_v", dst_k.dtype),
+        _reachable(src_dst_pairs, "src_dst_pairs", torch.int64) if n else None, n, Hkv, D, bs, Ns,
+        Nd, _dtype_code(dst_k), _stream(stream))
+    _check(rc, "swap_blocks")
+
+
+class _BmStats(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_int64) for name in (
+        "num_blocks", "free_blocks", "used_blocks", "allocated_slots", "used_slots",
+        "logical_allocated", "logical_used", "live_sequences", "swapped_sequences",
+        "host_free_blocks", "preemptions", "copy_on_write")]
+
+
+class BlockManager:
+    """The native block manager (include/pkv_block_manager.h): free lists,
+    block tables, refcounts, forks, copy-on-write pairs, swapping, counters."""
+
+    def __init__(self, num_blocks: int, block_size: int, num_host_blocks: int = 0, free_order=None):
+        import numpy as np
+
+        self._np = np
+        order = None
+        if free_order is not None:
+            order = np.ascontiguousarray(free_order, dtype=np.int32)
+        self.block_size = block_size
+        self._h = lib.pkv_bm_create(num_blocks, block_size, num_host_blocks,
+                                    order.ctypes.data if order is not None else None)
+        if not self._h:
+            raise ValueError("pkv_bm_create rejected its arguments")
+
+    def close(self) -> None:
+        if self._h:
+            lib.pkv_bm_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()
+
+    def _id(self, rc: int, where: str) -> int:
+        if rc < 0:
+            raise PagedKVError(rc, where)
+        return rc
+
+    def add_sequence(self) -> int:
+        return self._id(lib.pkv_bm_add_sequence(self._h), "pkv_bm_add_sequence")
+
+    def fork(self, parent: int) -> int:
+        return self._id(lib.pkv_bm_fork(self._h, parent), "pkv_bm_fork")
+
+    def append(self, seq: int, n: int):
+        """Slots of n new tokens (int64 [n]) and copy-on-write pairs (int64 [k][2])."""
+        np = self._np
+        slots = np.empty(max(n, 1), dtype=np.int64)
+        pairs = np.empty((1, 2), dtype=np.int64)
+        k = ctypes.c_int(0)
+        _check(lib.pkv_bm_append(self._h, seq, n, slots.ctypes.data, pairs.ctypes.data, 1,
+                                 ctypes.byref(k)), "pkv_bm_append")
+        return slots[:n].copy(), pairs[: k.value].copy()
+
+    def free(self, seq: int) -> None:
+        _check(lib.pkv_bm_free(self._h, seq), "pkv_bm_free")
+
+    def tables(self, seqs, max_blocks: int):
+        np = self._np
+        seqs = np.ascontiguousarray(seqs, dtype=np.int32)
+        bt = np.empty((len(seqs), max_blocks), dtype=np.int32)
+        lens = np.empty(len(seqs), dtype=np.int32)
+        _check(lib.pkv_bm_tables(self._h, seqs.ctypes.data, len(seqs), max_blocks, bt.ctypes.data,
+                                 lens.ctypes.data), "pkv_bm_tables")
+        return bt, lens
+
+    def length(self, seq: int) -> int:
+        return self._id(lib.pkv_bm_length(self._h, seq), "pkv_bm_length")
+
+    def pick_victim(self) -> int:
+        return int(lib.pkv_bm_pick_victim(self._h))
+
+    def _swap(self, fn, seq: int, where: str):
+        np = self._np
+        cap = 1 << 16
+        pairs = np.empty((cap, 2), dtype=np.int64)
+        k = ctypes.c_int(0)
+        _check(fn(self._h, seq, pairs.ctypes.data, cap, ctypes.byref(k)), where)
+        return pairs[: k.value].copy()
+
+    def swap_out(self, seq: int):
+        """(device_block, host_block) pairs to copy device -> host."""
+        return self._swap(lib.pkv_bm_swap_out, seq, "pkv_bm_swap_out")
+
+    def swap_in(self, seq: int):
+        """(host_block, device_block) pairs to copy host -> device."""
+        return self._swap(lib.pkv_bm_swap_in, seq, "pkv_bm_swap_in")
+
+    def stats(self) -> dict:
+        st = _BmStats()
+        _check(lib.pkv_bm_get_stats(self._h, ctypes.byref(st)), "pkv_bm_get_stats")
+        return {name: int(getattr(st, name)) for name, _ in _BmStats._fields_}
 
 
 def get_device_error(stream=None) -> int:

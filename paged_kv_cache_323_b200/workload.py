@@ -134,9 +134,19 @@ def _finish(name, dtype, rng, seed, device, *, lens, tables, cow_pairs, new_pos,
         v_new=v_new, meta=meta or {})
 
 
-def _private(lens, rng, num_blocks, bs, new_per_seq=1):
+class _InOrderPool(_Pool):
+    """Free list in ascending block order: each sequence's blocks come out
+    consecutive, as with one contiguous reservation per request."""
+
+    def __init__(self, num_blocks: int):
+        self.order = list(range(num_blocks))
+        self.pos = 0
+        self.ref = np.zeros(num_blocks, dtype=np.int64)
+
+
+def _private(lens, rng, num_blocks, bs, new_per_seq=1, contiguous=False):
     """Every sequence owns its blocks; the last ``new_per_seq`` positions are new."""
-    pool = _Pool(rng, num_blocks)
+    pool = _InOrderPool(num_blocks) if contiguous else _Pool(rng, num_blocks)
     tables, new_pos = [], []
     for L in lens:
         nb = -(-int(L) // bs)
@@ -156,12 +166,18 @@ def tiny(seed: int = 1, device="cpu") -> Workload:
 
 
 def mha(seed: int = 2, device="cpu", num_seqs: int = 64, ctx_range=(128, 2048),
-        num_blocks: int = 16384, heads: int = 32, head_dim: int = 128, block_size: int = 16,
-        dtype: str = "bf16") -> Workload:
-    """Batch 64, 32 = 32 heads, d 128, bf16, bs 16, ctx U[128, 2048], pool 16384."""
+        num_blocks: int | None = None, heads: int = 32, head_dim: int = 128, block_size: int = 16,
+        dtype: str = "bf16", contiguous: bool = False) -> Workload:
+    """Batch 64, 32 = 32 heads, d 128, bf16, bs 16, ctx U[128, 2048], pool of
+    16384 blocks (the same 256 Ki tokens at other block sizes).  With
+    ``contiguous`` every sequence's blocks are consecutive in the pool (the
+    layout of a contiguous per-request cache, still read through the table)
+    instead of a seeded random placement."""
     rng = np.random.Generator(np.random.PCG64(seed))
     lens = rng.integers(ctx_range[0], ctx_range[1], size=num_seqs, endpoint=True).tolist()
-    tables, new_pos = _private(lens, rng, num_blocks, block_size)
+    if num_blocks is None:
+        num_blocks = 16384 * 16 // block_size
+    tables, new_pos = _private(lens, rng, num_blocks, block_size, contiguous=contiguous)
     maxb = -(-ctx_range[1] // block_size)
     return _finish("mha", dtype, rng, seed, device, lens=lens, tables=tables, cow_pairs=[],
                    new_pos=new_pos, num_blocks=num_blocks, H=heads, Hkv=heads, D=head_dim,

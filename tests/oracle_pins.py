@@ -427,6 +427,31 @@ def pin_copy_blocks_pairs():
                 assert np.array_equal(kp[p].view(np.uint8), k0[p].view(np.uint8))
 
 
+def pin_swap_round_trip():
+    """Swapping moves whole blocks between pools: out and back in (to other
+    blocks) gives the same bytes; blocks not named stay as they were."""
+    for dtype in ("f32", "bf16"):
+        rng = np.random.default_rng(131)
+        dk = to_dtype(rng.standard_normal((8, 2, 4, 8)).astype(np.float32), dtype)
+        dv = to_dtype(rng.standard_normal((8, 2, 4, 8)).astype(np.float32), dtype)
+        hk = np.zeros((5, 2, 4, 8), dtype=dk.dtype)
+        hv = np.zeros((5, 2, 4, 8), dtype=dk.dtype)
+        k0, v0 = dk.copy(), dv.copy()
+        out_pairs = np.asarray([[6, 0], [1, 3], [4, 4]], dtype=np.int64)
+        oracle.swap_blocks(hk, hv, dk, dv, out_pairs)
+        for d, h in out_pairs:
+            assert np.array_equal(hk[h].view(np.uint8), k0[d].view(np.uint8))
+            assert np.array_equal(hv[h].view(np.uint8), v0[d].view(np.uint8))
+        assert not hk[[1, 2]].any()
+        back = np.asarray([[0, 2], [3, 7], [4, 5]], dtype=np.int64)
+        oracle.swap_blocks(dk, dv, hk, hv, back)
+        for (d, h), (h2, d2) in zip(out_pairs, back):
+            assert np.array_equal(dk[d2].view(np.uint8), k0[d].view(np.uint8))
+            assert np.array_equal(dv[d2].view(np.uint8), v0[d].view(np.uint8))
+        for p in (0, 1, 3, 4, 6):
+            assert np.array_equal(dk[p].view(np.uint8), k0[p].view(np.uint8))
+
+
 PINS = [
     pin_worked_example,
     pin_logical_block_ranges,
@@ -446,4 +471,5 @@ PINS = [
     pin_append_extends_logical,
     pin_copy_on_write,
     pin_copy_blocks_pairs,
+    pin_swap_round_trip,
 ]

@@ -37,6 +37,13 @@ def test_mha_reduced(pt):
     _full_check(w, partition_tokens=pt)
 
 
+@pytest.mark.parametrize("bs", [8, 32])
+def test_mha_contiguous_reduced(bs):
+    """The contiguous-placement comparator computes the same attention."""
+    w = wl.mha(num_seqs=6, num_blocks=2048 * 16 // bs, block_size=bs, contiguous=True)
+    _full_check(w)
+
+
 def test_gqa_sampling_reduced():
     w = wl.gqa_sampling(groups=6, prompt_median=300, prompt_max=2000)
     assert len(w.cow_pairs) > 0

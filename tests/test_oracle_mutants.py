@@ -44,6 +44,8 @@ MUTANTS = {
                        "int64_t dst = pairs[2 * i], src = pairs[2 * i + 1];"),
     "copy_one_head": ("(int64_t)num_kv_heads * block_size * head_dim * elem_bytes(dtype);",
                       "(int64_t)block_size * head_dim * elem_bytes(dtype);"),
+    "swap_direction": ("memcpy((char*)dst_k + dst * block_bytes, (const char*)src_k + src * block_bytes,",
+                       "memcpy((char*)dst_k + src * block_bytes, (const char*)src_k + dst * block_bytes,"),
     "physical_double_count": ("if (here > filled[p]) filled[p] = (int32_t)here;",
                               "filled[p] += (int32_t)here;"),
 }

@@ -120,3 +120,14 @@ def test_custom_edge_lengths():
 def test_bits_roundtrip():
     t = torch.randn(3, 5).to(torch.bfloat16)
     assert torch.equal(wl.from_numpy_bits(wl.to_numpy_bits(t), "bf16"), t)
+
+
+def test_contiguous_placement():
+    """The contiguous comparator lays each sequence's blocks out consecutively."""
+    w = wl.mha(num_seqs=5, num_blocks=700, contiguous=True)
+    nxt = 0
+    for s in range(5):
+        nb = oracle.blocks_needed(int(w.context_lens[s]), w.block_size)
+        assert w.block_tables[s][:nb].tolist() == list(range(nxt, nxt + nb))
+        nxt += nb
+    _check_tables(w)
