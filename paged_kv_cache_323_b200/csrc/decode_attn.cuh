@@ -75,8 +75,10 @@ struct DecodeCfg {
     static constexpr int EPC = Elem<T>::kPer16B;
     static constexpr int CPR = D / EPC;        // 16-byte chunks per row
     static constexpr int RPI = 32 / CPR;       // rows covered by one warp-wide load
-    static constexpr int TR = BS < 16 ? BS : 16;  // rows per sub-tile
-    static constexpr int NSUB = BS / TR;
+    static constexpr int ST = 16;              // tokens per stage: two bs-8 blocks, a bs-16 block,
+                                               // or half of a bs-32 block
+    static constexpr int TR = ST;              // rows per sub-tile (one stage)
+    static constexpr int BPS = BS < ST ? ST / BS : 1;  // whole blocks per stage
     static constexpr int RPL = TR / RPI;       // rows per lane per sub-tile
     static constexpr int V = GW * RPL;         // partial logits per lane before the butterfly
     static constexpr int VPL = V >= CPR ? V / CPR : 1;  // logits per lane after it
@@ -84,8 +86,10 @@ struct DecodeCfg {
     static constexpr int NBL = 4;              // block lanes
     static constexpr int NCW = NBL * NHS;      // consumer warps
     static constexpr int THREADS = (NCW + 1) * 32;
-    static constexpr int SLICE = BS * D * (int)sizeof(T);  // bytes of one (block, kv head)
-    static constexpr int STAGE = 2 * SLICE;                // K slice + V slice
+    static constexpr int ROWB = D * (int)sizeof(T);       // bytes of one token row
+    static constexpr int SLICE = BS * ROWB;               // bytes of one (block, kv head)
+    static constexpr int STAGE_K = ST * ROWB;             // K rows of one stage
+    static constexpr int STAGE = 2 * STAGE_K;             // K rows + V rows
     static constexpr int NST_RAW = (64 * 1024) / STAGE;
     static constexpr int NST = NST_RAW < NBL ? NBL : (NST_RAW > 16 ? 16 : NST_RAW);
     static constexpr int MAX_PART_TOKENS = 4096;
@@ -108,7 +112,8 @@ struct DecodeCfg {
     static_assert(GW <= CPR, "a lane's logits after the butterfly belong to one head");
     static_assert(MERGE_FLOATS * 4 <= STAGES_BYTES, "merge area reuses the stages");
     static_assert(MERGE_SCRATCH_BYTES <= STAGES_BYTES, "fused merge scratch reuses the stages");
-    static_assert(SLICE % 16 == 0, "bulk copies move multiples of 16 bytes");
+    static_assert(STAGE_K % 16 == 0 && SLICE % 16 == 0, "bulk copies move multiples of 16 bytes");
+    static_assert(BS % ST == 0 || ST % BS == 0, "stages and blocks nest");
 };
 
 // Transposing butterfly over the CPR lanes of a row group: at each xor step a
@@ -280,6 +285,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, BS, G>::THREADS, 2)
     const int tok1 = min(ctx, tok0 + PT);
     const int nblk = (tok1 - tok0 + BS - 1) / BS;
     const int blk0 = tok0 / BS;
+    const int nstg = (tok1 - tok0 + C::ST - 1) / C::ST;
 
     unsigned char* stages = smem;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
@@ -312,7 +318,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, BS, G>::THREADS, 2)
     }
     __syncthreads();
 
-    int issued = 0;  // producer lane 0 only
+    int issued = 0;  // stages issued (producer lane 0)
     // Per-warp softmax state (consumer warps).
     float m_run[C::GW];
     float o[C::GW][C::EPC];
@@ -331,10 +337,13 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, BS, G>::THREADS, 2)
 
     if (warp == C::NCW) {
         // ------------------------------------------------------ producer
+        // One lane issues every copy: spreading them over the warp measured
+        // slower here (32 lanes polling the ring's barriers take issue slots
+        // from the consumer warps).
         if (lane == 0) {
             const char* kbase = static_cast<const char*>(p.k_cache);
             const char* vbase = static_cast<const char*>(p.v_cache);
-            for (int j = 0; j < nblk; ++j) {
+            for (int j = 0; j < nstg; ++j) {
                 const int st = j % C::NST;
                 if (j >= C::NST) {
                     if (!mbar_wait_bounded(&empty[st], ((j / C::NST) - 1) & 1, abort_flag)) {
@@ -343,15 +352,40 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, BS, G>::THREADS, 2)
                         break;
                     }
                 }
-                const int e = phys[j];
-                if (e >= 0) {
-                    const long long off = ((long long)e * Hkv + g) * C::SLICE;
-                    unsigned char* dst = stages + st * C::STAGE;
-                    mbar_arrive_expect_tx(&full[st], 2 * C::SLICE);
-                    bulk_g2s(dst, kbase + off, C::SLICE, &full[st]);
-                    bulk_g2s(dst + C::SLICE, vbase + off, C::SLICE, &full[st]);
+                unsigned char* dst = stages + st * C::STAGE;
+                if constexpr (BS >= C::ST) {
+                    // 16 rows of one block (the whole block when bs = 16)
+                    const int e = phys[j * C::ST / BS];
+                    if (e >= 0) {
+                        const long long off =
+                            (((long long)e * Hkv + g) * BS + (j * C::ST) % BS) * C::ROWB;
+                        mbar_arrive_expect_tx(&full[st], 2 * C::STAGE_K);
+                        bulk_g2s(dst, kbase + off, C::STAGE_K, &full[st]);
+                        bulk_g2s(dst + C::STAGE_K, vbase + off, C::STAGE_K, &full[st]);
+                    } else {
+                        mbar_arrive(&full[st]);  // a skipped block still completes its phase
+                    }
                 } else {
-                    mbar_arrive(&full[st]);  // a skipped block still completes its phase
+                    // whole blocks stacked row after row
+                    int cnt = 0;
+#pragma unroll
+                    for (int b = 0; b < C::BPS; ++b) {
+                        const int jb = j * C::BPS + b;
+                        cnt += jb < nblk && phys[jb] >= 0;
+                    }
+                    if (cnt > 0) {
+                        mbar_arrive_expect_tx(&full[st], (uint32_t)(cnt * 2 * C::SLICE));
+#pragma unroll
+                        for (int b = 0; b < C::BPS; ++b) {
+                            const int jb = j * C::BPS + b;
+                            if (jb >= nblk || phys[jb] < 0) continue;
+                            const long long off = ((long long)phys[jb] * Hkv + g) * C::SLICE;
+                            bulk_g2s(dst + b * C::SLICE, kbase + off, C::SLICE, &full[st]);
+                            bulk_g2s(dst + C::STAGE_K + b * C::SLICE, vbase + off, C::SLICE, &full[st]);
+                        }
+                    } else {
+                        mbar_arrive(&full[st]);
+                    }
                 }
                 issued = j + 1;
             }
@@ -372,7 +406,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, BS, G>::THREADS, 2)
         const int vbase_idx = (C::V >= C::CPR) ? c * C::VPL : c / (C::CPR / C::V);
         const bool l_owner = (C::V >= C::CPR) || (c % (C::CPR / C::V) == 0);
 
-        for (int j = bl; j < nblk; j += C::NBL) {
+        for (int j = bl; j < nstg; j += C::NBL) {
             const int st = j % C::NST;
             // every lane waits (bounded); the warp leaves together if any lane gave up
             const bool ready = mbar_wait_bounded(&full[st], (j / C::NST) & 1, abort_flag);
@@ -383,14 +417,25 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, BS, G>::THREADS, 2)
                 }
                 break;
             }
-            if (phys[j] >= 0) {
-                const uint4* Ks = reinterpret_cast<const uint4*>(stages + st * C::STAGE);
-                const uint4* Vs = reinterpret_cast<const uint4*>(stages + st * C::STAGE + C::SLICE);
-                const int nvalid = min(BS, tok1 - (tok0 + j * BS));
+            // rows of this stage that hold tokens of the partition, from blocks
+            // whose table entry was valid (warp-uniform)
+            const int nvalid = min(C::ST, tok1 - (tok0 + j * C::ST));
+            uint32_t rowmask = nvalid >= 32 ? 0xffffffffu : ((1u << nvalid) - 1u);
+            if constexpr (BS >= C::ST) {
+                if (phys[j * C::ST / BS] < 0) rowmask = 0;
+            } else {
 #pragma unroll
-                for (int sub = 0; sub < C::NSUB; ++sub) {
-                    const int rbase = sub * C::TR;
-                    if (rbase >= nvalid) break;
+                for (int b = 0; b < C::BPS; ++b) {
+                    const int jb = j * C::BPS + b;
+                    if (jb >= nblk || phys[jb] < 0) rowmask &= ~(((1u << BS) - 1u) << (b * BS));
+                }
+            }
+            if (rowmask != 0) {
+                const uint4* Ks = reinterpret_cast<const uint4*>(stages + st * C::STAGE);
+                const uint4* Vs = reinterpret_cast<const uint4*>(stages + st * C::STAGE + C::STAGE_K);
+                const bool tail = rowmask != (1u << C::ST) - 1u;
+                {
+                    constexpr int rbase = 0;
                     // ---- QK^T: partial dot products over this lane's chunk
                     float sc[C::V];
 #pragma unroll
@@ -412,7 +457,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, BS, G>::THREADS, 2)
 #pragma unroll
                     for (int i = 0; i < C::VPL; ++i) {
                         const int k = (vbase_idx + i) % C::RPL;
-                        const bool valid = rbase + r0 + k * C::RPI < nvalid;
+                        const bool valid = (rowmask >> (rbase + r0 + k * C::RPI)) & 1u;
                         sc[i] = valid ? sc[i] : -INFINITY;
                         mloc = fmaxf(mloc, sc[i]);
                     }
@@ -452,7 +497,6 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, BS, G>::THREADS, 2)
                     }
                     __syncwarp();
                     // ---- PV over this lane's rows and chunk
-                    const bool tail = nvalid - rbase < C::TR;
 #pragma unroll
                     for (int k = 0; k < C::RPL; ++k) {
                         const int row = rbase + r0 + k * C::RPI;
@@ -472,7 +516,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, BS, G>::THREADS, 2)
                         }
                         float vf[C::EPC];
                         Elem<T>::unpack(Vs[row * C::CPR + c], vf);
-                        if (tail && row >= nvalid) continue;  // unused slot: never read into o
+                        if (tail && !((rowmask >> row) & 1u)) continue;  // never read an unused slot into o
 #pragma unroll
                         for (int gi = 0; gi < C::GW; ++gi)
 #pragma unroll
