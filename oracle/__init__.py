@@ -17,11 +17,15 @@ from .binding import (  # noqa: F401
     build,
     compile_source,
     copy_blocks,
+    e4m3_encode,
+    e4m3_value,
     gather,
     kv_append,
+    kv_append_fp8,
     library_path,
     open_library,
     paged_attention,
+    paged_attention_fp8,
     swap_blocks,
     use_library,
     waste_per_sequence,

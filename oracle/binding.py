@@ -59,6 +59,14 @@ def open_library(path: str):
     lib.oracle_kv_append.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32]
     lib.oracle_copy_blocks.argtypes = [P, P, P, i32, i32, i32, i32, i32]
     lib.oracle_swap_blocks.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32]
+    lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_value.restype = dbl
+    lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+    lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+    lib.oracle_kv_append_fp8.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32]
+    lib.oracle_paged_attention_fp8.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32,
+                                               i32, dbl]
+    lib.oracle_paged_attention_fp8.restype = i32
     return lib
 
 
@@ -191,3 +199,47 @@ def swap_blocks(dst_k: np.ndarray, dst_v: np.ndarray, src_k: np.ndarray, src_v: 
     _load().oracle_swap_blocks(_ptr(dst_k), _ptr(dst_v), _ptr(np.ascontiguousarray(src_k)),
                                _ptr(np.ascontiguousarray(src_v)), _ptr(pairs), pairs.shape[0], hkv,
                                d, bs, code)
+
+
+def e4m3_value(code: int) -> float:
+    return float(_load().oracle_e4m3_value(int(code)))
+
+
+def e4m3_encode(y: float) -> int:
+    return int(_load().oracle_e4m3_encode(float(y)))
+
+
+def kv_append_fp8(k_cache: np.ndarray, v_cache: np.ndarray, k_scales, v_scales, k: np.ndarray,
+                  v: np.ndarray, slot_mapping) -> None:
+    """In place on uint8 (e4m3 code) caches; k, v are bf16 bit patterns."""
+    assert k_cache.dtype == np.uint8 and k.dtype == np.uint16
+    ks = np.ascontiguousarray(k_scales, dtype=np.float32)
+    vs = np.ascontiguousarray(v_scales, dtype=np.float32)
+    sm = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    k = np.ascontiguousarray(k)
+    v = np.ascontiguousarray(v)
+    _, hkv, bs, d = k_cache.shape
+    _load().oracle_kv_append_fp8(_ptr(k_cache), _ptr(v_cache), _ptr(ks), _ptr(vs), _ptr(k), _ptr(v),
+                                 _ptr(sm), len(sm), hkv, d, bs)
+
+
+def paged_attention_fp8(q, k_cache, v_cache, k_scales, v_scales, block_tables, context_lens,
+                        scale: float) -> np.ndarray:
+    """fp64 decode attention over e4m3 caches with per-kv-head scales; q is bf16 bits."""
+    q = np.ascontiguousarray(q)
+    k_cache = np.ascontiguousarray(k_cache)
+    v_cache = np.ascontiguousarray(v_cache)
+    assert q.dtype == np.uint16 and k_cache.dtype == np.uint8
+    ks = np.ascontiguousarray(k_scales, dtype=np.float32)
+    vs = np.ascontiguousarray(v_scales, dtype=np.float32)
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    ctx = np.ascontiguousarray(context_lens, dtype=np.int32)
+    B, H, D = q.shape
+    _, hkv, bs, _ = k_cache.shape
+    out = np.zeros((B, H, D), dtype=np.float64)
+    rc = _load().oracle_paged_attention_fp8(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                            _ptr(ks), _ptr(vs), _ptr(bt), _ptr(ctx), B, H, hkv, D,
+                                            bs, bt.shape[1], float(scale))
+    if rc != 0:
+        raise ValueError("oracle_paged_attention_fp8 rejected its arguments")
+    return out

@@ -159,6 +159,34 @@ typedef struct {
     pthread_mutex_t lock;
 } attn_job;
 
+/* Steps 2-4 of the definition for one query row over contiguous K and V
+ * (L rows of D values, fp64): logits, softmax weights, weighted sum of V. */
+static void attend_rows(double* o, const double* qd, const double* Kc, const double* Vc, int L,
+                        int D, double scale) {
+    double* x = (double*)malloc(sizeof(double) * (size_t)L);
+    /* step 2: logits */
+    for (int t = 0; t < L; ++t) {
+        double acc = 0.0;
+        for (int d = 0; d < D; ++d) acc += qd[d] * Kc[(int64_t)t * D + d];
+        x[t] = scale * acc;
+    }
+    /* step 3: softmax weights */
+    double m = x[0];
+    for (int t = 1; t < L; ++t)
+        if (x[t] > m) m = x[t];
+    double Z = 0.0;
+    for (int t = 0; t < L; ++t) {
+        x[t] = exp(x[t] - m);
+        Z += x[t];
+    }
+    /* step 4: weighted sum of values */
+    for (int t = 0; t < L; ++t) {
+        double w = x[t] / Z;
+        for (int d = 0; d < D; ++d) o[d] += w * Vc[(int64_t)t * D + d];
+    }
+    free(x);
+}
+
 /* One (s, h) unit, written as the definition. */
 static void attend_one(attn_job* job, int unit) {
     int s, h;
@@ -179,7 +207,6 @@ static void attend_one(attn_job* job, int unit) {
 
     double* Kc = (double*)malloc(sizeof(double) * (size_t)L * D);
     double* Vc = (double*)malloc(sizeof(double) * (size_t)L * D);
-    double* x = (double*)malloc(sizeof(double) * (size_t)L);
     double* qd = (double*)malloc(sizeof(double) * (size_t)D);
 
     /* step 1: the logical (contiguous) view of this sequence's cache */
@@ -190,29 +217,9 @@ static void attend_one(attn_job* job, int unit) {
     for (int d = 0; d < D; ++d)
         qd[d] = load_elem(job->q, ((int64_t)s * job->num_heads + h) * D + d, job->dtype);
 
-    /* step 2: logits */
-    for (int t = 0; t < L; ++t) {
-        double acc = 0.0;
-        for (int d = 0; d < D; ++d) acc += qd[d] * Kc[(int64_t)t * D + d];
-        x[t] = job->scale * acc;
-    }
-    /* step 3: softmax weights */
-    double m = x[0];
-    for (int t = 1; t < L; ++t)
-        if (x[t] > m) m = x[t];
-    double Z = 0.0;
-    for (int t = 0; t < L; ++t) {
-        x[t] = exp(x[t] - m);
-        Z += x[t];
-    }
-    /* step 4: weighted sum of values */
-    for (int t = 0; t < L; ++t) {
-        double w = x[t] / Z;
-        for (int d = 0; d < D; ++d) o[d] += w * Vc[(int64_t)t * D + d];
-    }
+    attend_rows(o, qd, Kc, Vc, L, D, job->scale);
     free(Kc);
     free(Vc);
-    free(x);
     free(qd);
 }
 
@@ -332,4 +339,122 @@ void oracle_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void*
         memcpy((char*)dst_v + dst * block_bytes, (const char*)src_v + src * block_bytes,
                (size_t)block_bytes);
     }
+}
+
+/* ------------------------------------------------ fp8 (e4m3) KV cache */
+/* "What does PagedAttention change in LLM KV allocation?", section "Sharing
+ * requires more than allocation": where the raw KV data does not fit, cache
+ * quantization is one of the remedies.  Reading used here: K and V stored as
+ * OCP FP8 E4M3 (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; no
+ * infinities; S.1111.111 is NaN; largest finite 448), one float scale per kv
+ * head: stored value = code * scale. */
+
+/* Exact value of an e4m3 code. */
+double oracle_e4m3_value(uint8_t code) {
+    const int sign = code >> 7;
+    const int e = (code >> 3) & 15;
+    const int m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9); /* subnormal: m/8 * 2^-6 */
+    else
+        v = ldexp(8.0 + m, e - 10); /* (1 + m/8) * 2^(e-7) */
+    return sign ? -v : v;
+}
+
+/* Nearest e4m3 code to y, ties to the even code, magnitudes of 448 and more
+ * clamped to 448 (saturating); NaN stays NaN.  Written as a search over the
+ * 127 non-negative finite codes, which is the definition of rounding. */
+uint8_t oracle_e4m3_encode(float y) {
+    if (isnan(y)) return 0x7F;
+    const uint8_t sign = signbit(y) ? 0x80 : 0x00;
+    const double a = fabs((double)y);
+    if (a >= 448.0) return sign | 0x7E;
+    int best = 0;
+    double best_err = a;
+    for (int c = 1; c <= 0x7E; ++c) {
+        const double err = fabs(oracle_e4m3_value((uint8_t)c) - a);
+        if (err < best_err || (err == best_err && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_err = err;
+        }
+    }
+    return sign | (uint8_t)best;
+}
+
+/* Append with quantization: token i's bf16 rows (raw bits) become codes of
+ * (float)x / scale[g] (one correctly rounded fp32 division) at slot
+ * slot_mapping[i]; -1 skips. */
+void oracle_kv_append_fp8(uint8_t* k_cache, uint8_t* v_cache, const float* k_scales,
+                          const float* v_scales, const uint16_t* k, const uint16_t* v,
+                          const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                          int head_dim, int block_size) {
+    for (int i = 0; i < num_tokens; ++i) {
+        const int64_t slot = slot_mapping[i];
+        if (slot < 0) { /* no write for this token */
+            continue;
+        }
+        const int64_t blk = slot / block_size;
+        const int64_t off = slot - blk * block_size;
+        for (int g = 0; g < num_kv_heads; ++g) {
+            const int64_t dst = ((blk * num_kv_heads + g) * block_size + off) * head_dim;
+            const int64_t src = ((int64_t)i * num_kv_heads + g) * head_dim;
+            for (int d = 0; d < head_dim; ++d) {
+                const float kx = (float)load_elem(k, src + d, ORACLE_BF16);
+                const float vx = (float)load_elem(v, src + d, ORACLE_BF16);
+                k_cache[dst + d] = oracle_e4m3_encode(kx / k_scales[g]);
+                v_cache[dst + d] = oracle_e4m3_encode(vx / v_scales[g]);
+            }
+        }
+    }
+}
+
+/* Offset of token t (kv head g) in a [block][kv head][slot][dim] pool, the
+ * token's block taken from this sequence's table row. */
+static int64_t fp8_token_row(const int32_t* table_row, int t, int block_size, int num_kv_heads,
+                             int g, int head_dim) {
+    const int32_t blk = table_row[t / block_size];
+    return (((int64_t)blk * num_kv_heads + g) * block_size + t % block_size) * head_dim;
+}
+
+/* Decode attention over an e4m3 cache: the same definition as
+ * oracle_paged_attention with K[t][d] = code * k_scale[g] and V likewise
+ * (each product exact in fp64); q (bf16 bits) and out as there. */
+int oracle_paged_attention_fp8(double* out, const uint16_t* q, const uint8_t* k_cache,
+                               const uint8_t* v_cache, const float* k_scales,
+                               const float* v_scales, const int32_t* block_tables,
+                               const int32_t* context_lens, int num_seqs, int num_heads,
+                               int num_kv_heads, int head_dim, int block_size,
+                               int max_blocks_per_seq, double scale) {
+    if (num_kv_heads <= 0 || num_heads % num_kv_heads != 0 || head_dim > 1024) return -1;
+    const int D = head_dim, group = num_heads / num_kv_heads;
+    for (int s = 0; s < num_seqs; ++s) {
+        const int L = context_lens[s];
+        if (L > (int64_t)max_blocks_per_seq * block_size) return -1;
+        const int32_t* table_row = block_tables + (int64_t)s * max_blocks_per_seq;
+        for (int h = 0; h < num_heads; ++h) {
+            const int g = h / group; /* contiguous query-head groups */
+            double* o = out + ((int64_t)s * num_heads + h) * D;
+            for (int d = 0; d < D; ++d) o[d] = 0.0;
+            if (L <= 0) continue;
+            /* the logical view, dequantised: code * scale of the kv head */
+            double* Kc = (double*)malloc(sizeof(double) * (size_t)L * D);
+            double* Vc = (double*)malloc(sizeof(double) * (size_t)L * D);
+            double qd[1024];
+            for (int t = 0; t < L; ++t) {
+                const int64_t row = fp8_token_row(table_row, t, block_size, num_kv_heads, g, D);
+                for (int d = 0; d < D; ++d) {
+                    Kc[(int64_t)t * D + d] = oracle_e4m3_value(k_cache[row + d]) * (double)k_scales[g];
+                    Vc[(int64_t)t * D + d] = oracle_e4m3_value(v_cache[row + d]) * (double)v_scales[g];
+                }
+            }
+            for (int d = 0; d < D; ++d)
+                qd[d] = load_elem(q, ((int64_t)s * num_heads + h) * D + d, ORACLE_BF16);
+            attend_rows(o, qd, Kc, Vc, L, D, scale);
+            free(Kc);
+            free(Vc);
+        }
+    }
+    return 0;
 }

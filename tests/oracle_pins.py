@@ -452,6 +452,110 @@ def pin_swap_round_trip():
             assert np.array_equal(dk[p].view(np.uint8), k0[p].view(np.uint8))
 
 
+def _torch_e4m3_codes(x: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def pin_e4m3_decode():
+    """Every e4m3 code's value equals torch's float8_e4m3fn conversion."""
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).double().numpy()
+    got = np.asarray([oracle.e4m3_value(int(c)) for c in codes])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert oracle.e4m3_value(0x7E) == 448.0 and oracle.e4m3_value(0x01) == 2.0 ** -9
+
+
+def pin_e4m3_encode():
+    """Round to nearest (ties to even) as torch does inside the finite range;
+    saturation to +-448 beyond it (torch gives NaN there); NaN stays NaN;
+    every finite code round-trips."""
+    rng = np.random.default_rng(141)
+    xs = np.concatenate([
+        rng.uniform(-463, 463, 4000), rng.normal(0, 1, 4000), rng.normal(0, 1e-2, 2000),
+        np.ldexp(rng.uniform(-1, 1, 2000), -8),
+        # exact grid points and midpoints between neighbouring codes
+        [oracle.e4m3_value(c) for c in range(0x7F)],
+        [(oracle.e4m3_value(c) + oracle.e4m3_value(c + 1)) / 2 for c in range(0x7E)],
+    ]).astype(np.float32)
+    ref = _torch_e4m3_codes(xs)
+    got = np.asarray([oracle.e4m3_encode(float(x)) for x in xs], dtype=np.uint8)
+    assert np.array_equal(got, ref), np.flatnonzero(got != ref)[:5]
+    for y, code in ((464.0, 0x7E), (1e9, 0x7E), (-500.0, 0xFE), (float("inf"), 0x7E),
+                    (float("-inf"), 0xFE)):
+        assert oracle.e4m3_encode(y) == code, (y, oracle.e4m3_encode(y))
+    assert oracle.e4m3_encode(float("nan")) & 0x7F == 0x7F
+    for c in list(range(0x7F)) + list(range(0x80, 0xFF)):
+        assert oracle.e4m3_encode(oracle.e4m3_value(c)) == c
+
+
+def _fp8_case(seed, lens, H, Hkv, D, bs, ks, vs):
+    rng = np.random.default_rng(seed)
+    nblk = sum(-(-L // bs) for L in lens) + 3
+    kc = rng.integers(0, 256, size=(nblk, Hkv, bs, D)).astype(np.uint8)
+    vc = rng.integers(0, 256, size=(nblk, Hkv, bs, D)).astype(np.uint8)
+    for c in (kc, vc):  # no NaN codes
+        c[(c & 0x7F) == 0x7F] = 0x7E
+    perm = rng.permutation(nblk)
+    bt = np.full((len(lens), max(-(-L // bs) for L in lens)), -1, dtype=np.int32)
+    nxt = 0
+    for s, L in enumerate(lens):
+        for j in range(-(-L // bs)):
+            bt[s, j] = perm[nxt]
+            nxt += 1
+    q = to_dtype(rng.standard_normal((len(lens), H, D)).astype(np.float32) * 0.05, "bf16")
+    return q, kc, vc, np.asarray(ks, np.float32), np.asarray(vs, np.float32), bt, np.asarray(lens, np.int32)
+
+
+def pin_fp8_attention():
+    """With power-of-two scales every dequantised value is an fp32 number, and
+    the fp8 oracle equals the plain oracle on the dequantised caches exactly;
+    with other scales it matches a numpy brute force."""
+    H, Hkv, D, bs = 4, 2, 16, 8
+    q, kc, vc, ks, vs, bt, lens = _fp8_case(151, [19, 40, 3, 0], H, Hkv, D, bs, [0.25, 0.0625], [0.5, 2.0])
+    got = oracle.paged_attention_fp8(q, kc, vc, ks, vs, bt, lens, 0.3)
+    deq = np.vectorize(oracle.e4m3_value)
+    kf = (deq(kc) * ks[None, :, None, None]).astype(np.float32)
+    vf = (deq(vc) * vs[None, :, None, None]).astype(np.float32)
+    qf = values(q).astype(np.float32)
+    ref = oracle.paged_attention(qf, kf, vf, bt, lens, 0.3)
+    assert np.array_equal(got, ref)
+    q, kc, vc, ks, vs, bt, lens = _fp8_case(152, [33, 7], H, Hkv, D, bs, [0.013, 0.021], [0.017, 0.3])
+    got = oracle.paged_attention_fp8(q, kc, vc, ks, vs, bt, lens, 0.25)
+    for s, L in enumerate(lens):
+        for h in range(H):
+            g = h // (H // Hkv)
+            rows = [bt[s, t // bs] for t in range(L)]
+            K = np.stack([deq(kc[p, g, t % bs]) for t, p in enumerate(rows)]) * float(ks[g])
+            V = np.stack([deq(vc[p, g, t % bs]) for t, p in enumerate(rows)]) * float(vs[g])
+            ref = attention_contiguous(values(q)[s, h], K, V, 0.25)
+            assert np.abs(got[s, h] - ref).max() <= 1e-12
+
+
+def pin_fp8_append():
+    """Appended rows hold torch's e4m3 codes of (fp32 x) / scale; -1 skips."""
+    rng = np.random.default_rng(161)
+    Hkv, D, bs = 2, 16, 4
+    kc = np.zeros((6, Hkv, bs, D), np.uint8)
+    vc = np.zeros((6, Hkv, bs, D), np.uint8)
+    k = to_dtype(rng.standard_normal((3, Hkv, D)).astype(np.float32) * 3, "bf16")
+    v = to_dtype(rng.standard_normal((3, Hkv, D)).astype(np.float32) * 3, "bf16")
+    ks = np.asarray([0.02, 0.5], np.float32)
+    vs = np.asarray([0.125, 0.03], np.float32)
+    slots = np.asarray([5, -1, 17], np.int64)
+    oracle.kv_append_fp8(kc, vc, ks, vs, k, v, slots)
+    for i, slot in enumerate(slots):
+        if slot < 0:
+            continue
+        for g in range(Hkv):
+            kx = values(k)[i, g].astype(np.float32) / ks[g]
+            vx = values(v)[i, g].astype(np.float32) / vs[g]
+            assert np.array_equal(kc[slot // bs, g, slot % bs], _torch_e4m3_codes(np.clip(kx, -448, 448)))
+            assert np.array_equal(vc[slot // bs, g, slot % bs], _torch_e4m3_codes(np.clip(vx, -448, 448)))
+    assert not kc[[0, 2, 3, 5]].any()  # token 1 was skipped; only blocks 1 and 4 written
+
+
 PINS = [
     pin_worked_example,
     pin_logical_block_ranges,
@@ -472,4 +576,8 @@ PINS = [
     pin_copy_on_write,
     pin_copy_blocks_pairs,
     pin_swap_round_trip,
+    pin_e4m3_decode,
+    pin_e4m3_encode,
+    pin_fp8_attention,
+    pin_fp8_append,
 ]

@@ -21,7 +21,7 @@ ROOT = os.path.dirname(HERE)
 SRC = os.path.join(ROOT, "oracle", "pkv_oracle.c")
 
 MUTANTS = {
-    "dropped_scale": ("x[t] = job->scale * acc;", "x[t] = acc;"),
+    "dropped_scale": ("x[t] = scale * acc;", "x[t] = acc;"),
     "exp_sign": ("x[t] = exp(x[t] - m);", "x[t] = exp(m - x[t]);"),
     "no_max_shift": ("double m = x[0];\n    for (int t = 1; t < L; ++t)\n        if (x[t] > m) m = x[t];",
                      "double m = 0.0;"),
@@ -29,7 +29,7 @@ MUTANTS = {
     "k_for_v": ("o[d] += w * Vc[(int64_t)t * D + d];", "o[d] += w * Kc[(int64_t)t * D + d];"),
     "block_index": ("max_blocks_per_seq + t / block_size];", "max_blocks_per_seq + t / (block_size + 1)];"),
     "slot_index": ("int slot = t % block_size;", "int slot = (t + 1) % block_size;"),
-    "gqa_map": ("const int g = h / group;", "const int g = h % job->num_kv_heads;"),
+    "gqa_map": ("const int g = h / group;\n    const int L", "const int g = h % job->num_kv_heads;\n    const int L"),
     "q_row": ("((int64_t)s * job->num_heads + h) * D + d", "((int64_t)s * job->num_heads) * D + d"),
     "last_token_dropped": ("for (int t = 0; t < L; ++t) {\n        double acc",
                            "for (int t = 0; t < L; ++t) {\n        if (t == L - 1 && L > 1) { x[t] = -1e300; continue; }\n        double acc"),
@@ -46,6 +46,21 @@ MUTANTS = {
                       "(int64_t)block_size * head_dim * elem_bytes(dtype);"),
     "swap_direction": ("memcpy((char*)dst_k + dst * block_bytes, (const char*)src_k + src * block_bytes,",
                        "memcpy((char*)dst_k + src * block_bytes, (const char*)src_k + dst * block_bytes,"),
+    "e4m3_subnormal": ("v = ldexp((double)m, -9);", "v = ldexp((double)m, -10);"),
+    "e4m3_bias": ("v = ldexp(8.0 + m, e - 10);", "v = ldexp(8.0 + m, e - 9);"),
+    "e4m3_tie_odd": ("(err == best_err && (c & 1) == 0 && (best & 1) == 1)",
+                     "(err == best_err && (c & 1) == 1 && (best & 1) == 0)"),
+    "e4m3_no_saturation": ("if (a >= 448.0) return sign | 0x7E;", "if (a >= 448.0) return sign | 0x7F;"),
+    "fp8_k_scale_dropped": ("Kc[(int64_t)t * D + d] = oracle_e4m3_value(k_cache[row + d]) * (double)k_scales[g];",
+                            "Kc[(int64_t)t * D + d] = oracle_e4m3_value(k_cache[row + d]);"),
+    "fp8_v_uses_k_scale": ("Vc[(int64_t)t * D + d] = oracle_e4m3_value(v_cache[row + d]) * (double)v_scales[g];",
+                           "Vc[(int64_t)t * D + d] = oracle_e4m3_value(v_cache[row + d]) * (double)k_scales[g];"),
+    "fp8_gqa_map": ("const int g = h / group; /* contiguous query-head groups */",
+                    "const int g = h % num_kv_heads; /* contiguous query-head groups */"),
+    "fp8_block_index": ("const int32_t blk = table_row[t / block_size];",
+                        "const int32_t blk = table_row[t / (block_size + 1)];"),
+    "fp8_append_multiplies": ("k_cache[dst + d] = oracle_e4m3_encode(kx / k_scales[g]);",
+                              "k_cache[dst + d] = oracle_e4m3_encode(kx * k_scales[g]);"),
     "physical_double_count": ("if (here > filled[p]) filled[p] = (int32_t)here;",
                               "filled[p] += (int32_t)here;"),
 }
