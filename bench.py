@@ -59,13 +59,16 @@ WORKLOADS = {
                         lambda dev, seed: wl.mha(seed=seed, device=dev, contiguous=True)),
     "mha_contig_bs32": ("mha_decode_b64_h32_kv32_d128_bs32_contiguous_bf16",
                         lambda dev, seed: wl.mha(seed=seed, device=dev, block_size=32, contiguous=True)),
+    # the same MHA batch with an fp8 (e4m3) cache and per-kv-head scales: half the KV bytes
+    "mha_fp8": ("mha_decode_b64_h32_kv32_d128_bs16_ctxU128-2048_fp8e4m3_cache",
+                lambda dev, seed: wl.mha(seed=seed, device=dev, dtype="fp8")),
     # a smaller MHA batch for profiler captures: 16 sequences, 4096-block pool (1 GB), ~0.3 GB KV per step
     "mha_small": ("mha_decode_b16_h32_kv32_d128_bs16_ctxU128-2048_bf16_pool4096",
                   lambda dev, seed: wl.mha(seed=seed, device=dev, num_seqs=16, num_blocks=4096)),
 }
 DEFAULT_SEED = {"mha": 2, "gqa_sampling": 3, "long_context": 4, "prefix_bs8": 5, "prefix_bs16": 5,
                 "prefix_bs32": 5, "tiny": 1, "mha_small": 2, "mha_bs8": 2, "mha_bs32": 2,
-                "mha_contig_bs8": 2, "mha_contig_bs16": 2, "mha_contig_bs32": 2}
+                "mha_contig_bs8": 2, "mha_contig_bs16": 2, "mha_contig_bs32": 2, "mha_fp8": 2}
 
 
 def measured_peak():
@@ -238,8 +241,12 @@ def compact_subset(w: wl.Workload, seqs):
     order = sorted(blocks)
     remap = {b: i for i, b in enumerate(order)}
     idx = torch.tensor(order, dtype=torch.long, device=w.k_cache.device)
-    kc = wl.to_numpy_bits(w.k_cache.index_select(0, idx))
-    vc = wl.to_numpy_bits(w.v_cache.index_select(0, idx))
+    if w.dtype == "fp8":  # gather the codes as bytes
+        kc = w.k_cache.view(torch.uint8).index_select(0, idx).cpu().numpy()
+        vc = w.v_cache.view(torch.uint8).index_select(0, idx).cpu().numpy()
+    else:
+        kc = wl.to_numpy_bits(w.k_cache.index_select(0, idx))
+        vc = wl.to_numpy_bits(w.v_cache.index_select(0, idx))
     bt = np.full((len(seqs), w.max_blocks_per_seq), -1, dtype=np.int32)
     for i, s in enumerate(seqs):
         nb = -(-int(w.context_lens[s]) // bs)
@@ -254,6 +261,7 @@ def compact_subset(w: wl.Workload, seqs):
     return dict(q=q, kc=kc, vc=vc, bt=bt, ctx=w.context_lens[seqs].copy(), slots=slots,
                 k_new=wl.to_numpy_bits(w.k_new.index_select(0, tok_idx)),
                 v_new=wl.to_numpy_bits(w.v_new.index_select(0, tok_idx)), pairs=pairs,
+                k_scales=w.k_scales, v_scales=w.v_scales,
                 kv_bytes=int(w.context_lens[seqs].astype(np.int64).sum()) * w.num_kv_heads
                 * w.head_dim * 2 * w.elt)
 
@@ -266,6 +274,12 @@ def oracle_sample_step(sub, scale, threads):
     t0 = time.perf_counter()
     if len(sub["pairs"]):
         oracle.copy_blocks(kc, vc, sub["pairs"])
+    if sub["k_scales"] is not None:  # fp8 cache
+        oracle.kv_append_fp8(kc, vc, sub["k_scales"], sub["v_scales"], sub["k_new"], sub["v_new"],
+                             sub["slots"])
+        oracle.paged_attention_fp8(sub["q"], kc, vc, sub["k_scales"], sub["v_scales"], sub["bt"],
+                                   sub["ctx"], scale)
+        return time.perf_counter() - t0
     oracle.kv_append(kc, vc, sub["k_new"], sub["v_new"], sub["slots"])
     oracle.paged_attention(sub["q"], kc, vc, sub["bt"], sub["ctx"], scale, nthreads=threads)
     return time.perf_counter() - t0
@@ -369,9 +383,21 @@ def run_gpu(args, world, rank, local):
     ws = torch.zeros(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
+    fp8 = w.dtype == "fp8"
+    if fp8:
+        ks = torch.from_numpy(w.k_scales).to(dev)
+        vs = torch.from_numpy(w.v_scales).to(dev)
+
     def step(q, k_new, v_new, bt, ctx, slots):
         if len(w.cow_pairs):
             pk.copy_blocks(t["k_cache"], t["v_cache"], t["pairs"])
+        if fp8:
+            pk.kv_cache_append_fp8(t["k_cache"], t["v_cache"], ks, vs, k_new, v_new, slots)
+            pk.paged_attention_decode_fp8(out, q, t["k_cache"], t["v_cache"], ks, vs, bt, ctx,
+                                          w.scale, num_blocks=w.num_blocks,
+                                          partition_tokens=args.partition_tokens,
+                                          workspace=ws if ws_bytes else None)
+            return
         pk.kv_cache_append(t["k_cache"], t["v_cache"], k_new, v_new, slots)
         pk.paged_attention_decode_ex(out, q, t["k_cache"], t["v_cache"], bt, ctx, w.scale,
                                      num_blocks=w.num_blocks,

@@ -74,8 +74,9 @@ typedef enum {
     PKV_ERR_OUT_OF_BLOCKS = -8  /* block manager: the free list cannot cover the request */
 } pkv_status;
 
-/* Element types of q, out, the pools and the new tokens. */
-typedef enum { PKV_F32 = 0, PKV_BF16 = 1 } pkv_dtype;
+/* Element types of q, out, the pools and the new tokens.  PKV_FP8_E4M3
+ * (OCP FP8 E4M3, one byte) is a cache type only: see the _fp8 calls. */
+typedef enum { PKV_F32 = 0, PKV_BF16 = 1, PKV_FP8_E4M3 = 2 } pkv_dtype;
 
 /* Kernels reported by the launch profiler. */
 typedef enum {
@@ -137,6 +138,34 @@ PKV_API int paged_attention_decode_ex(void* out, const void* q, const void* k_ca
 PKV_API int paged_attention_partition_tokens(int num_seqs, int num_heads, int num_kv_heads,
                                              int head_dim, int block_size, int max_context,
                                              int dtype, int partition_tokens);
+
+/*
+ * Quantised KV cache ("What does PagedAttention change in LLM KV
+ * allocation?", section "Sharing requires more than allocation": when the raw
+ * KV data does not fit, cache quantization is one of the remedies).  The
+ * pools hold fp8 e4m3 codes; one float scale per kv head (device arrays
+ * k_scales, v_scales [num_kv_heads]) gives the stored value code * scale.  q
+ * and out are bf16.  Otherwise exactly paged_attention_decode_ex (same
+ * workspace, partitions, faults); the kernel is the CUDA-core one, reading
+ * half the bytes of a bf16 cache per token.
+ */
+PKV_API int paged_attention_decode_fp8(void* out, const void* q, const void* k_cache,
+                                       const void* v_cache, const float* k_scales,
+                                       const float* v_scales, const int32_t* block_tables,
+                                       const int32_t* context_lens, int num_seqs, int num_heads,
+                                       int num_kv_heads, int head_dim, int block_size,
+                                       int max_blocks_per_seq, float scale, int num_blocks,
+                                       int partition_tokens, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
+/* Append to fp8 pools: new bf16 rows k, v [num_tokens][num_kv_heads][head_dim]
+ * are stored as the e4m3 codes of x / scale (the division correctly rounded
+ * in fp32; round to nearest even; magnitudes beyond 448 saturate to 448).
+ * Slots as in kv_cache_append; head_dim a multiple of 16. */
+PKV_API int kv_cache_append_fp8(void* k_cache, void* v_cache, const float* k_scales,
+                                const float* v_scales, const void* k, const void* v,
+                                const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                                int head_dim, int block_size, int num_blocks, void* stream);
 
 /* Bytes of split-K workspace paged_attention_decode_ex needs; 0 when every
  * sequence fits one partition.  With partition_tokens 0 the result covers

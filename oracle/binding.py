@@ -14,6 +14,7 @@ import numpy as np
 
 ORACLE_F32 = 0
 ORACLE_BF16 = 1
+ORACLE_FP8 = 2  # e4m3 codes (uint8): byte moves only; attention has its own fp8 entry
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "pkv_oracle.c")
@@ -100,6 +101,8 @@ def _dtype_code(a: np.ndarray) -> int:
         return ORACLE_F32
     if a.dtype == np.uint16:
         return ORACLE_BF16
+    if a.dtype == np.uint8:
+        return ORACLE_FP8
     raise TypeError(f"oracle takes float32 or bf16 bit patterns (uint16), got {a.dtype}")
 
 

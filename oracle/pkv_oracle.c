@@ -45,6 +45,7 @@
 
 #define ORACLE_F32 0
 #define ORACLE_BF16 1
+#define ORACLE_FP8 2 /* e4m3 codes: moved as bytes by append / copy / swap */
 
 /* ---------------------------------------------------------------- values */
 
@@ -62,7 +63,7 @@ static double load_elem(const void* base, int64_t index, int dtype) {
     return (double)f;
 }
 
-static int elem_bytes(int dtype) { return dtype == ORACLE_F32 ? 4 : 2; }
+static int elem_bytes(int dtype) { return dtype == ORACLE_F32 ? 4 : (dtype == ORACLE_FP8 ? 1 : 2); }
 
 /* ------------------------------------------------- block-count accounting */
 

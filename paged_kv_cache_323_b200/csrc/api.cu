@@ -110,7 +110,9 @@ int launch(int kind, cudaStream_t st, Fn&& fn) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int elt_bytes(int dtype) { return dtype == PKV_F32 ? 4 : 2; }
+int elt_bytes(int dtype) { return dtype == PKV_F32 ? 4 : dtype == PKV_FP8_E4M3 ? 1 : 2; }
+
+bool known_dtype(int dtype) { return dtype == PKV_F32 || dtype == PKV_BF16 || dtype == PKV_FP8_E4M3; }
 
 bool decode_shape_supported(int head_dim, int block_size, int group) {
     const bool d_ok = head_dim == 64 || head_dim == 128;
@@ -229,12 +231,19 @@ int paged_attention_partition_tokens(int num_seqs, int num_heads, int num_kv_hea
                                     max_context, dtype, partition_tokens);
 }
 
-int paged_attention_decode_ex(void* out, const void* q, const void* k_cache, const void* v_cache,
-                              const int32_t* block_tables, const int32_t* context_lens,
-                              int num_seqs, int num_heads, int num_kv_heads, int head_dim,
-                              int block_size, int max_blocks_per_seq, float scale, int num_blocks,
-                              int dtype, int partition_tokens, void* workspace,
-                              size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared body of the decode entry points.  dtype: q and out; kv_dtype: the
+// caches (dtype itself, or PKV_FP8_E4M3 with bf16 q / out and per-kv-head
+// scales k_scales / v_scales in device memory).
+int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                const float* k_scales, const float* v_scales, const int32_t* block_tables,
+                const int32_t* context_lens, int num_seqs, int num_heads, int num_kv_heads,
+                int head_dim, int block_size, int max_blocks_per_seq, float scale, int num_blocks,
+                int dtype, int kv_dtype, int partition_tokens, void* workspace,
+                size_t workspace_bytes, void* stream) {
     if (num_seqs < 0) return PKV_ERR_INVALID;
     if (num_seqs == 0) return PKV_OK;
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PKV_ERR_NULL;
@@ -242,6 +251,9 @@ int paged_attention_decode_ex(void* out, const void* q, const void* k_cache, con
     if (head_dim <= 0 || block_size <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0)
         return PKV_ERR_INVALID;
     if (dtype != PKV_F32 && dtype != PKV_BF16) return PKV_ERR_INVALID;
+    const bool fp8 = kv_dtype == PKV_FP8_E4M3;
+    if (kv_dtype != dtype && !(fp8 && dtype == PKV_BF16)) return PKV_ERR_INVALID;
+    if (fp8 && (!k_scales || !v_scales)) return PKV_ERR_NULL;
     if (!isfinite(scale)) return PKV_ERR_INVALID;
     const int group = num_heads / num_kv_heads;
     if (!decode_shape_supported(head_dim, block_size, group)) return PKV_ERR_UNSUPPORTED;
@@ -253,7 +265,7 @@ int paged_attention_decode_ex(void* out, const void* q, const void* k_cache, con
     const long long max_ctx = (long long)max_blocks_per_seq * block_size;
     if (max_ctx > INT_MAX) return PKV_ERR_INVALID;
     const int pt = resolve_partition_tokens(num_seqs, num_heads, num_kv_heads, head_dim,
-                                            block_size, max_ctx, dtype, partition_tokens);
+                                            block_size, max_ctx, kv_dtype, partition_tokens);
     const long long parts = (max_ctx + pt - 1) / pt;
     const long long grid = parts * num_kv_heads * (long long)num_seqs;
     if (grid > INT_MAX || (long long)num_seqs * num_heads > INT_MAX) return PKV_ERR_INVALID;
@@ -280,6 +292,8 @@ int paged_attention_decode_ex(void* out, const void* q, const void* k_cache, con
     p.ws_o = need > 0 ? reinterpret_cast<float*>(wsb + wl.o_off) : nullptr;
     p.ws_ml = need > 0 ? reinterpret_cast<float2*>(wsb + wl.ml_off) : nullptr;
     p.counters = need > 0 ? reinterpret_cast<int*>(wsb + wl.cnt_off) : nullptr;
+    p.k_scales = fp8 ? k_scales : nullptr;
+    p.v_scales = fp8 ? v_scales : nullptr;
     p.err = err;
     p.num_seqs = num_seqs;
     p.num_heads = num_heads;
@@ -292,12 +306,42 @@ int paged_attention_decode_ex(void* out, const void* q, const void* k_cache, con
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool use_tc = g_tc_gqa.load() != 0 &&
-                        pkv::decode_tc_supported(dtype, head_dim, block_size, group, pt);
+                        pkv::decode_tc_supported(kv_dtype, head_dim, block_size, group, pt);
     return launch(PKV_KERNEL_DECODE, st, [&] {
         if (use_tc) return pkv::launch_decode_tc(p, block_size, group, grid, st);
+        if (fp8) return pkv::launch_decode_partition_fp8(p, head_dim, block_size, group, grid, st);
         return dtype == PKV_F32 ? pkv::launch_decode_partition_f32(p, head_dim, block_size, group, grid, st)
                                 : pkv::launch_decode_partition_bf16(p, head_dim, block_size, group, grid, st);
     });
+}
+
+}  // namespace
+
+extern "C" {
+
+int paged_attention_decode_ex(void* out, const void* q, const void* k_cache, const void* v_cache,
+                              const int32_t* block_tables, const int32_t* context_lens,
+                              int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                              int block_size, int max_blocks_per_seq, float scale, int num_blocks,
+                              int dtype, int partition_tokens, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+    return decode_impl(out, q, k_cache, v_cache, nullptr, nullptr, block_tables, context_lens,
+                       num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                       max_blocks_per_seq, scale, num_blocks, dtype, dtype, partition_tokens,
+                       workspace, workspace_bytes, stream);
+}
+
+int paged_attention_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                               const float* k_scales, const float* v_scales,
+                               const int32_t* block_tables, const int32_t* context_lens,
+                               int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                               int block_size, int max_blocks_per_seq, float scale,
+                               int num_blocks, int partition_tokens, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+    return decode_impl(out, q, k_cache, v_cache, k_scales, v_scales, block_tables, context_lens,
+                       num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                       max_blocks_per_seq, scale, num_blocks, PKV_BF16, PKV_FP8_E4M3,
+                       partition_tokens, workspace, workspace_bytes, stream);
 }
 
 int paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -373,6 +417,48 @@ int kv_cache_append(void* k_cache, void* v_cache, const void* k, const void* v,
     });
 }
 
+int kv_cache_append_fp8(void* k_cache, void* v_cache, const float* k_scales,
+                        const float* v_scales, const void* k, const void* v,
+                        const int64_t* slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                        int block_size, int num_blocks, void* stream) {
+    if (num_tokens < 0) return PKV_ERR_INVALID;
+    if (num_tokens == 0) return PKV_OK;
+    if (!k_cache || !v_cache || !k_scales || !v_scales || !k || !v || !slot_mapping)
+        return PKV_ERR_NULL;
+    if (num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+        return PKV_ERR_INVALID;
+    if (head_dim % 16 != 0 || head_dim > 256 * 16) return PKV_ERR_UNSUPPORTED;
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k) || !aligned16(v))
+        return PKV_ERR_INVALID;
+    int dev = 0;
+    if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
+    int* err = nullptr;
+    if (error_word(dev, &err) != PKV_OK) return PKV_ERR_CUDA;
+    pkv::AppendFp8Params p;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.k_scales = k_scales;
+    p.v_scales = v_scales;
+    p.k = k;
+    p.v = v;
+    p.slot_mapping = slot_mapping;
+    p.err = err;
+    p.num_slots = (long long)num_blocks * block_size;
+    p.num_tokens = num_tokens;
+    p.num_kv_heads = num_kv_heads;
+    p.block_size = block_size;
+    p.chunks_per_row = head_dim / 16;
+    const long long rows = (long long)num_tokens * num_kv_heads;
+    const long long rows_per_cta = 256 / p.chunks_per_row;
+    long long blocks = (rows + rows_per_cta - 1) / rows_per_cta;
+    if (blocks > 148LL * 16) blocks = 148LL * 16;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return launch(PKV_KERNEL_APPEND, st, [&] {
+        pkv::kv_append_fp8_kernel<<<(unsigned)blocks, 256, 0, st>>>(p);
+        return cudaGetLastError();
+    });
+}
+
 int copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_pairs, int num_pairs,
                 int num_kv_heads, int head_dim, int block_size, int num_blocks, int dtype,
                 void* stream) {
@@ -381,7 +467,7 @@ int copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_pairs, int 
     if (!k_cache || !v_cache || !src_dst_pairs) return PKV_ERR_NULL;
     if (num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
         return PKV_ERR_INVALID;
-    if (dtype != PKV_F32 && dtype != PKV_BF16) return PKV_ERR_INVALID;
+    if (!known_dtype(dtype)) return PKV_ERR_INVALID;
     const long long block_bytes = (long long)num_kv_heads * block_size * head_dim * elt_bytes(dtype);
     if (block_bytes % 16 != 0) return PKV_ERR_UNSUPPORTED;
     if (!aligned16(k_cache) || !aligned16(v_cache)) return PKV_ERR_INVALID;
@@ -419,7 +505,7 @@ int swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
     if (num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_src_blocks <= 0 ||
         num_dst_blocks <= 0 || num_pairs > 65535)
         return PKV_ERR_INVALID;
-    if (dtype != PKV_F32 && dtype != PKV_BF16) return PKV_ERR_INVALID;
+    if (!known_dtype(dtype)) return PKV_ERR_INVALID;
     const long long block_bytes = (long long)num_kv_heads * block_size * head_dim * elt_bytes(dtype);
     if (block_bytes % 16 != 0) return PKV_ERR_UNSUPPORTED;
     // every pointer must be device memory or page-locked host memory the

@@ -4,6 +4,8 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -151,6 +153,27 @@ struct Elem<__nv_bfloat16> {
     }
     static __device__ __forceinline__ void store(__nv_bfloat16* dst, float v) {
         *dst = __float2bfloat16_rn(v);
+    }
+};
+
+// fp8 e4m3 cache elements (stored value = code * per-kv-head scale).
+template <>
+struct Elem<__nv_fp8_e4m3> {
+    static constexpr int kPer16B = 16;
+    // 16 bytes -> 16 floats, each code widened exactly (e4m3 -> f16 -> f32)
+    static __device__ __forceinline__ void unpack(const uint4& r, float* f) {
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
+                    (__nv_fp8x2_storage_t)((w[i] >> (16 * h)) & 0xffffu), __NV_E4M3);
+                const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+                f[4 * i + 2 * h] = f2.x;
+                f[4 * i + 2 * h + 1] = f2.y;
+            }
+        }
     }
 };
 

@@ -57,6 +57,8 @@ struct DecodeParams {
     float* ws_o;    // [B][H][P][D] unnormalised partial outputs
     float2* ws_ml;  // [B][H][P] (running max in log2 units, running sum)
     int* counters;  // [B][Hkv] partitions finished, zero between launches
+    const float* k_scales;  // fp8 caches: per-kv-head dequantisation scales (else null)
+    const float* v_scales;
     int* err;
     int num_seqs;
     int num_heads;
@@ -68,11 +70,12 @@ struct DecodeParams {
     float qscale;        // scale * log2(e)
 };
 
-template <typename T, int D, int BS, int G>
+// T: type of q and out; TKV: type of the cached K and V (T, or fp8 e4m3).
+template <typename T, typename TKV, int D, int BS, int G>
 struct DecodeCfg {
-    static constexpr int GW = G < 4 ? G : 4;  // query heads per warp
+    static constexpr int EPC = Elem<TKV>::kPer16B;
+    static constexpr int GW = G < (EPC > 8 ? 2 : 4) ? G : (EPC > 8 ? 2 : 4);  // query heads per warp
     static constexpr int NHS = G / GW;        // warps sharing one staged block
-    static constexpr int EPC = Elem<T>::kPer16B;
     static constexpr int CPR = D / EPC;        // 16-byte chunks per row
     static constexpr int RPI = 32 / CPR;       // rows covered by one warp-wide load
     static constexpr int ST = 16;              // tokens per stage: two bs-8 blocks, a bs-16 block,
@@ -86,7 +89,7 @@ struct DecodeCfg {
     static constexpr int NBL = 4;              // block lanes
     static constexpr int NCW = NBL * NHS;      // consumer warps
     static constexpr int THREADS = (NCW + 1) * 32;
-    static constexpr int ROWB = D * (int)sizeof(T);       // bytes of one token row
+    static constexpr int ROWB = D * (int)sizeof(TKV);     // bytes of one token row
     static constexpr int SLICE = BS * ROWB;               // bytes of one (block, kv head)
     static constexpr int STAGE_K = ST * ROWB;             // K rows of one stage
     static constexpr int STAGE = 2 * STAGE_K;             // K rows + V rows
@@ -253,10 +256,12 @@ __device__ __forceinline__ void zero_rows(const DecodeParams& p, int s, int g) {
     for (int i = threadIdx.x; i < G * D; i += blockDim.x) Elem<T>::store(out + i, 0.f);
 }
 
-template <typename T, int D, int BS, int G>
-__global__ void __launch_bounds__(DecodeCfg<T, D, BS, G>::THREADS, 2)
+template <typename T, typename TKV, int D, int BS, int G>
+__global__ void __launch_bounds__(DecodeCfg<T, TKV, D, BS, G>::THREADS,
+                                  DecodeCfg<T, TKV, D, BS, G>::THREADS > 320 ? 1 : 2)
     decode_partition_kernel(const DecodeParams p) {
-    using C = DecodeCfg<T, D, BS, G>;
+    using C = DecodeCfg<T, TKV, D, BS, G>;
+    constexpr bool kFp8 = sizeof(TKV) == 1;
     extern __shared__ __align__(128) unsigned char smem[];
 
     const int P = p.num_partitions;
@@ -393,14 +398,19 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, BS, G>::THREADS, 2)
     } else {
         // ------------------------------------------------------ consumers
         const int hbase = g * G + hs * C::GW;
+        // fp8 caches: the kv head's K scale folds into the logit scale
+        const float qs = kFp8 ? p.qscale * p.k_scales[g] : p.qscale;
         float qf[C::GW][C::EPC];
 #pragma unroll
         for (int gi = 0; gi < C::GW; ++gi) {
+            // this lane's EPC dims of q (one or more 16-byte loads of T)
             const uint4* qrow = reinterpret_cast<const uint4*>(
-                static_cast<const T*>(p.q) + ((long long)s * p.num_heads + hbase + gi) * D);
-            Elem<T>::unpack(qrow[c], qf[gi]);
+                static_cast<const T*>(p.q) + ((long long)s * p.num_heads + hbase + gi) * D + c * C::EPC);
+            constexpr int QL = C::EPC / Elem<T>::kPer16B;
 #pragma unroll
-            for (int e = 0; e < C::EPC; ++e) qf[gi][e] *= p.qscale;
+            for (int u = 0; u < QL; ++u) Elem<T>::unpack(qrow[u], qf[gi] + u * Elem<T>::kPer16B);
+#pragma unroll
+            for (int e = 0; e < C::EPC; ++e) qf[gi][e] *= qs;
         }
         float* my_pscr = pscr + (warp * C::RPI + r0) * (C::RPL * C::GW);
         const int vbase_idx = (C::V >= C::CPR) ? c * C::VPL : c / (C::CPR / C::V);
@@ -442,7 +452,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, BS, G>::THREADS, 2)
                     for (int k = 0; k < C::RPL; ++k) {
                         const int row = rbase + r0 + k * C::RPI;
                         float kf[C::EPC];
-                        Elem<T>::unpack(Ks[row * C::CPR + c], kf);
+                        Elem<TKV>::unpack(Ks[row * C::CPR + c], kf);
 #pragma unroll
                         for (int gi = 0; gi < C::GW; ++gi) {
                             float acc = 0.f;
@@ -515,7 +525,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, BS, G>::THREADS, 2)
                             pk[0] = my_pscr[k];
                         }
                         float vf[C::EPC];
-                        Elem<T>::unpack(Vs[row * C::CPR + c], vf);
+                        Elem<TKV>::unpack(Vs[row * C::CPR + c], vf);
                         if (tail && !((rowmask >> row) & 1u)) continue;  // never read an unused slot into o
 #pragma unroll
                         for (int gi = 0; gi < C::GW; ++gi)
@@ -573,6 +583,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, BS, G>::THREADS, 2)
 
     const int H = p.num_heads;
     const long long sh0 = (long long)s * H + (long long)g * G;  // first query head of the group
+    const float vsc = kFp8 ? p.v_scales[g] : 1.f;  // fp8: the kv head's V scale
     for (int t = tid; t < G * D; t += blockDim.x) {
         const int hg = t / D;
         const int d = t % D;
@@ -589,6 +600,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, BS, G>::THREADS, 2)
                 O = fmaf(w, row[d], O);
             }
         }
+        O *= vsc;
         const long long sh = sh0 + hg;
         if (nparts == 1) {
             Elem<T>::store(static_cast<T*>(p.out) + sh * D + d, L > 0.f ? O / L : 0.f);

@@ -9,10 +9,10 @@
 
 namespace pkv {
 
-template <typename T, int D, int BS, int G>
+template <typename T, typename TKV, int D, int BS, int G>
 cudaError_t launch_partition_inst(const DecodeParams& p, long long grid, cudaStream_t st) {
-    using C = DecodeCfg<T, D, BS, G>;
-    auto kern = decode_partition_kernel<T, D, BS, G>;
+    using C = DecodeCfg<T, TKV, D, BS, G>;
+    auto kern = decode_partition_kernel<T, TKV, D, BS, G>;
     static std::atomic<unsigned long long> configured{0};  // one bit per device
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -29,34 +29,35 @@ cudaError_t launch_partition_inst(const DecodeParams& p, long long grid, cudaStr
     return cudaGetLastError();
 }
 
-template <typename T, int D, int BS>
+template <typename T, typename TKV, int D, int BS>
 cudaError_t dispatch_group(const DecodeParams& p, int G, long long grid, cudaStream_t st) {
     switch (G) {
-        case 1: return launch_partition_inst<T, D, BS, 1>(p, grid, st);
-        case 2: return launch_partition_inst<T, D, BS, 2>(p, grid, st);
-        case 4: return launch_partition_inst<T, D, BS, 4>(p, grid, st);
-        case 8: return launch_partition_inst<T, D, BS, 8>(p, grid, st);
+        case 1: return launch_partition_inst<T, TKV, D, BS, 1>(p, grid, st);
+        case 2: return launch_partition_inst<T, TKV, D, BS, 2>(p, grid, st);
+        case 4: return launch_partition_inst<T, TKV, D, BS, 4>(p, grid, st);
+        case 8: return launch_partition_inst<T, TKV, D, BS, 8>(p, grid, st);
         default: return cudaErrorInvalidValue;
     }
 }
 
-template <typename T, int D>
+template <typename T, typename TKV, int D>
 cudaError_t dispatch_block_size(const DecodeParams& p, int BS, int G, long long grid,
                                 cudaStream_t st) {
     switch (BS) {
-        case 8: return dispatch_group<T, D, 8>(p, G, grid, st);
-        case 16: return dispatch_group<T, D, 16>(p, G, grid, st);
-        case 32: return dispatch_group<T, D, 32>(p, G, grid, st);
+        case 8: return dispatch_group<T, TKV, D, 8>(p, G, grid, st);
+        case 16: return dispatch_group<T, TKV, D, 16>(p, G, grid, st);
+        case 32: return dispatch_group<T, TKV, D, 32>(p, G, grid, st);
         default: return cudaErrorInvalidValue;
     }
 }
 
-template <typename T>
+// q / out of type T, cached K / V of type TKV
+template <typename T, typename TKV = T>
 cudaError_t dispatch_partition(const DecodeParams& p, int D, int BS, int G, long long grid,
                                cudaStream_t st) {
     switch (D) {
-        case 64: return dispatch_block_size<T, 64>(p, BS, G, grid, st);
-        case 128: return dispatch_block_size<T, 128>(p, BS, G, grid, st);
+        case 64: return dispatch_block_size<T, TKV, 64>(p, BS, G, grid, st);
+        case 128: return dispatch_block_size<T, TKV, 128>(p, BS, G, grid, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -67,6 +67,79 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
     }
 }
 
+// Append with quantisation to fp8 e4m3 (per-kv-head scales): each thread
+// writes one 16-byte chunk of codes (16 elements) of one (token, kv head)
+// row from 32 bytes of bf16 input: code = e4m3(x / scale), the division
+// correctly rounded in fp32, round-to-nearest-even and saturation to +-448
+// in the conversion.
+struct AppendFp8Params {
+    void* k_cache;
+    void* v_cache;
+    const float* k_scales;
+    const float* v_scales;
+    const void* k;  // bf16 [T][Hkv][D]
+    const void* v;
+    const int64_t* slot_mapping;
+    int* err;
+    long long num_slots;
+    int num_tokens;
+    int num_kv_heads;
+    int block_size;
+    int chunks_per_row;  // head_dim / 16
+};
+
+__device__ __forceinline__ uint4 quantise16(const uint4 a, const uint4 b, float scale) {
+    const uint32_t in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t out[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t packed = 0;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t w = in[2 * i + h];  // two bf16 values
+            const float x0 = __uint_as_float(w << 16);
+            const float x1 = __uint_as_float(w & 0xffff0000u);
+            const __nv_fp8x2_storage_t q = __nv_cvt_float2_to_fp8x2(
+                make_float2(__fdiv_rn(x0, scale), __fdiv_rn(x1, scale)), __NV_SATFINITE, __NV_E4M3);
+            packed |= (uint32_t)q << (16 * h);
+        }
+        out[i] = packed;
+    }
+    return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+__global__ void __launch_bounds__(256) kv_append_fp8_kernel(const AppendFp8Params p) {
+    const int cpr = p.chunks_per_row;
+    const int rows_per_cta = blockDim.x / cpr;
+    const int r_in = threadIdx.x / cpr;
+    const int ch = threadIdx.x - r_in * cpr;
+    if (r_in >= rows_per_cta) return;
+    const long long nrows = (long long)p.num_tokens * p.num_kv_heads;
+    uint4* kc = static_cast<uint4*>(p.k_cache);
+    uint4* vc = static_cast<uint4*>(p.v_cache);
+    const uint4* kn = static_cast<const uint4*>(p.k);
+    const uint4* vn = static_cast<const uint4*>(p.v);
+    for (long long row = (long long)blockIdx.x * rows_per_cta + r_in; row < nrows;
+         row += (long long)gridDim.x * rows_per_cta) {
+        const long long x = (row * cpr + ch) * 2;  // two bf16 chunks per fp8 chunk
+        const uint4 k0 = kn[x], k1 = kn[x + 1];
+        const uint4 v0 = vn[x], v1 = vn[x + 1];
+        const long long i = row / p.num_kv_heads;
+        const long long g = row - i * p.num_kv_heads;
+        const long long slot = p.slot_mapping[i];
+        if (slot < 0) continue;  // -1: nothing to write for this token
+        if (slot >= p.num_slots) {
+            if (ch == 0 && g == 0) set_error(p.err, PKV_ERR_DEVICE_BOUNDS);
+            continue;
+        }
+        const long long blk = slot / p.block_size;
+        const long long off = slot - blk * p.block_size;
+        const long long dst = ((blk * p.num_kv_heads + g) * p.block_size + off) * cpr + ch;
+        kc[dst] = quantise16(k0, k1, p.k_scales[g]);
+        vc[dst] = quantise16(v0, v1, p.v_scales[g]);
+    }
+}
+
 struct CopyParams {
     void* dst_k;
     void* dst_v;

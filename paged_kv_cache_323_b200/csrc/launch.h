@@ -11,6 +11,9 @@ cudaError_t launch_decode_partition_f32(const DecodeParams& p, int D, int BS, in
                                         cudaStream_t st);
 cudaError_t launch_decode_partition_bf16(const DecodeParams& p, int D, int BS, int G,
                                          long long grid, cudaStream_t st);
+// fp8 (e4m3) caches, bf16 q and out, per-kv-head scales in p.k_scales / p.v_scales
+cudaError_t launch_decode_partition_fp8(const DecodeParams& p, int D, int BS, int G,
+                                        long long grid, cudaStream_t st);
 
 // Tensor-core (tcgen05) kernel for grouped-query heads: bf16, head_dim 128,
 // groups of 2, 4 or 8, partitions a multiple of 128 tokens.

@@ -34,6 +34,7 @@ PKV_ERR_TIMEOUT = -7
 PKV_ERR_OUT_OF_BLOCKS = -8
 PKV_F32 = 0
 PKV_BF16 = 1
+PKV_FP8_E4M3 = 2
 KERNEL_DECODE = 0
 KERNEL_APPEND = 1
 KERNEL_COPY_BLOCKS = 2
@@ -49,6 +50,9 @@ SIGNATURES = {
     "paged_attention_decode_ex": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float,
                                        _I, _I, _I, _P, _SZ, _P]),
     "paged_attention_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "paged_attention_decode_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
+                                        ctypes.c_float, _I, _I, _P, _SZ, _P]),
+    "kv_cache_append_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "paged_attention_partition_tokens": (_I, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "paged_attention_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
                                             ctypes.c_float, _I, _I, _I, _P]),
@@ -110,6 +114,8 @@ def _dtype_code(t: torch.Tensor) -> int:
         return PKV_F32
     if t.dtype == torch.bfloat16:
         return PKV_BF16
+    if t.dtype == torch.float8_e4m3fn:
+        return PKV_FP8_E4M3
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
@@ -163,6 +169,45 @@ def paged_attention_decode_ex(out, q, k_cache, v_cache, block_tables, context_le
         _dev(context_lens, "context_lens", torch.int32), B, H, Hkv, D, bs, maxb, float(scale),
         int(num_blocks), code, int(partition_tokens), ws_ptr, ws_bytes, _stream(stream))
     _check(rc, "paged_attention_decode_ex")
+
+
+def paged_attention_decode_fp8(out, q, k_cache, v_cache, k_scales, v_scales, block_tables,
+                               context_lens, scale: float, *, num_blocks: int | None = None,
+                               partition_tokens: int = 0, workspace: torch.Tensor | None = None,
+                               stream=None) -> None:
+    """fp8 (float8_e4m3fn) caches with per-kv-head float32 scales (CUDA
+    tensors [num_kv_heads]); q and out bf16."""
+    B, H, D = q.shape
+    N, Hkv, bs, D2 = k_cache.shape
+    if D2 != D or tuple(out.shape) != (B, H, D) or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("shape mismatch between q, out and the caches")
+    maxb = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    need = paged_attention_workspace_size(B, H, maxb * bs, D, partition_tokens)
+    if workspace is None and need > 0:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
+    rc = lib.paged_attention_decode_fp8(
+        _dev(out, "out", torch.bfloat16), _dev(q, "q", torch.bfloat16),
+        _dev(k_cache, "k_cache", torch.float8_e4m3fn), _dev(v_cache, "v_cache", torch.float8_e4m3fn),
+        _dev(k_scales, "k_scales", torch.float32), _dev(v_scales, "v_scales", torch.float32),
+        _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32), B, H, Hkv, D, bs, maxb, float(scale),
+        N if num_blocks is None else int(num_blocks), int(partition_tokens),
+        workspace.data_ptr() if workspace is not None else None,
+        workspace.numel() if workspace is not None else 0, _stream(stream))
+    _check(rc, "paged_attention_decode_fp8")
+
+
+def kv_cache_append_fp8(k_cache, v_cache, k_scales, v_scales, k, v, slot_mapping, stream=None) -> None:
+    """Quantise bf16 rows k, v [T][Hkv][D] into the fp8 pools."""
+    T = slot_mapping.shape[0]
+    N, Hkv, bs, D = k_cache.shape
+    rc = lib.kv_cache_append_fp8(
+        _dev(k_cache, "k_cache", torch.float8_e4m3fn), _dev(v_cache, "v_cache", torch.float8_e4m3fn),
+        _dev(k_scales, "k_scales", torch.float32), _dev(v_scales, "v_scales", torch.float32),
+        _dev(k, "k", torch.bfloat16) if T else None, _dev(v, "v", torch.bfloat16) if T else None,
+        _dev(slot_mapping, "slot_mapping", torch.int64) if T else None, T, Hkv, D, bs, N,
+        _stream(stream))
+    _check(rc, "kv_cache_append_fp8")
 
 
 # Size of the fixed device scratch of paged_attention_decode_noalloc.

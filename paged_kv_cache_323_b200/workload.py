@@ -33,7 +33,7 @@ from dataclasses import dataclass, field
 import numpy as np
 import torch
 
-DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}
+DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.float8_e4m3fn}
 
 
 @dataclass
@@ -60,6 +60,8 @@ class Workload:
     k_new: torch.Tensor  # [T][Hkv][D]
     v_new: torch.Tensor
     meta: dict = field(default_factory=dict)
+    k_scales: np.ndarray | None = None  # fp8 caches: float32 [Hkv], stored value = code * scale
+    v_scales: np.ndarray | None = None
 
     @property
     def group(self) -> int:
@@ -67,7 +69,7 @@ class Workload:
 
     @property
     def elt(self) -> int:
-        return 4 if self.dtype == "f32" else 2
+        return {"f32": 4, "bf16": 2, "fp8": 1}[self.dtype]
 
     def kv_bytes_logical(self) -> int:
         """K and V bytes one decode step reads, counting every sequence."""
@@ -91,14 +93,25 @@ class _Pool:
         return b
 
 
-def _normal(shape, rng: np.random.Generator, tgen, device, dtype: str, mult: float = 1.0):
+def _normal(shape, rng: np.random.Generator, tgen, device, dtype: str, mult=1.0):
+    """N(0, 1) fp32 draws times `mult` (a number, or per-kv-head values
+    broadcast over dim 1), rounded to `dtype` (nearest even, by torch)."""
     if device == "cpu" or device is None:
         x = torch.from_numpy(rng.standard_normal(size=shape, dtype=np.float32))
     else:
         x = torch.randn(*shape, generator=tgen, device=device, dtype=torch.float32)
-    if mult != 1.0:
+    if isinstance(mult, np.ndarray):
+        x = x * torch.from_numpy(mult.astype(np.float32)).to(x.device).view(1, -1, *([1] * (len(shape) - 2)))
+    elif mult != 1.0:
         x = x * mult
     return x.to(DTYPES[dtype]).contiguous()
+
+
+def fp8_scales(num_kv_heads: int):
+    """Per-kv-head scales of the fp8 workloads (stored value = code * scale):
+    codes of N(0, 1) / scale stay well inside e4m3's +-448."""
+    g = np.arange(num_kv_heads, dtype=np.float32)
+    return ((1.0 + 0.37 * g) / 32.0).astype(np.float32), ((1.0 + 0.21 * g) / 24.0).astype(np.float32)
 
 
 def _finish(name, dtype, rng, seed, device, *, lens, tables, cow_pairs, new_pos, num_blocks,
@@ -115,12 +128,18 @@ def _finish(name, dtype, rng, seed, device, *, lens, tables, cow_pairs, new_pos,
     if device not in (None, "cpu"):
         tgen = torch.Generator(device=device)
         tgen.manual_seed(seed)
-    q = _normal((B, H, D), rng, tgen, device, dtype, q_mult)
-    k_cache = _normal((num_blocks, Hkv, bs, D), rng, tgen, device, dtype)
-    v_cache = _normal((num_blocks, Hkv, bs, D), rng, tgen, device, dtype)
+    act = "bf16" if dtype == "fp8" else dtype  # q and new tokens of an fp8 cache are bf16
+    ks = vs = None
+    kmul = vmul = 1.0
+    if dtype == "fp8":
+        ks, vs = fp8_scales(Hkv)
+        kmul, vmul = 1.0 / ks, 1.0 / vs
+    q = _normal((B, H, D), rng, tgen, device, act, q_mult)
+    k_cache = _normal((num_blocks, Hkv, bs, D), rng, tgen, device, dtype, kmul)
+    v_cache = _normal((num_blocks, Hkv, bs, D), rng, tgen, device, dtype, vmul)
     T = len(slot_mapping)
-    k_new = _normal((T, Hkv, D), rng, tgen, device, dtype)
-    v_new = _normal((T, Hkv, D), rng, tgen, device, dtype)
+    k_new = _normal((T, Hkv, D), rng, tgen, device, act)
+    v_new = _normal((T, Hkv, D), rng, tgen, device, act)
     bt = np.full((B, maxb), -1, dtype=np.int32)
     for s, row in enumerate(tables):
         bt[s, : len(row)] = row
@@ -131,7 +150,7 @@ def _finish(name, dtype, rng, seed, device, *, lens, tables, cow_pairs, new_pos,
         block_tables=bt, cow_pairs=np.asarray(cow_pairs, dtype=np.int64).reshape(-1, 2),
         slot_mapping=slot_mapping, token_seq=np.asarray(owners, dtype=np.int32),
         pair_seq=np.asarray(pair_seq, dtype=np.int32), q=q, k_cache=k_cache, v_cache=v_cache, k_new=k_new,
-        v_new=v_new, meta=meta or {})
+        v_new=v_new, meta=meta or {}, k_scales=ks, v_scales=vs)
 
 
 class _InOrderPool(_Pool):
@@ -305,6 +324,8 @@ def to_numpy_bits(t: torch.Tensor) -> np.ndarray:
         return t.view(torch.int16).numpy().view(np.uint16)
     if t.dtype == torch.float32:
         return t.numpy()
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8).numpy()
     raise TypeError(t.dtype)
 
 

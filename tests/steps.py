@@ -46,10 +46,19 @@ def gpu_step(w: wl.Workload, t: dict | None = None, partition_tokens: int = 0,
         t = to_device(w)
     if len(w.cow_pairs):
         pk.copy_blocks(t["k_cache"], t["v_cache"], t["cow_pairs"])
-    pk.kv_cache_append(t["k_cache"], t["v_cache"], t["k_new"], t["v_new"], t["slot_mapping"])
-    pk.paged_attention_decode_ex(t["out"], t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
-                                 t["context_lens"], w.scale, num_blocks=w.num_blocks,
-                                 partition_tokens=partition_tokens)
+    if w.dtype == "fp8":
+        ks = torch.from_numpy(w.k_scales).to(t["q"].device)
+        vs = torch.from_numpy(w.v_scales).to(t["q"].device)
+        pk.kv_cache_append_fp8(t["k_cache"], t["v_cache"], ks, vs, t["k_new"], t["v_new"],
+                               t["slot_mapping"])
+        pk.paged_attention_decode_fp8(t["out"], t["q"], t["k_cache"], t["v_cache"], ks, vs,
+                                      t["block_tables"], t["context_lens"], w.scale,
+                                      num_blocks=w.num_blocks, partition_tokens=partition_tokens)
+    else:
+        pk.kv_cache_append(t["k_cache"], t["v_cache"], t["k_new"], t["v_new"], t["slot_mapping"])
+        pk.paged_attention_decode_ex(t["out"], t["q"], t["k_cache"], t["v_cache"],
+                                     t["block_tables"], t["context_lens"], w.scale,
+                                     num_blocks=w.num_blocks, partition_tokens=partition_tokens)
     torch.cuda.synchronize()
     if check_error:
         code = pk.get_device_error()
@@ -63,6 +72,12 @@ def oracle_step(w: wl.Workload):
     vc = wl.to_numpy_bits(w.v_cache).copy()
     if len(w.cow_pairs):
         oracle.copy_blocks(kc, vc, w.cow_pairs)
+    if w.dtype == "fp8":
+        oracle.kv_append_fp8(kc, vc, w.k_scales, w.v_scales, wl.to_numpy_bits(w.k_new),
+                             wl.to_numpy_bits(w.v_new), w.slot_mapping)
+        out = oracle.paged_attention_fp8(wl.to_numpy_bits(w.q), kc, vc, w.k_scales, w.v_scales,
+                                         w.block_tables, w.context_lens, w.scale)
+        return out, kc, vc
     oracle.kv_append(kc, vc, wl.to_numpy_bits(w.k_new), wl.to_numpy_bits(w.v_new), w.slot_mapping)
     out = oracle.paged_attention(wl.to_numpy_bits(w.q), kc, vc, w.block_tables, w.context_lens,
                                  w.scale)
@@ -109,8 +124,12 @@ def subset(w: wl.Workload, seqs, pool_device_k=None, pool_device_v=None) -> wl.W
     order = sorted(blocks)
     remap = {b: i for i, b in enumerate(order)}
     idx = torch.tensor(order, dtype=torch.long, device=kpool.device)
-    k_sub = kpool.index_select(0, idx).cpu()
-    v_sub = vpool.index_select(0, idx).cpu()
+    if kpool.dtype == torch.float8_e4m3fn:  # gather the codes as bytes
+        k_sub = kpool.view(torch.uint8).index_select(0, idx).cpu().view(torch.float8_e4m3fn)
+        v_sub = vpool.view(torch.uint8).index_select(0, idx).cpu().view(torch.float8_e4m3fn)
+    else:
+        k_sub = kpool.index_select(0, idx).cpu()
+        v_sub = vpool.index_select(0, idx).cpu()
     bt = np.full((len(seqs), w.max_blocks_per_seq), -1, dtype=np.int32)
     for i, s in enumerate(seqs):
         nb = -(-int(w.context_lens[s]) // bs)
@@ -132,4 +151,5 @@ def subset(w: wl.Workload, seqs, pool_device_k=None, pool_device_v=None) -> wl.W
         pair_seq=np.asarray([seqs.index(int(w.pair_seq[i])) for i in sel_pairs], dtype=np.int32),
         q=w.q.index_select(0, seq_idx.to(w.q.device)).cpu(), k_cache=k_sub, v_cache=v_sub,
         k_new=w.k_new.index_select(0, tok_idx.to(w.k_new.device)).cpu(),
-        v_new=w.v_new.index_select(0, tok_idx.to(w.v_new.device)).cpu(), meta={})
+        v_new=w.v_new.index_select(0, tok_idx.to(w.v_new.device)).cpu(), meta={},
+        k_scales=w.k_scales, v_scales=w.v_scales)
