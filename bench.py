@@ -543,7 +543,8 @@ def run_gpu(args, world, rank, local):
                    "partition_tokens": pk.paged_attention_partition_tokens(
                        w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.block_size,
                        w.max_blocks_per_seq * w.block_size,
-                       pk.PKV_F32 if w.dtype == "f32" else pk.PKV_BF16, args.partition_tokens),
+                       {"f32": pk.PKV_F32, "bf16": pk.PKV_BF16, "fp8": pk.PKV_FP8_E4M3}[w.dtype],
+                       args.partition_tokens),
                    "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush",
                    "parallelism": f"{world} independent batches, one per GPU"},
         "tokens_per_s": world * w.num_seqs / step_s,

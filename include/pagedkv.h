@@ -256,6 +256,13 @@ PKV_API int swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void*
  * (PKV_OK, PKV_ERR_DEVICE_BOUNDS or PKV_ERR_TIMEOUT) and clear it. */
 PKV_API int pkv_get_device_error(void* stream, int* code);
 
+/* Self-test of the failure path: launches one warp that waits, with the
+ * kernels' bounded wait, on a barrier nothing arrives at; after timeout_us
+ * microseconds (1 .. 1e6) the wait gives up and the device error word becomes
+ * PKV_ERR_TIMEOUT (read it with pkv_get_device_error).  Nothing traps and the
+ * context stays usable. */
+PKV_API int pkv_selftest_bounded_wait(int timeout_us, void* stream);
+
 /* Static English text of a status code. */
 PKV_API const char* pkv_status_string(int status);
 

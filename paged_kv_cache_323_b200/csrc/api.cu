@@ -154,7 +154,8 @@ size_t workspace_bytes_for(long long num_seqs, long long num_heads, long long pa
 //    fixed set-up and drain cost, so long partitions pay: on B200 the
 //    parallel-sampling GQA batch ran at 0.55 / 0.75 / 0.88 / 0.97 of peak
 //    with 512 / 1024 / 2048 / 4096-token partitions.
-int auto_partition_tokens(long long num_seqs, long long num_kv_heads, long long max_ctx, bool tc) {
+int auto_partition_tokens(long long num_seqs, long long num_kv_heads, long long max_ctx, bool tc,
+                          bool fp8 = false) {
     if (tc) {
         long long pt = kMaxPartitionTokens;
         const long long min_ctas = 8LL * 148 * 2;
@@ -162,7 +163,9 @@ int auto_partition_tokens(long long num_seqs, long long num_kv_heads, long long 
             pt /= 2;
         return (int)pt;
     }
-    long long pt = kAutoPartitionTokens;
+    // fp8 caches carry half the bytes per token, so a CTA's fixed cost weighs
+    // twice as much: 2048 tokens (on batch-64 MHA 154 us at 1024, 139 us at 2048)
+    long long pt = fp8 ? 2 * kAutoPartitionTokens : kAutoPartitionTokens;
     const long long min_ctas = 4LL * 148 * 3;
     while (pt < kMaxPartitionTokens && (max_ctx + pt - 1) / pt > 64 &&
            num_seqs * num_kv_heads * ((max_ctx + 2 * pt - 1) / (2 * pt)) >= min_ctas)
@@ -181,7 +184,8 @@ int resolve_partition_tokens(int num_seqs, int num_heads, int num_kv_heads, int 
     if (partition_tokens != 0) return partition_tokens;
     const int group = num_kv_heads > 0 ? num_heads / num_kv_heads : 1;
     return auto_partition_tokens(num_seqs, num_kv_heads, max_ctx,
-                                 tc_shape(dtype, head_dim, block_size, group));
+                                 tc_shape(dtype, head_dim, block_size, group),
+                                 dtype == PKV_FP8_E4M3);
 }
 
 }  // namespace
@@ -550,6 +554,17 @@ int swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
         pkv::copy_blocks_kernel<<<dim3((unsigned)per_pair, (unsigned)num_pairs), 256, 0, st>>>(p);
         return cudaGetLastError();
     });
+}
+
+int pkv_selftest_bounded_wait(int timeout_us, void* stream) {
+    if (timeout_us <= 0 || timeout_us > 1000000) return PKV_ERR_INVALID;
+    int dev = 0;
+    if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
+    int* err = nullptr;
+    if (error_word(dev, &err) != PKV_OK) return PKV_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    pkv::bounded_wait_selftest_kernel<<<1, 32, 0, st>>>(err, 1000ull * (unsigned long long)timeout_us);
+    return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
 int pkv_get_device_error(void* stream, int* code) {

@@ -78,8 +78,10 @@ struct DecodeCfg {
     static constexpr int NHS = G / GW;        // warps sharing one staged block
     static constexpr int CPR = D / EPC;        // 16-byte chunks per row
     static constexpr int RPI = 32 / CPR;       // rows covered by one warp-wide load
-    static constexpr int ST = 16;              // tokens per stage: two bs-8 blocks, a bs-16 block,
-                                               // or half of a bs-32 block
+    // tokens per stage: 16 (two bs-8 blocks, a bs-16 block or half of a bs-32
+    // block), 32 for one-byte (fp8) caches so a stage still carries 4 KB of K
+    static constexpr int ST = sizeof(TKV) == 1 ? 32 : 16;
+    static constexpr uint32_t FULL_ROWS = ST == 32 ? 0xffffffffu : ((1u << ST) - 1u);
     static constexpr int TR = ST;              // rows per sub-tile (one stage)
     static constexpr int BPS = BS < ST ? ST / BS : 1;  // whole blocks per stage
     static constexpr int RPL = TR / RPI;       // rows per lane per sub-tile
@@ -443,7 +445,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, TKV, D, BS, G>::THREADS,
             if (rowmask != 0) {
                 const uint4* Ks = reinterpret_cast<const uint4*>(stages + st * C::STAGE);
                 const uint4* Vs = reinterpret_cast<const uint4*>(stages + st * C::STAGE + C::STAGE_K);
-                const bool tail = rowmask != (1u << C::ST) - 1u;
+                const bool tail = rowmask != C::FULL_ROWS;
                 {
                     constexpr int rbase = 0;
                     // ---- QK^T: partial dot products over this lane's chunk

@@ -193,4 +193,21 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(const CopyParams p) {
     }
 }
 
+// Self-test of the failure path: one warp waits, with the same bounded wait
+// the kernels use, on an mbarrier that nothing ever arrives at.  The wait
+// gives up after timeout_ns, records PKV_ERR_TIMEOUT and the kernel returns;
+// no trap, and the context stays usable.
+__global__ void bounded_wait_selftest_kernel(int* err, unsigned long long timeout_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    __syncthreads();
+    const bool ok = mbar_wait_bounded(&bar, 0, &abort_flag, timeout_ns);
+    if (!__all_sync(0xffffffffu, ok) && threadIdx.x == 0) set_error(err, PKV_ERR_TIMEOUT);
+}
+
 }  // namespace pkv

@@ -72,6 +72,7 @@ SIGNATURES = {
     "pkv_bm_swap_in": (_I, [_P, _I, _P, _I, ctypes.POINTER(_I)]),
     "pkv_bm_get_stats": (_I, [_P, _P]),
     "pkv_get_device_error": (_I, [_P, ctypes.POINTER(_I)]),
+    "pkv_selftest_bounded_wait": (_I, [_I, _P]),
     "pkv_status_string": (ctypes.c_char_p, [_I]),
     "pkv_profile_enable": (_I, [_I]),
     "pkv_profile_read": (_I, [_I, ctypes.POINTER(ctypes.c_longlong), ctypes.POINTER(ctypes.c_double)]),
@@ -401,6 +402,11 @@ def get_device_error(stream=None) -> int:
     code = ctypes.c_int(0)
     _check(lib.pkv_get_device_error(_stream(stream), ctypes.byref(code)), "pkv_get_device_error")
     return code.value
+
+
+def selftest_bounded_wait(timeout_us: int, stream=None) -> None:
+    """Launch a wait that runs out after timeout_us (see include/pagedkv.h)."""
+    _check(lib.pkv_selftest_bounded_wait(int(timeout_us), _stream(stream)), "pkv_selftest_bounded_wait")
 
 
 def profile_enable(on: bool = True) -> None:

@@ -299,3 +299,20 @@ def test_launch_count_and_profiler():
     n, _ = pk.profile_read(pk.KERNEL_APPEND)
     assert n == 1
     pk.profile_reset()
+
+
+def test_bounded_wait_runs_out_without_fault():
+    """A device wait that nothing satisfies gives up after its limit and
+    reports PKV_ERR_TIMEOUT; the context then keeps working."""
+    import time
+
+    from paged_kv_cache_323_b200 import pagedkv as pk
+
+    assert pk.get_device_error() == 0
+    t0 = time.perf_counter()
+    pk.selftest_bounded_wait(20000)  # 20 ms
+    code = pk.get_device_error()
+    elapsed = time.perf_counter() - t0
+    assert code == pk.PKV_ERR_TIMEOUT
+    assert 0.015 <= elapsed < 5.0
+    _full_check(wl.tiny())  # the context is still usable
