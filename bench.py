@@ -65,6 +65,9 @@ WORKLOADS = {
     # a smaller MHA batch for profiler captures: 16 sequences, 4096-block pool (1 GB), ~0.3 GB KV per step
     "mha_small": ("mha_decode_b16_h32_kv32_d128_bs16_ctxU128-2048_bf16_pool4096",
                   lambda dev, seed: wl.mha(seed=seed, device=dev, num_seqs=16, num_blocks=4096)),
+    "mha_bs8_small": ("mha_decode_b16_h32_kv32_d128_bs8_ctxU128-2048_bf16_pool8192",
+                      lambda dev, seed: wl.mha(seed=seed, device=dev, num_seqs=16, num_blocks=8192,
+                                               block_size=8)),
     "mha_fp8_small": ("mha_decode_b16_h32_kv32_d128_bs16_ctxU128-2048_fp8e4m3_cache_pool4096",
                       lambda dev, seed: wl.mha(seed=seed, device=dev, num_seqs=16, num_blocks=4096,
                                                dtype="fp8")),
@@ -72,7 +75,7 @@ WORKLOADS = {
 DEFAULT_SEED = {"mha": 2, "gqa_sampling": 3, "long_context": 4, "prefix_bs8": 5, "prefix_bs16": 5,
                 "prefix_bs32": 5, "tiny": 1, "mha_small": 2, "mha_bs8": 2, "mha_bs32": 2,
                 "mha_contig_bs8": 2, "mha_contig_bs16": 2, "mha_contig_bs32": 2, "mha_fp8": 2,
-                "mha_fp8_small": 2}
+                "mha_fp8_small": 2, "mha_bs8_small": 2}
 
 
 def measured_peak():

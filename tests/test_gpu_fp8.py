@@ -54,3 +54,18 @@ def test_fp8_saturates_large_values():
     w = wl.custom(5, [40, 17], heads=4, kv_heads=2, head_dim=128, block_size=16, dtype="fp8")
     w.k_new = (w.k_new.float() * 1e4).to(torch.bfloat16)
     _full_check(w)
+
+
+@pytest.mark.parametrize("q_pow2", [-30, 20, 60])
+def test_fp8_query_magnitudes(q_pow2):
+    """Queries far outside f16's range, or deep below it, with the softmax
+    scale compensating: the logits, and so the outputs, are those of the
+    unscaled query.  One dimension is also made 2^12 times larger than the
+    rest, so small elements of a head sit far below its largest."""
+    w = wl.custom(21, [1, 37, 300, 999], heads=8, kv_heads=2, head_dim=128, block_size=16,
+                  dtype="fp8")
+    q = w.q.float()
+    q[:, :, 5] *= 2.0 ** 12
+    w.q = (q * 2.0 ** q_pow2).to(torch.bfloat16)
+    w.scale = w.scale * 2.0 ** -(q_pow2 + 12)
+    _full_check(w)
