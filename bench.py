@@ -65,6 +65,11 @@ WORKLOADS = {
     # a smaller MHA batch for profiler captures: 16 sequences, 4096-block pool (1 GB), ~0.3 GB KV per step
     "mha_small": ("mha_decode_b16_h32_kv32_d128_bs16_ctxU128-2048_bf16_pool4096",
                   lambda dev, seed: wl.mha(seed=seed, device=dev, num_seqs=16, num_blocks=4096)),
+    # fp8 (e4m3) caches on the grouped-query workloads
+    "gqa_sampling_fp8": ("gqa_sampling_b256_g64x4_h32_kv8_d128_bs16_fp8e4m3_cache",
+                         lambda dev, seed: wl.gqa_sampling(seed=seed, device=dev, dtype="fp8")),
+    "long_context_fp8": ("long_context_b8_h64_kv8_d128_bs32_ctxU32768-131072_fp8e4m3_cache",
+                         lambda dev, seed: wl.long_context(seed=seed, device=dev, dtype="fp8")),
     "mha_bs8_small": ("mha_decode_b16_h32_kv32_d128_bs8_ctxU128-2048_bf16_pool8192",
                       lambda dev, seed: wl.mha(seed=seed, device=dev, num_seqs=16, num_blocks=8192,
                                                block_size=8)),
@@ -75,7 +80,7 @@ WORKLOADS = {
 DEFAULT_SEED = {"mha": 2, "gqa_sampling": 3, "long_context": 4, "prefix_bs8": 5, "prefix_bs16": 5,
                 "prefix_bs32": 5, "tiny": 1, "mha_small": 2, "mha_bs8": 2, "mha_bs32": 2,
                 "mha_contig_bs8": 2, "mha_contig_bs16": 2, "mha_contig_bs32": 2, "mha_fp8": 2,
-                "mha_fp8_small": 2, "mha_bs8_small": 2}
+                "mha_fp8_small": 2, "mha_bs8_small": 2, "gqa_sampling_fp8": 3, "long_context_fp8": 4}
 
 
 def measured_peak():
@@ -442,12 +447,16 @@ def run_gpu(args, world, rank, local):
 
     pk.profile_reset()
     pk.profile_enable(True)
+    step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     ev0.record(stream)
-    for _ in range(args.steps):
+    step_ev[0].record(stream)
+    for i in range(args.steps):
         step(*dev_args)
+        step_ev[i + 1].record(stream)
     ev1.record(stream)
     torch.cuda.synchronize()
     pk.profile_enable(False)
+    step_ms = sorted(step_ev[i].elapsed_time(step_ev[i + 1]) for i in range(args.steps))
     clock_info = clocks.stop()
     barrier(world)
     ms_profiled = max_over_ranks(world, ev0.elapsed_time(ev1))
@@ -559,6 +568,9 @@ def run_gpu(args, world, rank, local):
         "pct_of_peak_hbm": 100.0 * value / peak,
         "per_kernel_us": per_kernel,
         "ms_per_step_profiled": ms_profiled / args.steps,
+        "ms_per_step_profiled_pct": {"p10": step_ms[len(step_ms) // 10],
+                                     "p50": step_ms[len(step_ms) // 2],
+                                     "p90": step_ms[(9 * len(step_ms)) // 10]},
         "roofline": roofline,
         "gpu_launches": launches,
         "e2e": {"value": job_value(world, kv_bytes, ms_e2e / args.steps), "unit": "GB/s",
@@ -581,6 +593,11 @@ def run_gpu(args, world, rank, local):
                                 "cores": threads, "kind": "oracle",
                                 "sample": f"{n} of {w.num_seqs} sequences (seeded), all heads; "
                                           f"{steps} steps in {spent:.1f} s"}
+        # and on one core, over a smaller sample (about 3 s)
+        sub1, n1, _ = pick_sample(w, target_s=3.0, threads=1)
+        t1 = oracle_sample_step(sub1, w.scale, 1)
+        line["cpu_baseline"]["value_1_core"] = sub1["kv_bytes"] / t1 / 1e9
+        line["cpu_baseline"]["sample_1_core"] = f"{n1} of {w.num_seqs} sequences (seeded), one step"
     print(json.dumps(line), flush=True)
 
 
