@@ -118,7 +118,7 @@ def kernel_source_sha() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_323_b200", "csrc")
     for name in ("common.cuh", "decode_attn.cuh", "decode_launch.cuh", "decode_tc.cuh",
-                 "decode_tc.cu"):  # the decode kernels' source
+                 "decode_tc.cu", "decode_tc_fp8.cuh"):  # the decode kernels' source
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())

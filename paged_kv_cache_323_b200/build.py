@@ -17,7 +17,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpagedkv.so")
-SOURCES = ["api.cu", "decode_f32.cu", "decode_bf16.cu", "decode_fp8.cu", "decode_tc.cu", "noalloc.cu",
+SOURCES = ["api.cu", "decode_f32.cu", "decode_bf16.cu", "decode_fp8.cu", "decode_tc.cu", "decode_tc_fp8.cu",
+           "noalloc.cu",
            "block_manager.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + [

@@ -312,7 +312,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     const bool use_tc = g_tc_gqa.load() != 0 &&
                         pkv::decode_tc_supported(kv_dtype, head_dim, block_size, group, pt);
     return launch(PKV_KERNEL_DECODE, st, [&] {
-        if (use_tc) return pkv::launch_decode_tc(p, block_size, group, grid, st);
+        if (use_tc) return pkv::launch_decode_tc(p, kv_dtype, block_size, group, grid, st);
         if (fp8) return pkv::launch_decode_partition_fp8(p, head_dim, block_size, group, grid, st);
         return dtype == PKV_F32 ? pkv::launch_decode_partition_f32(p, head_dim, block_size, group, grid, st)
                                 : pkv::launch_decode_partition_bf16(p, head_dim, block_size, group, grid, st);

@@ -28,22 +28,28 @@ EncodeTiledFn encoder() {
     return fn;
 }
 
-// The pool [num_blocks][Hkv][bs][128] bf16 as a 4-D tensor (dims innermost
-// first: dim, slot, kv head, block); boxes of 64 dims x bs slots of one
-// (block, kv head), 128-byte swizzle.
-cudaError_t make_pool_map(CUtensorMap* map, const void* pool, int Hkv, int BS, int num_blocks) {
+}  // namespace
+
+// The pool [num_blocks][Hkv][bs][128] as a 4-D tensor (dims innermost first:
+// dim, slot, kv head, block); boxes of one 128-byte row span (64 bf16 dims or
+// 128 e4m3 codes) x bs slots of one (block, kv head), 128-byte swizzle.
+cudaError_t make_tc_pool_map(CUtensorMap* map, const void* pool, int Hkv, int BS, int num_blocks,
+                             int elem_bytes) {
     EncodeTiledFn fn = encoder();
     if (fn == nullptr) return cudaErrorNotSupported;
+    const cuuint64_t eb = (cuuint64_t)elem_bytes;
     const cuuint64_t dims[4] = {128, (cuuint64_t)BS, (cuuint64_t)Hkv, (cuuint64_t)num_blocks};
-    const cuuint64_t strides[3] = {128 * 2, (cuuint64_t)BS * 128 * 2, (cuuint64_t)Hkv * BS * 128 * 2};
-    const cuuint32_t box[4] = {64, (cuuint32_t)BS, 1, 1};
+    const cuuint64_t strides[3] = {128 * eb, (cuuint64_t)BS * 128 * eb, (cuuint64_t)Hkv * BS * 128 * eb};
+    const cuuint32_t box[4] = {(cuuint32_t)(128 / elem_bytes), (cuuint32_t)BS, 1, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(pool), dims,
-                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    const CUresult r = fn(map, elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                          4, const_cast<void*>(pool), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
+
+namespace {
 
 template <int BS, int G>
 cudaError_t launch_inst(const DecodeParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
@@ -77,18 +83,22 @@ cudaError_t launch_group(const DecodeParams& p, int G, const CUtensorMap& mk, co
 
 }  // namespace
 
-bool decode_tc_supported(int dtype, int D, int BS, int G, int partition_tokens) {
-    return dtype == PKV_BF16 && D == 128 && (BS == 8 || BS == 16 || BS == 32) &&
-           (G == 2 || G == 4 || G == 8) && partition_tokens % 128 == 0;
+bool decode_tc_supported(int kv_dtype, int D, int BS, int G, int partition_tokens) {
+    const bool shape = D == 128 && (BS == 8 || BS == 16 || BS == 32) && partition_tokens % 128 == 0;
+    if (kv_dtype == PKV_BF16) return shape && (G == 2 || G == 4 || G == 8);
+    if (kv_dtype == PKV_FP8_E4M3) return shape && (G == 1 || G == 2 || G == 4 || G == 8);
+    return false;
 }
 
-cudaError_t launch_decode_tc(const DecodeParams& p, int BS, int G, long long grid,
+cudaError_t launch_decode_tc(const DecodeParams& p, int kv_dtype, int BS, int G, long long grid,
                              cudaStream_t st) {
+    const int eb = kv_dtype == PKV_FP8_E4M3 ? 1 : 2;
     CUtensorMap mk, mv;
-    cudaError_t e = make_pool_map(&mk, p.k_cache, p.num_kv_heads, BS, p.num_blocks);
+    cudaError_t e = make_tc_pool_map(&mk, p.k_cache, p.num_kv_heads, BS, p.num_blocks, eb);
     if (e != cudaSuccess) return e;
-    e = make_pool_map(&mv, p.v_cache, p.num_kv_heads, BS, p.num_blocks);
+    e = make_tc_pool_map(&mv, p.v_cache, p.num_kv_heads, BS, p.num_blocks, eb);
     if (e != cudaSuccess) return e;
+    if (kv_dtype == PKV_FP8_E4M3) return launch_decode_tc_fp8(p, mk, mv, BS, G, grid, st);
     switch (BS) {
         case 8: return launch_group<8>(p, G, mk, mv, grid, st);
         case 16: return launch_group<16>(p, G, mk, mv, grid, st);

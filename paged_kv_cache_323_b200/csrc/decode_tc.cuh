@@ -79,13 +79,25 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem desc] . B[smem desc], bf16 inputs, fp32 accumulator.
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                         uint32_t idesc, uint32_t accumulate) {
+// D[tmem] (+)= A[smem desc] . B[smem desc], 16-bit inputs (bf16 or f16, as
+// the instruction descriptor says), fp32 accumulator.
+__device__ __forceinline__ void mma_kind_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// The same with 8-bit inputs (e4m3 here), K = 32 per instruction.
+__device__ __forceinline__ void mma_kind_f8f6f4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
@@ -133,11 +145,17 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
     return d;
 }
 
-// Instruction descriptor, kind::f16 with bf16 A and B, fp32 D.
-constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+// Instruction descriptor: fp32 D (bit 4), A and B formats (bits 7-9 and
+// 10-12: for kind::f16 0 = f16, 1 = bf16; for kind::f8f6f4 0 = e4m3), A and
+// B major-ness (bits 15, 16: 1 = MN-major), N / 8 (bits 17-22), M / 16
+// (bits 24-28).
+constexpr uint32_t idesc_make(int M, int N, uint32_t ab_format, bool a_mn_major, bool b_mn_major) {
+    return (1u << 4) | (ab_format << 7) | (ab_format << 10) | ((a_mn_major ? 1u : 0u) << 15) |
            ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
            ((uint32_t)(M >> 4) << 24);
+}
+constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
+    return idesc_make(M, N, 1u, a_mn_major, b_mn_major);
 }
 
 template <int BS, int G>
@@ -357,7 +375,7 @@ __global__ void __launch_bounds__(192, 2)
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint64_t a = sw128_desc(k_base + (kk >> 2) * C::HALF + (kk & 3) * 32, 16, 1024);
                     const uint64_t b = sw128_desc(q_base + (kk >> 2) * (C::NPAD * C::ROW) + (kk & 3) * 32, 16, 1024);
-                    mma_bf16(tmem + C::S_COL + (c & 1) * 16, a, b, C::IDESC_QK, kk > 0);
+                    mma_kind_f16(tmem + C::S_COL + (c & 1) * 16, a, b, C::IDESC_QK, kk > 0);
                 }
                 mma_commit(&s_full[c & 1]);
                 mma_commit(&empty[st]);
@@ -377,7 +395,7 @@ __global__ void __launch_bounds__(192, 2)
                     // A = V^T, MN-major: 64-dim halves C::HALF apart, 8-token groups 1024 B apart
                     const uint64_t a = sw128_desc(v_base + kk * 16 * C::ROW, C::HALF, 1024);
                     const uint64_t b = sw128_desc(p_base + (kk >> 2) * (C::NPAD * C::ROW) + (kk & 3) * 32, 16, 1024);
-                    mma_bf16(tmem + C::O_COL + (c & 1) * 16, a, b, C::IDESC_PV, kk > 0);
+                    mma_kind_f16(tmem + C::O_COL + (c & 1) * 16, a, b, C::IDESC_PV, kk > 0);
                 }
                 mma_commit(&o_full[c & 1]);
                 mma_commit(&empty[st]);

@@ -1,6 +1,7 @@
 // launch.h -- host-side entry points of the per-dtype decode translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "decode_attn.cuh"
@@ -15,9 +16,16 @@ cudaError_t launch_decode_partition_bf16(const DecodeParams& p, int D, int BS, i
 cudaError_t launch_decode_partition_fp8(const DecodeParams& p, int D, int BS, int G,
                                         long long grid, cudaStream_t st);
 
-// Tensor-core (tcgen05) kernel for grouped-query heads: bf16, head_dim 128,
-// groups of 2, 4 or 8, partitions a multiple of 128 tokens.
-bool decode_tc_supported(int dtype, int D, int BS, int G, int partition_tokens);
-cudaError_t launch_decode_tc(const DecodeParams& p, int BS, int G, long long grid, cudaStream_t st);
+// Tensor-core (tcgen05) kernels, head_dim 128, partitions a multiple of 128
+// tokens: bf16 caches with groups of 2, 4 or 8 query heads, fp8 (e4m3)
+// caches with groups of 1, 2, 4 or 8.
+bool decode_tc_supported(int kv_dtype, int D, int BS, int G, int partition_tokens);
+cudaError_t launch_decode_tc(const DecodeParams& p, int kv_dtype, int BS, int G, long long grid,
+                             cudaStream_t st);
+// internal to the tensor-core translation units
+cudaError_t make_tc_pool_map(CUtensorMap* map, const void* pool, int Hkv, int BS, int num_blocks,
+                             int elem_bytes);
+cudaError_t launch_decode_tc_fp8(const DecodeParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
+                                 int BS, int G, long long grid, cudaStream_t st);
 
 }  // namespace pkv

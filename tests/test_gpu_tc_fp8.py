@@ -1,0 +1,119 @@
+"""The tensor-core decode kernel over fp8 (e4m3) caches against the oracle, and
+against the CUDA-core fp8 kernel on the same inputs.
+
+It serves head_dim 128, groups of 1/2/4/8 query heads and partitions that
+are multiples of 128 tokens: QK^T on e4m3 tensor cores with q split into two
+e4m3 terms, PV on f16 tensor cores over V widened in shared memory.  The
+cases span partial 128-token chunks, partial blocks, several partitions
+(fused split-K merge), NaN codes in unused slots, bad table entries, and
+block permutations.
+"""
+import numpy as np
+import pytest
+import torch
+
+from paged_kv_cache_323_b200 import workload as wl
+from steps import assert_close, assert_pool_equal, gpu_step, oracle_step, subset, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture
+def tc_mode():
+    from paged_kv_cache_323_b200 import pagedkv as pk
+
+    prev = pk.set_tensor_core_gqa(True)
+    yield pk
+    pk.set_tensor_core_gqa(prev)
+
+
+@pytest.mark.parametrize("bs", [8, 16, 32])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_tc_fp8_small(tc_mode, bs, G):
+    lens = [1, 5, 127, 128, 129, 300, 640]
+    w = wl.custom(400 + G + bs, lens, heads=2 * G, kv_heads=2, head_dim=128, block_size=bs,
+                  dtype="fp8", maxb=-(-640 // bs) + 1)
+    ref, kref, vref = oracle_step(w)
+    out, kc, vc = gpu_step(w, partition_tokens=256)
+    assert_pool_equal(kc, kref, "k pool (codes)")
+    assert_pool_equal(vc, vref, "v pool (codes)")
+    assert_close(out, ref, "bf16")
+
+
+@pytest.mark.parametrize("pt", [128, 512, 2048, 0])
+def test_tc_fp8_partitions(tc_mode, pt):
+    w = wl.gqa_sampling(groups=4, prompt_median=600, prompt_max=3000, dtype="fp8")
+    ref, _, _ = oracle_step(w)
+    out, _, _ = gpu_step(w, partition_tokens=pt)
+    assert_close(out, ref, "bf16")
+
+
+@pytest.mark.parametrize("G", [1, 4])
+def test_tc_fp8_matches_cuda_core(tc_mode, G):
+    pk = tc_mode
+    w = wl.custom(33 + G, [900, 77, 1500, 256], heads=8 * G, kv_heads=8, head_dim=128,
+                  block_size=16, dtype="fp8")
+    ref, _, _ = oracle_step(w)
+    out_tc, _, _ = gpu_step(w)
+    pk.set_tensor_core_gqa(False)
+    out_cc, _, _ = gpu_step(w)
+    pk.set_tensor_core_gqa(True)
+    assert_close(out_tc, ref, "bf16", "tensor-core kernel")
+    assert_close(out_cc, ref, "bf16", "CUDA-core kernel")
+    d = (out_tc.float() - out_cc.float()).abs().max().item()
+    assert d <= 2e-2, d
+
+
+def test_tc_fp8_nan_codes_and_bad_entry(tc_mode):
+    pk = tc_mode
+    w = wl.custom(78, [200, 333, 50], heads=16, kv_heads=2, head_dim=128, block_size=16,
+                  dtype="fp8", num_blocks=60, maxb=24)
+    bs = w.block_size
+    used = np.zeros((w.num_blocks, bs), dtype=bool)
+    for s in range(w.num_seqs):
+        for t in range(int(w.context_lens[s])):
+            used[w.block_tables[s][t // bs], t % bs] = True
+    mask = torch.from_numpy(~used)[:, None, :, None].expand(w.k_cache.shape)
+    w.k_cache = w.k_cache.view(torch.uint8).masked_fill(mask, 0x7F).view(torch.float8_e4m3fn)
+    w.v_cache = w.v_cache.view(torch.uint8).masked_fill(mask, 0xFF).view(torch.float8_e4m3fn)
+    ref, _, _ = oracle_step(w)
+    out, _, _ = gpu_step(w, partition_tokens=128)
+    assert_close(out, ref, "bf16")
+    # a table entry outside the pool: error word set, output finite
+    w.block_tables[1, 3] = w.num_blocks + 5
+    t = to_device(w)
+    out, _, _ = gpu_step(w, t, partition_tokens=128, check_error=False)
+    assert pk.get_device_error() == pk.PKV_ERR_DEVICE_BOUNDS
+    assert torch.isfinite(out.float()).all()
+
+
+def test_tc_fp8_permutation_bit_identical(tc_mode):
+    w = wl.custom(92, [700, 1000, 257], heads=32, kv_heads=8, head_dim=128, block_size=16,
+                  dtype="fp8")
+    out1, _, _ = gpu_step(w)
+    perm = np.random.default_rng(4).permutation(w.num_blocks)
+    w2 = wl.Workload(**{**w.__dict__})
+    p = torch.from_numpy(perm)
+    w2.k_cache = torch.empty_like(w.k_cache.view(torch.uint8))
+    w2.v_cache = torch.empty_like(w.v_cache.view(torch.uint8))
+    w2.k_cache[p] = w.k_cache.view(torch.uint8)
+    w2.v_cache[p] = w.v_cache.view(torch.uint8)
+    w2.k_cache = w2.k_cache.view(torch.float8_e4m3fn)
+    w2.v_cache = w2.v_cache.view(torch.float8_e4m3fn)
+    w2.block_tables = np.where(w.block_tables >= 0, perm[np.maximum(w.block_tables, 0)], -1).astype(np.int32)
+    bs = w.block_size
+    w2.slot_mapping = np.asarray([perm[s // bs] * bs + s % bs for s in w.slot_mapping], dtype=np.int64)
+    out2, _, _ = gpu_step(w2)
+    assert torch.equal(out1, out2)
+
+
+@pytest.mark.parametrize("make", [
+    lambda: wl.gqa_sampling(device="cuda", dtype="fp8"),
+    lambda: wl.long_context(device="cuda", dtype="fp8"),
+], ids=["gqa_sampling", "long_context"])
+def test_tc_fp8_full_size_sampled(tc_mode, make):
+    w = make()
+    seqs = sorted({0, w.num_seqs // 3, w.num_seqs - 1, int(np.argmax(w.context_lens))})
+    ref, _, _ = oracle_step(subset(w, seqs))
+    out, _, _ = gpu_step(w)
+    assert_close(out[torch.tensor(seqs, device=out.device)], ref, "bf16")
