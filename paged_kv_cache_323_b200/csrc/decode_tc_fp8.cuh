@@ -89,10 +89,21 @@ struct TcFp8Cfg {
     static_assert(SMEM_BYTES <= 113 * 1024, "two CTAs per SM");
 };
 
-// Two e4m3 codes (low byte first) widened exactly to an f16 pair, as 32 bits.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_bits(uint32_t two_codes) {
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two_codes & 0xffffu), __NV_E4M3);
-    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+// Four e4m3 codes (low byte first) widened exactly to two f16 pairs.
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t codes, uint32_t& lo, uint32_t& hi) {
+    asm("{\n\t.reg .b16 c01, c23;\n\t"
+        "mov.b32 {c01, c23}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, c01;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, c23;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(codes));
+}
+
+// Maximum of v over the warp.
+__device__ __forceinline__ float warp_max(float v) {
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+    return r;
 }
 
 template <int BS, int G>
@@ -345,10 +356,11 @@ __global__ void __launch_bounds__(320, 2)
             for (int j = 0; j < 8; ++j) {  // codes 16j .. 16j+15 (swizzled chunk j of the row)
                 uint4 raw = make_uint4(0u, 0u, 0u, 0u);
                 if (valid) raw = *reinterpret_cast<const uint4*>(src + ((j ^ (r & 7)) * 16));
-                const uint4 lo = make_uint4(e4m3x2_to_f16x2_bits(raw.x), e4m3x2_to_f16x2_bits(raw.x >> 16),
-                                            e4m3x2_to_f16x2_bits(raw.y), e4m3x2_to_f16x2_bits(raw.y >> 16));
-                const uint4 hi = make_uint4(e4m3x2_to_f16x2_bits(raw.z), e4m3x2_to_f16x2_bits(raw.z >> 16),
-                                            e4m3x2_to_f16x2_bits(raw.w), e4m3x2_to_f16x2_bits(raw.w >> 16));
+                uint4 lo, hi;
+                e4m3x4_to_f16x4(raw.x, lo.x, lo.y);
+                e4m3x4_to_f16x4(raw.y, lo.z, lo.w);
+                e4m3x4_to_f16x4(raw.z, hi.x, hi.y);
+                e4m3x4_to_f16x4(raw.w, hi.z, hi.w);
                 // f16 dims 16j .. 16j+7 and 16j+8 .. 16j+15: half j / 4, chunks 2(j % 4) and 2(j % 4) + 1
                 unsigned char* half = dst + (j >> 2) * C::HALF16;
                 const int c0 = 2 * (j & 3);
@@ -410,9 +422,7 @@ __global__ void __launch_bounds__(320, 2)
             float* rm = red_max + (c & 1) * 4 * C::NPAD;
 #pragma unroll
             for (int h = 0; h < G; ++h) {
-                float v = x[h];
-#pragma unroll
-                for (int msk = 16; msk; msk >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, msk));
+                const float v = warp_max(x[h]);
                 if (lane == 0) rm[q4 * C::NPAD + h] = v;
             }
             __syncwarp();
