@@ -157,8 +157,12 @@ size_t workspace_bytes_for(long long num_seqs, long long num_heads, long long pa
 int auto_partition_tokens(long long num_seqs, long long num_kv_heads, long long max_ctx, bool tc,
                           bool fp8 = false) {
     if (tc) {
+        // The tensor-core kernels run 2 CTAs per SM, and a CTA's start (table
+        // and q fetch, first TMA round trip) and merge are a fixed cost: keep
+        // partitions as long as the grid still gives 4 waves (batch-8
+        // 128K-token GQA: 543 us at 4096 tokens, 565 us at 2048).
         long long pt = kMaxPartitionTokens;
-        const long long min_ctas = 8LL * 148 * 2;
+        const long long min_ctas = 4LL * 148 * 2;
         while (pt > kMinPartitionTokens && num_seqs * num_kv_heads * ((max_ctx + pt - 1) / pt) < min_ctas)
             pt /= 2;
         return (int)pt;

@@ -11,35 +11,37 @@
 // Why the tensor cores: an e4m3 code costs the CUDA-core kernel a widening
 // (e4m3 -> f16 -> f32) before each FMA, so per byte it issues twice the
 // instructions of a bf16 cache, and with grouped query heads every code feeds
-// G FMAs.  Here the codes are read by the tensor cores:
-//  * QK^T on kind::f8f6f4.  The K tile lands from the pool by TMA (128-byte
-//    swizzle, one 128-byte row of 128 codes per token) and is the A operand
-//    as it is.  q is made e4m3 without losing its bf16 value: each head is
-//    scaled by a power of two so that its largest |q| lies in [128, 256),
-//    then split as q = hi + lo, hi the nearest e4m3 of q and lo the nearest
-//    e4m3 of the remainder.  The remainder of a bf16 value (8 significant
-//    bits) after rounding to 4 has at most 4 significant bits, so the split
-//    is exact for every element whose remainder is above e4m3's subnormal
-//    quantum -- all elements within 2^-9 of the head's largest; smaller ones
-//    err by at most 2^-18 of it.  Column 2h of the S tile is K.hi_h^T, column
-//    2h+1 is K.lo_h^T, and the logit is their sum times the logit scale, the
-//    K scale and the inverse power of two.
-//  * PV on kind::f16.  Four widening warps turn each V tile's codes into f16
-//    (exact) in a shared-memory operand laid out as the bf16 kernel's TMA lays
-//    out a bf16 V tile (128-byte swizzle, tokens as rows), and write zeros for
-//    rows that are not tokens of the partition; P is f16 (11 significant
-//    bits).  The V scale multiplies the partition's output.
+// G FMAs.  Here both products run on kind::f8f6f4 and read the codes as the
+// TMA lands them (128-byte swizzle, one 128-byte row of 128 codes per token):
+//  * S^T = K . Q^T: the K tile is the K-major A operand.  q is made e4m3
+//    without losing its bf16 value: each head is scaled by a power of two so
+//    that its largest |q| lies in [128, 256), then split as q = hi + lo / 16,
+//    hi the nearest e4m3 of q and lo the nearest e4m3 of 16 (q - hi).  A bf16
+//    value has 8 significant bits; after rounding to hi's 4 the remainder has
+//    at most 4, so lo holds it exactly unless it falls below e4m3's subnormal
+//    quantum -- elements under 2^-13 of the head's largest, which then err by
+//    at most 2^-21 of it.  S column 2h is K.hi_h, column 2h+1 is K.lo_h, and
+//    the logit is (S_2h + S_2h+1 / 16) times the logit scale, the K scale and
+//    the inverse power of two.
+//  * O^T = V^T . P^T: the V tile is the A operand read MN-major (dims are
+//    contiguous in a token's row).  The probabilities p in [0, 1] are split
+//    the same way at scale 256: 256 p = hi + lo / 16, so every p keeps 8
+//    significant bits (as a bf16 P would) down to 2^-14, and errs by under
+//    2^-22 below that.  hi and lo go to two accumulators, O_hi and O_lo,
+//    combined as O_hi + O_lo / 16 when the chunk is folded; the running sums
+//    add the same represented values.  V rows that are not tokens of the
+//    partition are zeroed before PV (they may hold NaN codes).
 //
-// One CTA per (sequence, kv head, partition), 320 threads:
+// One CTA per (sequence, kv head, partition), 192 threads:
 //  * warp 0 -- producer: per 128-token chunk, one TMA copy per block of the K
-//    tile, then of the V tile, into a ring of four 16 KB slots (K tiles in
-//    slots 0 and 2, V tiles in 1 and 3); no multicast.
-//  * warp 1 -- TMEM owner (64 columns) and, lane 0, MMA issuer: S^T[128 x 16]
-//    = K_tile . Qs^T (M=128, N=16, K=128 in four K=32 steps), then O^T[128 x
-//    16] = V16^T . P^T (A MN-major, eight K=16 steps).
+//    tile, then of the V tile, into a ring of six 16 KB slots (three chunks
+//    in flight); no multicast.
+//  * warp 1 -- TMEM owner (128 columns) and, lane 0, MMA issuer: QK^T (M=128,
+//    N=16, four K=32 steps) and PV (M=128, N=16, four K=32 steps per term),
+//    each issued as soon as its operands are ready (the issuer polls both,
+//    so neither waits behind the other).
 //  * warps 2-5 -- softmax, as in the bf16 kernel: thread r owns TMEM lane r
 //    (token r of S, dimension r of O); S, P and O are double-buffered.
-//  * warps 6-9 -- V widening: thread r widens row r of each V tile.
 // Every wait is bounded; on timeout the CTA records the error, lets its copies
 // and MMAs land, frees TMEM and returns.
 #pragma once
@@ -55,48 +57,62 @@ struct TcFp8Cfg {
     static constexpr int TILE = 128;          // tokens per chunk
     static constexpr int BPT = TILE / BS;     // blocks per chunk
     static constexpr int NPAD = 16;           // MMA N: 2G columns used by QK, G by PV
-    static constexpr int ROW = 128;           // bytes of a swizzled row (128 codes or 64 f16)
-    static constexpr int SLOT = TILE * ROW;   // one fp8 K or V tile (16 KB)
-    static constexpr int NSLOT = 4;           // K in slots 0, 2; V in 1, 3
-    static constexpr int HALF16 = TILE * ROW; // one 64-dim half of the f16 V operand
-    static constexpr int QB = NPAD * ROW;     // Q operand: 16 rows of 128 codes
-    static constexpr int PB = 2 * NPAD * ROW; // one f16 P operand: 2 token halves x 16 rows
+    static constexpr int ROW = 128;           // bytes of a swizzled row: 128 codes
+    static constexpr int SLOT = TILE * ROW;   // one K or V tile (16 KB)
+    static constexpr int NSLOT = 6;           // K of chunk c at (2c) % 6, V at (2c+1) % 6
+    static constexpr int QB = NPAD * ROW;     // Q operand (hi and lo rows): 16 rows of 128 codes
+    static constexpr int PTERM = NPAD * ROW;  // one P term: 16 head rows of 128 token codes
+    static constexpr int PB = 2 * PTERM;      // one P buffer: the hi and lo terms
     static constexpr int MAX_PART_BLOCKS = 4096 / BS;
-    static constexpr int THREADS = 320;
-    static constexpr uint32_t TMEM_COLS = 64;
+    static constexpr int THREADS = 192;
+    static constexpr uint32_t TMEM_COLS = 128;
     static constexpr uint32_t S_COL = 0;      // two S buffers at columns 0 and 16
-    static constexpr uint32_t O_COL = 32;     // two O buffers at columns 32 and 48
+    static constexpr uint32_t O_COL = 32;     // two O buffers (hi 16 + lo 16 columns) at 32 and 64
     // shared-memory map, offsets from a 1024-byte aligned base
     static constexpr int Q_OFF = NSLOT * SLOT;
-    static constexpr int V16_OFF = Q_OFF + QB;
-    static constexpr int P_OFF = V16_OFF + 2 * HALF16;
+    static constexpr int P_OFF = Q_OFF + QB;
     static constexpr int BAR_OFF = P_OFF + 2 * PB;
-    // full[4] empty[4] s_full[2] s_free[2] p_full[2] o_full[2] o_free[2] red[2]
-    // mma_done v16_full v16_free
-    static constexpr int NBARS = 2 * NSLOT + 15;
+    // full[6] empty[6] s_full[2] s_free[2] p_full[2] o_full[2] o_free[2] red[2] mma_done
+    static constexpr int NBARS = 2 * NSLOT + 13;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;   // tmem address, abort, last flag
     static constexpr int KQ_OFF = MISC_OFF + 16;           // per-head power of two of q
     static constexpr int RED_OFF = KQ_OFF + 8 * 4;         // [2][4][16] chunk maxima, [4][16] sums
     static constexpr int PHYS_OFF = RED_OFF + (2 * 4 * NPAD + 4 * NPAD) * 4;
     static constexpr int SMEM_BYTES = PHYS_OFF + MAX_PART_BLOCKS * 4 + 1024;
-    static constexpr uint32_t IDESC_QK = idesc_make(128, NPAD, 0u, false, false);  // e4m3 x e4m3
-    static constexpr uint32_t IDESC_PV = idesc_make(128, NPAD, 0u, true, false);   // f16 x f16
+    // e4m3 x e4m3: QK with both operands K-major, PV with A (V^T) MN-major
+    static constexpr uint32_t IDESC_QK = idesc_make(128, NPAD, 0u, false, false);
+    static constexpr uint32_t IDESC_PV = idesc_make(128, NPAD, 0u, true, false);
 
     static_assert(TILE % BS == 0 && (BS * ROW) % 1024 == 0, "blocks stack on swizzle atoms");
     static_assert(2 * G <= NPAD && G <= 8, "hi and lo columns of every head fit the MMA N");
-    static_assert(Q_OFF % 1024 == 0 && V16_OFF % 1024 == 0 && P_OFF % 1024 == 0, "operand alignment");
+    static_assert(Q_OFF % 1024 == 0 && P_OFF % 1024 == 0 && PTERM % 1024 == 0, "operand alignment");
     static_assert(merge_scratch_bytes<G, D, THREADS>() <= NSLOT * SLOT, "merge scratch reuses the ring");
     static_assert(SMEM_BYTES <= 113 * 1024, "two CTAs per SM");
 };
 
-// Four e4m3 codes (low byte first) widened exactly to two f16 pairs.
-__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t codes, uint32_t& lo, uint32_t& hi) {
-    asm("{\n\t.reg .b16 c01, c23;\n\t"
-        "mov.b32 {c01, c23}, %2;\n\t"
-        "cvt.rn.f16x2.e4m3x2 %0, c01;\n\t"
-        "cvt.rn.f16x2.e4m3x2 %1, c23;\n\t}"
-        : "=r"(lo), "=r"(hi)
-        : "r"(codes));
+// Two floats to two e4m3 codes (low byte first), round to nearest even,
+// saturating to +-448.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float a, float b) {
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+}
+
+// Two e4m3 codes (low byte first) back to floats, exactly.
+__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint32_t two_codes) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two_codes & 0xffffu), __NV_E4M3);
+    return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
+// Whether the phase of `bar` with the given parity has completed (no wait).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
 }
 
 // Maximum of v over the warp.
@@ -106,8 +122,27 @@ __device__ __forceinline__ float warp_max(float v) {
     return r;
 }
 
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+        "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+        "%30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+          "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+          "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 template <int BS, int G>
-__global__ void __launch_bounds__(320, 2)
+__global__ void __launch_bounds__(192, 2)
     decode_tc_fp8_kernel(const __grid_constant__ DecodeParams p,
                          const __grid_constant__ CUtensorMap tmk,
                          const __grid_constant__ CUtensorMap tmv) {
@@ -132,14 +167,14 @@ __global__ void __launch_bounds__(320, 2)
         }
         return;
     }
-    const int PT = p.partition_tokens;
-    const int nparts = (ctx + PT - 1) / PT;
+    const int PTOK = p.partition_tokens;
+    const int nparts = (ctx + PTOK - 1) / PTOK;
     if (part >= nparts) {
         if (ctx == 0 && part == 0) zero_rows<T, D, G>(p, s, g);
         return;
     }
-    const int tok0 = part * PT;
-    const int tok1 = min(ctx, tok0 + PT);
+    const int tok0 = part * PTOK;
+    const int tok1 = min(ctx, tok0 + PTOK);
     const int nblk = (tok1 - tok0 + BS - 1) / BS;
     const int blk0 = tok0 / BS;
     const int nchunks = (tok1 - tok0 + C::TILE - 1) / C::TILE;
@@ -154,8 +189,6 @@ __global__ void __launch_bounds__(320, 2)
     uint64_t* o_free = o_full + 2;
     uint64_t* red_bar = o_free + 2;
     uint64_t* mma_done = red_bar + 2;
-    uint64_t* v16_full = mma_done + 1;
-    uint64_t* v16_free = v16_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
     int* last_flag = reinterpret_cast<int*>(smem + C::MISC_OFF + 8);
@@ -171,7 +204,7 @@ __global__ void __launch_bounds__(320, 2)
     if (tid == 0) {
         for (int i = 0; i < C::NSLOT; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], (i & 1) ? 4 : 1);  // V slots: the four widening warps
+            mbar_init(&empty[i], 1);  // freed by the MMA that read the slot
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&s_full[b], 1);
@@ -182,8 +215,6 @@ __global__ void __launch_bounds__(320, 2)
             mbar_init(&red_bar[b], 4);
         }
         mbar_init(mma_done, 1);
-        mbar_init(v16_full, 4);
-        mbar_init(v16_free, 1);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -200,9 +231,9 @@ __global__ void __launch_bounds__(320, 2)
         }
         phys[j] = e;
     }
-    if (warp >= 2 && warp < 6) {
-        // Q operand: row n = 2h + term (hi, lo) of query head g*G+h, zero rows
-        // past 2G; thread t writes 16 codes (dims 16j .. 16j+15) of row t / 8.
+    if (warp >= 2) {
+        // Q operand: row n = 2h + term (hi, 16 x lo) of query head g*G+h, zero
+        // rows past 2G; thread t writes 16 codes (dims 16j .. 16j+15) of row t / 8.
         const int t = tid - 64;
         const int n = t >> 3, j = t & 7;
         float qv[16];
@@ -230,14 +261,11 @@ __global__ void __launch_bounds__(320, 2)
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
                 const float a = qv[4 * i + 2 * h2] * up, b = qv[4 * i + 2 * h2 + 1] * up;
-                const __nv_fp8x2_storage_t hc =
-                    __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
-                const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(hc, __NV_E4M3);
-                const float2 hv = __half22float2(*reinterpret_cast<const __half2*>(&hr));
-                const __nv_fp8x2_storage_t lc =
-                    __nv_cvt_float2_to_fp8x2(make_float2(a - hv.x, b - hv.y), __NV_SATFINITE, __NV_E4M3);
-                hw |= (uint32_t)hc << (16 * h2);
-                lw |= (uint32_t)lc << (16 * h2);
+                const uint32_t hc = f32x2_to_e4m3x2(a, b);
+                const float2 hv = e4m3x2_to_f32x2(hc);
+                const uint32_t lc = f32x2_to_e4m3x2((a - hv.x) * 16.f, (b - hv.y) * 16.f);
+                hw |= hc << (16 * h2);
+                lw |= lc << (16 * h2);
             }
             w[i] = (n & 1) ? lw : hw;
         }
@@ -293,85 +321,65 @@ __global__ void __launch_bounds__(320, 2)
         // --------------------------------------------------------- MMA issuer
         if (lane == 0) {
             const uint32_t q_base = smem_addr(smem + C::Q_OFF);
-            const uint32_t v16_base = smem_addr(smem + C::V16_OFF);
-            auto wait_or_abort = [&](uint64_t* bar, uint32_t parity) -> bool {
-                if (mbar_wait_bounded(bar, parity, abort_flag)) return true;
-                set_error(p.err, PKV_ERR_TIMEOUT);
-                *abort_flag = 1;
-                return false;
-            };
-            auto issue_qk = [&](int c) -> bool {
-                const int li = 2 * c, st = li % C::NSLOT;
-                if (!wait_or_abort(&full[st], (li / C::NSLOT) & 1)) return false;
-                if (c >= 2 && !wait_or_abort(&s_free[c & 1], ((c >> 1) - 1) & 1)) return false;
-                tc_fence_after();
-                const uint32_t k_base = smem_addr(smem + st * C::SLOT);
+            int nq = 0, np = 0;  // next chunk for QK^T, for PV
+            unsigned long long t_last = globaltimer_ns();
+            while (np < nchunks) {
+                bool progressed = false;
+                if (nq < nchunks) {
+                    const int li = 2 * nq, st = li % C::NSLOT;
+                    if (mbar_test(&full[st], (li / C::NSLOT) & 1) &&
+                        (nq < 2 || mbar_test(&s_free[nq & 1], ((nq >> 1) - 1) & 1))) {
+                        tc_fence_after();
+                        const uint32_t k_base = smem_addr(smem + st * C::SLOT);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {  // 32 codes (bytes) per step
-                    const uint64_t a = sw128_desc(k_base + kk * 32, 16, 1024);
-                    const uint64_t b = sw128_desc(q_base + kk * 32, 16, 1024);
-                    mma_kind_f8f6f4(tmem + C::S_COL + (c & 1) * 16, a, b, C::IDESC_QK, kk > 0);
+                        for (int kk = 0; kk < 4; ++kk) {  // 32 codes (bytes) per step
+                            const uint64_t a = sw128_desc(k_base + kk * 32, 16, 1024);
+                            const uint64_t b = sw128_desc(q_base + kk * 32, 16, 1024);
+                            mma_kind_f8f6f4(tmem + C::S_COL + (nq & 1) * 16, a, b, C::IDESC_QK, kk > 0);
+                        }
+                        mma_commit(&s_full[nq & 1]);
+                        mma_commit(&empty[st]);
+                        ++nq;
+                        ++mma_issued;
+                        progressed = true;
+                    }
                 }
-                mma_commit(&s_full[c & 1]);
-                mma_commit(&empty[st]);
-                ++mma_issued;
-                return true;
-            };
-            auto issue_pv = [&](int c) -> bool {
-                if (!wait_or_abort(v16_full, c & 1)) return false;
-                if (!wait_or_abort(&p_full[c & 1], (c >> 1) & 1)) return false;
-                if (c >= 2 && !wait_or_abort(&o_free[c & 1], ((c >> 1) - 1) & 1)) return false;
-                tc_fence_after();
-                const uint32_t p_base = smem_addr(smem + C::P_OFF + (c & 1) * C::PB);
+                if (np < nq) {
+                    const int li = 2 * np + 1, st = li % C::NSLOT;
+                    if (mbar_test(&full[st], (li / C::NSLOT) & 1) &&
+                        mbar_test(&p_full[np & 1], (np >> 1) & 1) &&
+                        (np < 2 || mbar_test(&o_free[np & 1], ((np >> 1) - 1) & 1))) {
+                        tc_fence_after();
+                        const uint32_t v_base = smem_addr(smem + st * C::SLOT);
+                        const uint32_t p_base = smem_addr(smem + C::P_OFF + (np & 1) * C::PB);
+                        const uint32_t o_hi = tmem + C::O_COL + (np & 1) * 32;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    // A = V16^T, MN-major: 64-dim halves HALF16 apart, 8-token groups 1024 B apart
-                    const uint64_t a = sw128_desc(v16_base + kk * 16 * C::ROW, C::HALF16, 1024);
-                    const uint64_t b = sw128_desc(p_base + (kk >> 2) * (C::NPAD * C::ROW) + (kk & 3) * 32, 16, 1024);
-                    mma_kind_f16(tmem + C::O_COL + (c & 1) * 16, a, b, C::IDESC_PV, kk > 0);
+                        for (int kk = 0; kk < 4; ++kk) {
+                            // A = V^T, MN-major: the 128 dims of a token are one swizzled
+                            // row; 32 tokens per step, 8-token groups 1024 B apart
+                            const uint64_t a = sw128_desc(v_base + kk * 32 * C::ROW, 16, 1024);
+                            const uint64_t bh = sw128_desc(p_base + kk * 32, 16, 1024);
+                            const uint64_t bl = sw128_desc(p_base + C::PTERM + kk * 32, 16, 1024);
+                            mma_kind_f8f6f4(o_hi, a, bh, C::IDESC_PV, kk > 0);
+                            mma_kind_f8f6f4(o_hi + 16, a, bl, C::IDESC_PV, kk > 0);
+                        }
+                        mma_commit(&o_full[np & 1]);
+                        mma_commit(&empty[st]);
+                        ++np;
+                        ++mma_issued;
+                        progressed = true;
+                    }
                 }
-                mma_commit(&o_full[c & 1]);
-                mma_commit(v16_free);
-                ++mma_issued;
-                return true;
-            };
-            bool ok = issue_qk(0);
-            for (int c = 0; ok && c < nchunks; ++c) {
-                if (c + 1 < nchunks) ok = issue_qk(c + 1);
-                if (ok) ok = issue_pv(c);
-            }
-        }
-    } else if (warp >= 6) {
-        // ------------------------------------------------------- V widening
-        const int r = tid - 192;  // token row of the tile
-        for (int c = 0; c < nchunks; ++c) {
-            const int li = 2 * c + 1, st = li % C::NSLOT;
-            if (!wait_all(&full[st], (li / C::NSLOT) & 1)) break;
-            if (c >= 1 && !wait_all(v16_free, (c - 1) & 1)) break;
-            const int rel = c * C::TILE + r;
-            const bool valid = tok0 + rel < tok1 && phys[rel / BS] >= 0;
-            const unsigned char* src = smem + st * C::SLOT + r * C::ROW;
-            unsigned char* dst = smem + C::V16_OFF + r * C::ROW;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {  // codes 16j .. 16j+15 (swizzled chunk j of the row)
-                uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-                if (valid) raw = *reinterpret_cast<const uint4*>(src + ((j ^ (r & 7)) * 16));
-                uint4 lo, hi;
-                e4m3x4_to_f16x4(raw.x, lo.x, lo.y);
-                e4m3x4_to_f16x4(raw.y, lo.z, lo.w);
-                e4m3x4_to_f16x4(raw.z, hi.x, hi.y);
-                e4m3x4_to_f16x4(raw.w, hi.z, hi.w);
-                // f16 dims 16j .. 16j+7 and 16j+8 .. 16j+15: half j / 4, chunks 2(j % 4) and 2(j % 4) + 1
-                unsigned char* half = dst + (j >> 2) * C::HALF16;
-                const int c0 = 2 * (j & 3);
-                *reinterpret_cast<uint4*>(half + ((c0 ^ (r & 7)) * 16)) = lo;
-                *reinterpret_cast<uint4*>(half + (((c0 + 1) ^ (r & 7)) * 16)) = hi;
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&empty[st]);
-                mbar_arrive(v16_full);
+                if (progressed) {
+                    t_last = globaltimer_ns();
+                } else {
+                    if (*abort_flag) break;
+                    if (globaltimer_ns() - t_last > kWaitTimeoutNs) {
+                        set_error(p.err, PKV_ERR_TIMEOUT);
+                        *abort_flag = 1;
+                        break;
+                    }
+                }
             }
         }
     } else {
@@ -392,13 +400,13 @@ __global__ void __launch_bounds__(320, 2)
         auto fold = [&](int cc, const float* alpha) -> bool {
             if (!wait_all(&o_full[cc & 1], (cc >> 1) & 1)) return false;
             tc_fence_after();
-            float ov[16];
-            tmem_ld16(lane_addr + C::O_COL + (cc & 1) * 16, ov);
+            float ov[32];
+            tmem_ld32(lane_addr + C::O_COL + (cc & 1) * 32, ov);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&o_free[cc & 1]);
 #pragma unroll
-            for (int h = 0; h < G; ++h) acc[h] = fmaf(acc[h], alpha[h], ov[h]);
+            for (int h = 0; h < G; ++h) acc[h] = fmaf(acc[h], alpha[h], fmaf(ov[16 + h], 0.0625f, ov[h]));
             return true;
         };
         bool ok = true;
@@ -418,7 +426,8 @@ __global__ void __launch_bounds__(320, 2)
             const bool valid = tok0 + rel < tok1 && phys[rel / BS] >= 0;
             float x[G];
 #pragma unroll
-            for (int h = 0; h < G; ++h) x[h] = valid ? (sv[2 * h] + sv[2 * h + 1]) * qsk[h] : -INFINITY;
+            for (int h = 0; h < G; ++h)
+                x[h] = valid ? fmaf(sv[2 * h + 1], 0.0625f, sv[2 * h]) * qsk[h] : -INFINITY;
             float* rm = red_max + (c & 1) * 4 * C::NPAD;
 #pragma unroll
             for (int h = 0; h < G; ++h) {
@@ -431,20 +440,49 @@ __global__ void __launch_bounds__(320, 2)
                 ok = false;
                 break;
             }
-            float alpha[G];
-            unsigned char* pbuf = smem + C::P_OFF + (c & 1) * C::PB;
-            const int th = r / 64, tr = r % 64;  // token half and row within it
+            constexpr int GP = G + (G & 1);  // heads rounded up to pairs
+            float alpha[G], pr[GP];
 #pragma unroll
             for (int h = 0; h < G; ++h) {
                 const float mc = fmaxf(fmaxf(rm[h], rm[C::NPAD + h]), fmaxf(rm[2 * C::NPAD + h], rm[3 * C::NPAD + h]));
                 const float m_new = fmaxf(m_run[h], mc);
                 alpha[h] = m_new == -INFINITY ? 1.f : exp2f(m_run[h] - m_new);
                 m_run[h] = m_new;
-                const float pr = valid ? exp2f(x[h] - m_new) : 0.f;
-                const __half ph = __float2half_rn(pr);
-                l_run[h] = fmaf(l_run[h], alpha[h], __half2float(ph));
-                *reinterpret_cast<__half*>(pbuf + th * (C::NPAD * C::ROW) + h * C::ROW +
-                                           ((((tr >> 3) ^ (h & 7)) << 4)) + (tr & 7) * 2) = ph;
+                pr[h] = valid ? exp2f(x[h] - m_new) * 256.f : 0.f;
+            }
+            if constexpr (GP > G) pr[G] = 0.f;
+            // 256 p = hi + lo / 16, both e4m3; P^T rows are heads, K-major over tokens
+            unsigned char* pbuf = smem + C::P_OFF + (c & 1) * C::PB;
+#pragma unroll
+            for (int h = 0; h < GP; h += 2) {
+                const uint32_t hc = f32x2_to_e4m3x2(pr[h], pr[h + 1]);
+                const float2 hv = e4m3x2_to_f32x2(hc);
+                const uint32_t lc = f32x2_to_e4m3x2((pr[h] - hv.x) * 16.f, (pr[h + 1] - hv.y) * 16.f);
+                const float2 lv = e4m3x2_to_f32x2(lc);
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int hh = h + u;
+                    if (hh >= G) break;
+                    const float rep = (u ? fmaf(lv.y, 0.0625f, hv.y) : fmaf(lv.x, 0.0625f, hv.x)) * 0.00390625f;
+                    l_run[hh] = fmaf(l_run[hh], alpha[hh], rep);
+                    const int off = hh * C::ROW + (((r >> 4) ^ (hh & 7)) << 4) + (r & 15);
+                    pbuf[off] = (unsigned char)(hc >> (8 * u));
+                    pbuf[C::PTERM + off] = (unsigned char)(lc >> (8 * u));
+                }
+            }
+            // the V tile must have landed; rows that are not valid tokens get
+            // zero codes (they may hold NaN ones)
+            {
+                const int li = 2 * c + 1, st = li % C::NSLOT;
+                if (!wait_all(&full[st], (li / C::NSLOT) & 1)) {
+                    ok = false;
+                    break;
+                }
+                if (!valid) {
+                    uint4* row = reinterpret_cast<uint4*>(smem + st * C::SLOT + r * C::ROW);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) row[k] = make_uint4(0u, 0u, 0u, 0u);
+                }
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -470,7 +508,8 @@ __global__ void __launch_bounds__(320, 2)
             if (wait_all(&red_bar[nchunks & 1], (nchunks >> 1) & 1)) {
                 const int H = p.num_heads;
                 const long long sh0 = (long long)s * H + (long long)g * G;
-                const float vsc = p.v_scales[g];
+                // O accumulated 256 p; the V scale and 1/256 go on here
+                const float vsc = p.v_scales[g] * 0.00390625f;
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
                     const float L = (red_sum[h] + red_sum[C::NPAD + h]) +
