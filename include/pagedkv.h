@@ -146,8 +146,12 @@ PKV_API int paged_attention_partition_tokens(int num_seqs, int num_heads, int nu
  * pools hold fp8 e4m3 codes; one float scale per kv head (device arrays
  * k_scales, v_scales [num_kv_heads]) gives the stored value code * scale.  q
  * and out are bf16.  Otherwise exactly paged_attention_decode_ex (same
- * workspace, partitions, faults); the kernel is the CUDA-core one, reading
- * half the bytes of a bf16 cache per token.
+ * workspace, partitions, faults).  With head_dim 128 and 1, 2, 4 or 8 query
+ * heads per kv head (and partitions a multiple of 128 tokens) the tensor-core
+ * kernel serves it: both products on e4m3 tensor cores over the codes as
+ * they land, q and the probabilities each split into two e4m3 terms that
+ * keep 8 significant bits; otherwise the CUDA-core kernel, widening each
+ * code.  Either reads half the bytes of a bf16 cache per token.
  */
 PKV_API int paged_attention_decode_fp8(void* out, const void* q, const void* k_cache,
                                        const void* v_cache, const float* k_scales,
@@ -276,11 +280,12 @@ PKV_API int pkv_profile_enable(int on);
 PKV_API int pkv_profile_read(int kind, long long* launches, double* total_ms);
 PKV_API int pkv_profile_reset(void);
 
-/* Choose the decode kernel for grouped-query heads (2, 4 or 8 query heads
- * per kv head, bf16, head_dim 128, partitions a multiple of 128 tokens):
- * 1 (default) runs the tensor-core kernel (tcgen05 MMAs into tensor memory),
- * 0 the CUDA-core kernel that serves every other shape.  Both compute the
- * same attention; returns the previous setting.  Process-wide. */
+/* Choose the decode kernel where a tensor-core one applies (head_dim 128,
+ * partitions a multiple of 128 tokens; bf16 caches with 2, 4 or 8 query heads
+ * per kv head, fp8 caches with 1, 2, 4 or 8): 1 (default) runs the
+ * tensor-core kernel (tcgen05 MMAs into tensor memory), 0 the CUDA-core
+ * kernel that serves every other shape.  Both compute the same attention;
+ * returns the previous setting.  Process-wide. */
 PKV_API int pkv_set_tensor_core_gqa(int enable);
 
 /* Kernels launched by this library in this process so far (all kinds). */

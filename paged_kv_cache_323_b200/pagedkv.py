@@ -429,6 +429,7 @@ def launch_count() -> int:
 
 
 def set_tensor_core_gqa(enable: bool) -> bool:
-    """Select the tensor-core (True) or CUDA-core (False) decode kernel for
-    grouped-query heads; returns the previous setting."""
+    """Select the tensor-core (True) or CUDA-core (False) decode kernels
+    where a tensor-core one applies (bf16 caches with grouped query heads,
+    fp8 caches); returns the previous setting."""
     return bool(lib.pkv_set_tensor_core_gqa(1 if enable else 0))
