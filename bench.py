@@ -112,13 +112,32 @@ def committed_traffic(kernel: str, workload: str, source_sha: str):
         return None
 
 
-def kernel_source_sha() -> str:
+# source files of each decode kernel family (what the DRAM-traffic counters
+# in profiles/ were taken on)
+KERNEL_SOURCES = {
+    "cuda_core": ("common.cuh", "decode_attn.cuh", "decode_launch.cuh"),
+    "tc_bf16": ("common.cuh", "decode_attn.cuh", "decode_tc.cuh", "decode_tc.cu"),
+    "tc_fp8": ("common.cuh", "decode_attn.cuh", "decode_tc.cuh", "decode_tc_fp8.cuh", "decode_tc_fp8.cu"),
+}
+
+
+def decode_kernel_family(w) -> str:
+    """Which decode kernel the library runs for this workload (tensor-core
+    kernels on, as by default)."""
+    group = w.num_heads // w.num_kv_heads
+    if w.head_dim == 128 and w.dtype == "fp8" and group in (1, 2, 4, 8):
+        return "tc_fp8"
+    if w.head_dim == 128 and w.dtype == "bf16" and group in (2, 4, 8):
+        return "tc_bf16"
+    return "cuda_core"
+
+
+def kernel_source_sha(family: str = "cuda_core") -> str:
     import hashlib
 
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_323_b200", "csrc")
-    for name in ("common.cuh", "decode_attn.cuh", "decode_launch.cuh", "decode_tc.cuh",
-                 "decode_tc.cu", "decode_tc_fp8.cuh"):  # the decode kernels' source
+    for name in KERNEL_SOURCES[family]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -544,7 +563,7 @@ def run_gpu(args, world, rank, local):
     roofline = None
     if part:
         achieved = kv_bytes / (part["avg_us"] * 1e-6) / 1e9
-        traffic = committed_traffic("decode", args.workload, kernel_source_sha())
+        traffic = committed_traffic("decode", args.workload, kernel_source_sha(decode_kernel_family(w)))
         roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                     "frac": achieved / peak, "traffic": traffic,
                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
