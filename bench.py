@@ -556,6 +556,7 @@ def run_gpu(args, world, rank, local):
     if rank != 0:
         return
     kv_bytes = w.kv_bytes_logical()
+    kv_unique = w.kv_bytes_unique()
     step_s = ms / args.steps / 1e3
     value = job_value(world, kv_bytes, ms / args.steps)
     peak, peak_src = measured_peak()
@@ -575,6 +576,7 @@ def run_gpu(args, world, rank, local):
         "config": {"workload": name, "num_seqs_per_gpu": w.num_seqs, "num_heads": w.num_heads,
                    "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
                    "block_size": w.block_size, "kv_bytes_per_step_per_gpu": kv_bytes,
+                   "kv_bytes_unique_per_step_per_gpu": kv_unique,
                    "partition_tokens": pk.paged_attention_partition_tokens(
                        w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.block_size,
                        w.max_blocks_per_seq * w.block_size,
@@ -584,6 +586,8 @@ def run_gpu(args, world, rank, local):
                    "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush",
                    "parallelism": f"{world} independent batches, one per GPU"},
         "tokens_per_s": world * w.num_seqs / step_s,
+        # shared blocks counted once (equal to `value` when nothing is shared)
+        "unique_kv_gbs": job_value(world, kv_unique, ms / args.steps),
         "pct_of_peak_hbm": 100.0 * value / peak,
         "per_kernel_us": per_kernel,
         "ms_per_step_profiled": ms_profiled / args.steps,

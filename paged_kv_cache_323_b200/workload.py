@@ -75,6 +75,18 @@ class Workload:
         """K and V bytes one decode step reads, counting every sequence."""
         return int(self.context_lens.astype(np.int64).sum()) * self.num_kv_heads * self.head_dim * 2 * self.elt
 
+    def kv_bytes_unique(self) -> int:
+        """The same over distinct physical blocks: a block shared by several
+        sequences counts once, with the longest prefix any of them uses."""
+        bs = self.block_size
+        used = {}
+        for s in range(self.num_seqs):
+            L = int(self.context_lens[s])
+            for j in range(-(-L // bs)):
+                b = int(self.block_tables[s][j])
+                used[b] = max(used.get(b, 0), min(bs, L - j * bs))
+        return sum(used.values()) * self.num_kv_heads * self.head_dim * 2 * self.elt
+
 
 class _Pool:
     """Free list of physical blocks in a seeded random order, with refcounts."""

@@ -117,3 +117,16 @@ def test_tc_fp8_full_size_sampled(tc_mode, make):
     ref, _, _ = oracle_step(subset(w, seqs))
     out, _, _ = gpu_step(w)
     assert_close(out[torch.tensor(seqs, device=out.device)], ref, "bf16")
+
+
+@pytest.mark.parametrize("pt", [0, 1024])
+def test_tc_fp8_group8_bs32_long_partitions(tc_mode, pt):
+    """Eight query heads per kv head, 32-token blocks, partitions of many
+    128-token chunks (the ring of slots wraps several times) and several
+    partitions per sequence, at a size the oracle checks in full."""
+    w = wl.custom(57, [9000, 4097, 300, 12345], heads=64, kv_heads=8, head_dim=128,
+                  block_size=32, dtype="fp8")
+    ref, kref, vref = oracle_step(w)
+    out, kc, vc = gpu_step(w, partition_tokens=pt)
+    assert_pool_equal(kc, kref, "k pool (codes)")
+    assert_close(out, ref, "bf16")

@@ -131,3 +131,18 @@ def test_contiguous_placement():
         assert w.block_tables[s][:nb].tolist() == list(range(nxt, nxt + nb))
         nxt += nb
     _check_tables(w)
+
+
+def test_kv_bytes_unique_counts_shared_blocks_once():
+    from paged_kv_cache_323_b200 import workload as wl
+
+    w = wl.tiny()
+    assert w.kv_bytes_unique() == w.kv_bytes_logical()  # no sharing
+    # two sequences over one shared full block (16 slots) plus private tails of
+    # 5 and 9 slots; the shared block counts 16 slots once
+    w.block_tables = np.array([[3, 7, -1, -1], [3, 9, -1, -1], [0, -1, -1, -1], [1, 2, 4, 5]],
+                              dtype=np.int32)
+    w.context_lens = np.array([21, 25, 0, 50], dtype=np.int32)
+    per_slot = w.num_kv_heads * w.head_dim * 2 * w.elt
+    assert w.kv_bytes_unique() == (16 + 5 + 9 + 50) * per_slot
+    assert w.kv_bytes_logical() == (21 + 25 + 50) * per_slot
