@@ -2,11 +2,11 @@
 against the CUDA-core fp8 kernel on the same inputs.
 
 It serves head_dim 128, groups of 1/2/4/8 query heads and partitions that
-are multiples of 128 tokens: QK^T on e4m3 tensor cores with q split into two
-e4m3 terms, PV on f16 tensor cores over V widened in shared memory.  The
-cases span partial 128-token chunks, partial blocks, several partitions
-(fused split-K merge), NaN codes in unused slots, bad table entries, and
-block permutations.
+are multiples of 128 tokens: both products on e4m3 tensor cores over the
+codes as they land, q and the probabilities each split into two e4m3 terms.
+The cases span partial 128-token chunks, partial blocks, several partitions
+(fused split-K merge), long partitions that wrap the ring of slots, NaN codes
+in unused slots, bad table entries, and block permutations.
 """
 import numpy as np
 import pytest
