@@ -344,24 +344,23 @@ __global__ void __launch_bounds__(DecodeCfg<T, TKV, D, BS, G>::THREADS,
 
     if (warp == C::NCW) {
         // ------------------------------------------------------ producer
-        // One lane issues every copy: spreading them over the warp measured
-        // slower here (32 lanes polling the ring's barriers take issue slots
-        // from the consumer warps).
-        if (lane == 0) {
-            const char* kbase = static_cast<const char*>(p.k_cache);
-            const char* vbase = static_cast<const char*>(p.v_cache);
-            for (int j = 0; j < nstg; ++j) {
-                const int st = j % C::NST;
-                if (j >= C::NST) {
-                    if (!mbar_wait_bounded(&empty[st], ((j / C::NST) - 1) & 1, abort_flag)) {
-                        set_error(p.err, PKV_ERR_TIMEOUT);
-                        *abort_flag = 1;
-                        break;
+        const char* kbase = static_cast<const char*>(p.k_cache);
+        const char* vbase = static_cast<const char*>(p.v_cache);
+        if constexpr (BS >= C::ST) {
+            // One lane issues every copy (16 rows of one block, the whole
+            // block when bs = 16): spreading two copies over the warp measured
+            // slower here.
+            if (lane == 0) {
+                for (int j = 0; j < nstg; ++j) {
+                    const int st = j % C::NST;
+                    if (j >= C::NST) {
+                        if (!mbar_wait_bounded(&empty[st], ((j / C::NST) - 1) & 1, abort_flag)) {
+                            set_error(p.err, PKV_ERR_TIMEOUT);
+                            *abort_flag = 1;
+                            break;
+                        }
                     }
-                }
-                unsigned char* dst = stages + st * C::STAGE;
-                if constexpr (BS >= C::ST) {
-                    // 16 rows of one block (the whole block when bs = 16)
+                    unsigned char* dst = stages + st * C::STAGE;
                     const int e = phys[j * C::ST / BS];
                     if (e >= 0) {
                         const long long off =
@@ -372,27 +371,41 @@ __global__ void __launch_bounds__(DecodeCfg<T, TKV, D, BS, G>::THREADS,
                     } else {
                         mbar_arrive(&full[st]);  // a skipped block still completes its phase
                     }
-                } else {
-                    // whole blocks stacked row after row
-                    int cnt = 0;
-#pragma unroll
-                    for (int b = 0; b < C::BPS; ++b) {
-                        const int jb = j * C::BPS + b;
-                        cnt += jb < nblk && phys[jb] >= 0;
+                    issued = j + 1;
+                }
+            }
+        } else {
+            // Whole blocks stacked row after row, several per stage: lane 0
+            // waits for the slot and registers the byte count, then lane 2b
+            // copies block b's K slice and lane 2b+1 its V slice, so the
+            // stage's copies issue side by side.
+            for (int j = 0; j < nstg; ++j) {
+                const int st = j % C::NST;
+                bool ready = true;
+                if (lane == 0 && j >= C::NST)
+                    ready = mbar_wait_bounded(&empty[st], ((j / C::NST) - 1) & 1, abort_flag);
+                if (!__shfl_sync(0xffffffffu, ready, 0)) {
+                    if (lane == 0) {
+                        set_error(p.err, PKV_ERR_TIMEOUT);
+                        *abort_flag = 1;
                     }
-                    if (cnt > 0) {
-                        mbar_arrive_expect_tx(&full[st], (uint32_t)(cnt * 2 * C::SLICE));
-#pragma unroll
-                        for (int b = 0; b < C::BPS; ++b) {
-                            const int jb = j * C::BPS + b;
-                            if (jb >= nblk || phys[jb] < 0) continue;
-                            const long long off = ((long long)phys[jb] * Hkv + g) * C::SLICE;
-                            bulk_g2s(dst + b * C::SLICE, kbase + off, C::SLICE, &full[st]);
-                            bulk_g2s(dst + C::STAGE_K + b * C::SLICE, vbase + off, C::SLICE, &full[st]);
-                        }
-                    } else {
+                    break;
+                }
+                const int b = lane >> 1;
+                const int jb = j * C::BPS + b;
+                const int e = (lane < 2 * C::BPS && jb < nblk) ? phys[jb] : -1;
+                const int nload = __popc(__ballot_sync(0xffffffffu, e >= 0));
+                if (lane == 0) {
+                    if (nload > 0)
+                        mbar_arrive_expect_tx(&full[st], (uint32_t)(nload * C::SLICE));
+                    else
                         mbar_arrive(&full[st]);
-                    }
+                }
+                __syncwarp();  // the byte count is registered before any copy lands
+                if (e >= 0) {
+                    const long long off = ((long long)e * Hkv + g) * C::SLICE;
+                    unsigned char* dst = stages + st * C::STAGE + (lane & 1) * C::STAGE_K + b * C::SLICE;
+                    bulk_g2s(dst, ((lane & 1) ? vbase : kbase) + off, C::SLICE, &full[st]);
                 }
                 issued = j + 1;
             }
