@@ -115,9 +115,9 @@ def committed_traffic(kernel: str, workload: str, source_sha: str):
 # source files of each decode kernel family (what the DRAM-traffic counters
 # in profiles/ were taken on)
 KERNEL_SOURCES = {
-    "cuda_core": ("common.cuh", "decode_attn.cuh", "decode_launch.cuh"),
-    "tc_bf16": ("common.cuh", "decode_attn.cuh", "decode_tc.cuh", "decode_tc.cu"),
-    "tc_fp8": ("common.cuh", "decode_attn.cuh", "decode_tc.cuh", "decode_tc_fp8.cuh", "decode_tc_fp8.cu"),
+    "cuda_core": ("common.cuh", "decode_common.cuh", "decode_attn.cuh", "decode_launch.cuh"),
+    "tc_bf16": ("common.cuh", "decode_common.cuh", "decode_tc.cuh", "decode_tc.cu"),
+    "tc_fp8": ("common.cuh", "decode_common.cuh", "decode_tc.cuh", "decode_tc_fp8.cuh", "decode_tc_fp8.cu"),
 }
 
 

@@ -39,7 +39,7 @@
 
 #include <cuda.h>
 
-#include "decode_attn.cuh"
+#include "decode_common.cuh"
 
 namespace pkv {
 namespace tc {

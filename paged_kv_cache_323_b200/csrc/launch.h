@@ -4,7 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include "decode_attn.cuh"
+#include "decode_common.cuh"
 
 namespace pkv {
 
