@@ -1,7 +1,8 @@
 // api.cu -- the C ABI of libpagedkv.so (declared in include/pagedkv.h):
 // argument validation, status codes, launch selection, the library-owned
 // split-K workspace, the per-device error word and the launch profiler.
-// Every compute step runs in the kernels of decode_attn.cuh and kv_ops.cuh.
+// Every compute step runs in the kernels of decode_attn.cuh, decode_tc.cuh,
+// decode_tc_fp8.cuh and kv_ops.cuh.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -149,11 +150,11 @@ size_t workspace_bytes_for(long long num_seqs, long long num_heads, long long pa
 //    of parallelism on batch-64 MHA), doubled (up to 4096) while a sequence
 //    of the maximum length would still be split into more than 64 partitions
 //    and the grid keeps at least four waves of 3 CTAs per SM.
-//  * Tensor-core kernel: 4096 tokens, halved (down to 512) while the grid
-//    would have fewer than eight waves of 2 CTAs per SM.  Its CTAs carry a
+//  * Tensor-core kernels: 4096 tokens, halved (down to 512) while the grid
+//    would have fewer than four waves of 2 CTAs per SM.  Their CTAs carry a
 //    fixed set-up and drain cost, so long partitions pay: on B200 the
-//    parallel-sampling GQA batch ran at 0.55 / 0.75 / 0.88 / 0.97 of peak
-//    with 512 / 1024 / 2048 / 4096-token partitions.
+//    parallel-sampling GQA batch ran at 0.75 / 0.88 / 0.97 of peak with
+//    1024 / 2048 / 4096-token partitions.
 int auto_partition_tokens(long long num_seqs, long long num_kv_heads, long long max_ctx, bool tc,
                           bool fp8 = false) {
     if (tc) {
@@ -496,10 +497,9 @@ int copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_pairs, int 
     p.num_dst_blocks = num_blocks;
     long long per_pair = (p.chunks_per_block + 1023) / 1024;  // 256 threads x 4 chunks
     if (per_pair > 64) per_pair = 64;
-    if (num_pairs > 65535) return PKV_ERR_INVALID;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return launch(PKV_KERNEL_COPY_BLOCKS, st, [&] {
-        pkv::copy_blocks_kernel<<<dim3((unsigned)per_pair, (unsigned)num_pairs), 256, 0, st>>>(p);
+        pkv::copy_blocks_kernel<<<dim3((unsigned)num_pairs, (unsigned)per_pair), 256, 0, st>>>(p);
         return cudaGetLastError();
     });
 }
@@ -511,7 +511,7 @@ int swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
     if (num_pairs == 0) return PKV_OK;
     if (!dst_k || !dst_v || !src_k || !src_v || !src_dst_pairs) return PKV_ERR_NULL;
     if (num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_src_blocks <= 0 ||
-        num_dst_blocks <= 0 || num_pairs > 65535)
+        num_dst_blocks <= 0)
         return PKV_ERR_INVALID;
     if (!known_dtype(dtype)) return PKV_ERR_INVALID;
     const long long block_bytes = (long long)num_kv_heads * block_size * head_dim * elt_bytes(dtype);
@@ -555,7 +555,7 @@ int swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
     if (per_pair > 64) per_pair = 64;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return launch(PKV_KERNEL_SWAP_BLOCKS, st, [&] {
-        pkv::copy_blocks_kernel<<<dim3((unsigned)per_pair, (unsigned)num_pairs), 256, 0, st>>>(p);
+        pkv::copy_blocks_kernel<<<dim3((unsigned)num_pairs, (unsigned)per_pair), 256, 0, st>>>(p);
         return cudaGetLastError();
     });
 }

@@ -158,11 +158,11 @@ struct CopyParams {
 // and destination in the same device pool) and swapping (one side in a
 // pinned host pool, reached through its device-mapped address).
 __global__ void __launch_bounds__(256) copy_blocks_kernel(const CopyParams p) {
-    const int pair = blockIdx.y;
+    const long long pair = blockIdx.x;  // blockIdx.y splits one pair's block
     const long long src = p.pairs[2 * pair];
     const long long dst = p.pairs[2 * pair + 1];
     if (src < 0 || src >= p.num_src_blocks || dst < 0 || dst >= p.num_dst_blocks) {
-        if (blockIdx.x == 0 && threadIdx.x == 0) set_error(p.err, PKV_ERR_DEVICE_BOUNDS);
+        if (blockIdx.y == 0 && threadIdx.x == 0) set_error(p.err, PKV_ERR_DEVICE_BOUNDS);
         return;
     }
     const uint4* ks = static_cast<const uint4*>(p.src_k) + src * p.chunks_per_block;
@@ -170,8 +170,8 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(const CopyParams p) {
     uint4* kd = static_cast<uint4*>(p.dst_k) + dst * p.chunks_per_block;
     uint4* vd = static_cast<uint4*>(p.dst_v) + dst * p.chunks_per_block;
     constexpr int U = 4;
-    const long long stride = (long long)gridDim.x * blockDim.x;
-    for (long long base = blockIdx.x * (long long)blockDim.x + threadIdx.x; base < p.chunks_per_block;
+    const long long stride = (long long)gridDim.y * blockDim.x;
+    for (long long base = blockIdx.y * (long long)blockDim.x + threadIdx.x; base < p.chunks_per_block;
          base += stride * U) {
         uint4 kr[U], vr[U];
 #pragma unroll

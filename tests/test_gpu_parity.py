@@ -10,6 +10,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from paged_kv_cache_323_b200 import workload as wl
 from steps import assert_close, assert_pool_equal, gpu_step, oracle_step, subset, to_device
 
@@ -361,3 +362,23 @@ def test_cuda_graph_capture_and_replay(kind):
     torch.cuda.synchronize()
     assert pk.get_device_error() == 0
     assert torch.equal(t["out"], eager)
+
+
+def test_copy_blocks_more_pairs_than_a_grid_row():
+    """70,000 copy-on-write pairs in one call (beyond 65,535, the largest
+    grid y extent), bit-exact against the oracle."""
+    from paged_kv_cache_323_b200 import pagedkv as pk
+
+    n, nb = 70000, 140010
+    g = torch.Generator().manual_seed(17)
+    kc = torch.randn(nb, 1, 8, 64, generator=g)
+    vc = torch.randn(nb, 1, 8, 64, generator=g)
+    perm = np.random.default_rng(17).permutation(nb)
+    pairs = np.stack([perm[:n], perm[n:2 * n]], 1).astype(np.int64)
+    k_ref, v_ref = kc.numpy().copy(), vc.numpy().copy()
+    oracle.copy_blocks(k_ref, v_ref, pairs)
+    kd, vd = kc.cuda(), vc.cuda()
+    pk.copy_blocks(kd, vd, torch.from_numpy(pairs).cuda())
+    torch.cuda.synchronize()
+    assert pk.get_device_error() == 0
+    assert np.array_equal(kd.cpu().numpy(), k_ref) and np.array_equal(vd.cpu().numpy(), v_ref)
