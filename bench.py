@@ -557,6 +557,9 @@ def run_gpu(args, world, rank, local):
         return
     kv_bytes = w.kv_bytes_logical()
     kv_unique = w.kv_bytes_unique()
+    wst = w.padded_slot_waste()
+    waste = {"per_sequence": wst["per_sequence_unused"] / max(1, wst["per_sequence_allocated"]),
+             "physical": wst["physical_unused"] / max(1, wst["physical_allocated"])}
     step_s = ms / args.steps / 1e3
     value = job_value(world, kv_bytes, ms / args.steps)
     peak, peak_src = measured_peak()
@@ -577,6 +580,7 @@ def run_gpu(args, world, rank, local):
                    "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
                    "block_size": w.block_size, "kv_bytes_per_step_per_gpu": kv_bytes,
                    "kv_bytes_unique_per_step_per_gpu": kv_unique,
+                   "padded_slot_waste": waste,
                    "partition_tokens": pk.paged_attention_partition_tokens(
                        w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.block_size,
                        w.max_blocks_per_seq * w.block_size,

@@ -75,6 +75,24 @@ class Workload:
         """K and V bytes one decode step reads, counting every sequence."""
         return int(self.context_lens.astype(np.int64).sum()) * self.num_kv_heads * self.head_dim * 2 * self.elt
 
+    def padded_slot_waste(self) -> dict:
+        """Slots allocated but holding no token: per sequence (every table
+        counted on its own) and physical (each distinct block once, with the
+        longest prefix any sequence uses)."""
+        bs = self.block_size
+        lens = self.context_lens.astype(np.int64)
+        alloc = int(((lens + bs - 1) // bs * bs).sum())
+        used_slots = {}
+        for s in range(self.num_seqs):
+            L = int(lens[s])
+            for j in range(-(-L // bs)):
+                b = int(self.block_tables[s][j])
+                used_slots[b] = max(used_slots.get(b, 0), min(bs, L - j * bs))
+        phys_alloc = len(used_slots) * bs
+        phys_used = sum(used_slots.values())
+        return {"per_sequence_allocated": alloc, "per_sequence_unused": alloc - int(lens.sum()),
+                "physical_allocated": phys_alloc, "physical_unused": phys_alloc - phys_used}
+
     def kv_bytes_unique(self) -> int:
         """The same over distinct physical blocks: a block shared by several
         sequences counts once, with the longest prefix any of them uses."""

@@ -1,0 +1,50 @@
+"""The committed DRAM-traffic figures (profiles/*.traffic.txt) that bench.py
+folds into its roofline must belong to the kernel sources as they are: each
+file's hash is the current source hash of the kernel family that serves its
+workload.  A kernel change without a new capture fails here."""
+import glob
+import os
+
+import pytest
+
+import bench
+from paged_kv_cache_323_b200 import workload as wl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+# which decode kernel serves each bench workload (by shape and cache type)
+FAMILY = {
+    "mha": "cuda_core", "gqa_sampling": "tc_bf16", "long_context": "tc_bf16",
+    "prefix_bs8": "tc_bf16", "prefix_bs16": "tc_bf16", "prefix_bs32": "tc_bf16",
+    "mha_fp8": "tc_fp8", "gqa_sampling_fp8": "tc_fp8", "long_context_fp8": "tc_fp8",
+}
+
+
+def _read(path):
+    kv = {}
+    for line in open(path):
+        if "=" in line and not line.startswith("#"):
+            k, v = line.split("=", 1)
+            kv[k.strip()] = v.strip()
+    return kv
+
+
+@pytest.mark.parametrize("path", sorted(glob.glob(os.path.join(ROOT, "profiles", "decode_*.traffic.txt"))),
+                         ids=os.path.basename)
+def test_traffic_file_matches_current_kernel_sources(path):
+    workload = os.path.basename(path)[len("decode_"):-len(".traffic.txt")]
+    assert workload in bench.WORKLOADS, workload
+    kv = _read(path)
+    assert kv["kernel_source_sha256"] == bench.kernel_source_sha(FAMILY[workload])
+    assert int(kv["dram_bytes_per_launch"]) > 0
+    assert bench.committed_traffic("decode", workload, bench.kernel_source_sha(FAMILY[workload])) == \
+        float(kv["dram_bytes_per_launch"])
+
+
+@pytest.mark.parametrize("heads,kv_heads,dtype,family", [
+    (32, 32, "bf16", "cuda_core"), (32, 8, "bf16", "tc_bf16"), (64, 8, "bf16", "tc_bf16"),
+    (32, 32, "fp8", "tc_fp8"), (32, 8, "fp8", "tc_fp8"), (8, 8, "f32", "cuda_core"),
+])
+def test_kernel_family_by_shape(heads, kv_heads, dtype, family):
+    w = wl.custom(1, [40, 7], heads=heads, kv_heads=kv_heads, head_dim=128, block_size=16, dtype=dtype)
+    assert bench.decode_kernel_family(w) == family

@@ -146,3 +146,16 @@ def test_kv_bytes_unique_counts_shared_blocks_once():
     per_slot = w.num_kv_heads * w.head_dim * 2 * w.elt
     assert w.kv_bytes_unique() == (16 + 5 + 9 + 50) * per_slot
     assert w.kv_bytes_logical() == (21 + 25 + 50) * per_slot
+
+
+@pytest.mark.parametrize("make", [lambda: wl.tiny(), lambda: wl.gqa_sampling(groups=8, prompt_max=3000),
+                                  lambda: wl.prefix_sweep(8, num_seqs=32, prefix=512)],
+                         ids=["tiny", "gqa_sampling", "prefix_bs8"])
+def test_padded_slot_waste_matches_oracle(make):
+    """The bench's waste figures equal the oracle's waste accounting."""
+    w = make()
+    got = w.padded_slot_waste()
+    alloc, unused = oracle.waste_per_sequence(w.context_lens, w.block_size)
+    assert (got["per_sequence_allocated"], got["per_sequence_unused"]) == (alloc, unused)
+    palloc, punused = oracle.waste_physical(w.block_tables, w.context_lens, w.block_size, w.num_blocks)
+    assert (got["physical_allocated"], got["physical_unused"]) == (palloc, punused)
