@@ -207,17 +207,20 @@ def test_plain_entry_point_matches_ex():
 
 
 # ------------------------------------------------------------ edge cases
-def test_edge_lengths():
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("pt", [64, 128, 0])
+def test_edge_lengths(dtype, pt):
     """Empty context (zero row), one token, exact block multiples, and the
-    maximum context the table can describe."""
+    maximum context the table can describe; partitions of 64 tokens run the
+    CUDA-core kernel, of 128 (and the automatic size) the tensor-core one."""
     bs = 16
     maxb = 12
     lens = [0, 1, bs, 2 * bs, maxb * bs, 5]
-    w = wl.custom(7, lens, heads=8, kv_heads=2, head_dim=128, block_size=bs, dtype="bf16", maxb=maxb)
+    w = wl.custom(7, lens, heads=8, kv_heads=2, head_dim=128, block_size=bs, dtype=dtype, maxb=maxb)
     ref, kref, vref = oracle_step(w)
-    out, kc, vc = gpu_step(w, partition_tokens=64)
+    out, kc, vc = gpu_step(w, partition_tokens=pt)
     assert_pool_equal(kc, kref, "k pool")
-    assert_close(out, ref, w.dtype)
+    assert_close(out, ref, "bf16")
     assert torch.count_nonzero(out[0]) == 0
 
 
