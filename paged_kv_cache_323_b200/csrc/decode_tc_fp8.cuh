@@ -155,9 +155,24 @@ __global__ void __launch_bounds__(192, 2)
     const int P = p.num_partitions;
     const int Hkv = p.num_kv_heads;
     const long long bid = blockIdx.x;
-    const int part = (int)(bid % P);
-    const int g = (int)((bid / P) % Hkv);
-    const int s = (int)(bid / ((long long)P * Hkv));
+    // Launch order.  With a few partitions per sequence (the grid is sized
+    // for the longest, so many CTAs lie past a shorter sequence's end)
+    // partition-major: all first partitions, then all second ones, and so on,
+    // so the CTAs that exit at once come last instead of taking SM slots
+    // between real work.  With many (long contexts) partition-fastest, so that
+    // a unit's partitions finish together and its merge is not left for the
+    // last wave.
+    int part, g, s;
+    if (P <= 4) {
+        const long long units = (long long)p.num_seqs * Hkv;
+        part = (int)(bid / units);
+        g = (int)((bid % units) % Hkv);
+        s = (int)((bid % units) / Hkv);
+    } else {
+        part = (int)(bid % P);
+        g = (int)((bid / P) % Hkv);
+        s = (int)(bid / ((long long)P * Hkv));
+    }
     const int ctx = p.context_lens[s];
     const int max_ctx = p.max_blocks_per_seq * BS;
     if (ctx < 0 || ctx > max_ctx) {
