@@ -34,8 +34,11 @@
 //
 // One CTA per (sequence, kv head, partition), 192 threads:
 //  * warp 0 -- producer: per 128-token chunk, one TMA copy per block of the K
-//    tile, then of the V tile, into a ring of six 16 KB slots (three chunks
-//    in flight); no multicast.
+//    tile, then of the V tile, into a ring of 16 KB slots; no multicast.
+//    Up to 4 query heads per kv head: three slots, which K and V tiles take
+//    in turn, so that three CTAs share an SM and their per-chunk chains
+//    overlap.  8 query heads need more registers (two CTAs per SM): six
+//    slots, K tiles in the even ones and V tiles in the odd ones.
 //  * warp 1 -- TMEM owner (128 columns) and, lane 0, MMA issuer: QK^T (M=128,
 //    N=16, four K=32 steps) and PV (M=128, N=16, four K=32 steps per term),
 //    each issued as soon as its operands are ready (the issuer polls both,
@@ -59,7 +62,9 @@ struct TcFp8Cfg {
     static constexpr int NPAD = 16;           // MMA N: 2G columns used by QK, G by PV
     static constexpr int ROW = 128;           // bytes of a swizzled row: 128 codes
     static constexpr int SLOT = TILE * ROW;   // one K or V tile (16 KB)
-    static constexpr int NSLOT = 6;           // K of chunk c at (2c) % 6, V at (2c+1) % 6
+    static constexpr int CTAS_PER_SM = G >= 8 ? 2 : 3;
+    static constexpr int NSLOT = CTAS_PER_SM == 2 ? 6 : 3;
+    // tile li (K of chunk li/2 when even, V when odd) sits in slot li % NSLOT
     static constexpr int QB = NPAD * ROW;     // Q operand (hi and lo rows): 16 rows of 128 codes
     static constexpr int PTERM = NPAD * ROW;  // one P term: 16 head rows of 128 token codes
     static constexpr int PB = 2 * PTERM;      // one P buffer: the hi and lo terms
@@ -72,7 +77,7 @@ struct TcFp8Cfg {
     static constexpr int Q_OFF = NSLOT * SLOT;
     static constexpr int P_OFF = Q_OFF + QB;
     static constexpr int BAR_OFF = P_OFF + 2 * PB;
-    // full[6] empty[6] s_full[2] s_free[2] p_full[2] o_full[2] o_free[2] red[2] mma_done
+    // full[NSLOT] empty[NSLOT] s_full[2] s_free[2] p_full[2] o_full[2] o_free[2] red[2] mma_done
     static constexpr int NBARS = 2 * NSLOT + 13;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;   // tmem address, abort, last flag
     static constexpr int KQ_OFF = MISC_OFF + 16;           // per-head power of two of q
@@ -87,7 +92,8 @@ struct TcFp8Cfg {
     static_assert(2 * G <= NPAD && G <= 8, "hi and lo columns of every head fit the MMA N");
     static_assert(Q_OFF % 1024 == 0 && P_OFF % 1024 == 0 && PTERM % 1024 == 0, "operand alignment");
     static_assert(merge_scratch_bytes<G, D, THREADS>() <= NSLOT * SLOT, "merge scratch reuses the ring");
-    static_assert(SMEM_BYTES <= 113 * 1024, "two CTAs per SM");
+    static_assert(CTAS_PER_SM * (SMEM_BYTES + 1024) <= 228 * 1024, "CTAs per SM by shared memory");
+    static_assert(CTAS_PER_SM * TMEM_COLS <= 512, "CTAs per SM by TMEM");
 };
 
 // Two floats to two e4m3 codes (low byte first), round to nearest even,
@@ -142,7 +148,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 }
 
 template <int BS, int G>
-__global__ void __launch_bounds__(192, 2)
+__global__ void __launch_bounds__(192, TcFp8Cfg<BS, G>::CTAS_PER_SM)
     decode_tc_fp8_kernel(const __grid_constant__ DecodeParams p,
                          const __grid_constant__ CUtensorMap tmk,
                          const __grid_constant__ CUtensorMap tmv) {
@@ -340,7 +346,12 @@ __global__ void __launch_bounds__(192, 2)
             unsigned long long t_last = globaltimer_ns();
             while (np < nchunks) {
                 bool progressed = false;
-                if (nq < nchunks) {
+                // With an odd ring, K of chunk nq takes the slot that V of chunk
+                // nq-2 held.  Until PV of chunk nq-2 has been issued (after the
+                // wait for that tile) the slot's barrier may still be one phase
+                // short, where the parity test of K(nq)'s phase passes as well:
+                // QK runs at most one chunk ahead of PV there.
+                if (nq < nchunks && (C::NSLOT % 2 == 0 || nq <= np + 1)) {
                     const int li = 2 * nq, st = li % C::NSLOT;
                     if (mbar_test(&full[st], (li / C::NSLOT) & 1) &&
                         (nq < 2 || mbar_test(&s_free[nq & 1], ((nq >> 1) - 1) & 1))) {
