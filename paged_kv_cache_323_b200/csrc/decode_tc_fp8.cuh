@@ -34,11 +34,11 @@
 //
 // One CTA per (sequence, kv head, partition), 192 threads:
 //  * warp 0 -- producer: per 128-token chunk, one TMA copy per block of the K
-//    tile, then of the V tile, into a ring of 16 KB slots; no multicast.
-//    Up to 4 query heads per kv head: three slots, which K and V tiles take
-//    in turn, so that three CTAs share an SM and their per-chunk chains
-//    overlap.  8 query heads need more registers (two CTAs per SM): six
-//    slots, K tiles in the even ones and V tiles in the odd ones.
+//    tile, then of the V tile, into a ring of 16 KB slots, K tiles in the
+//    even slots and V tiles in the odd ones; no multicast.  Up to 4 query
+//    heads per kv head: two slots, so that four CTAs share an SM and their
+//    per-chunk chains overlap.  8 query heads need more registers (two CTAs
+//    per SM): six slots.
 //  * warp 1 -- TMEM owner (128 columns) and, lane 0, MMA issuer: QK^T (M=128,
 //    N=16, four K=32 steps) and PV (M=128, N=16, four K=32 steps per term),
 //    each issued as soon as its operands are ready (the issuer polls both,
@@ -62,8 +62,8 @@ struct TcFp8Cfg {
     static constexpr int NPAD = 16;           // MMA N: 2G columns used by QK, G by PV
     static constexpr int ROW = 128;           // bytes of a swizzled row: 128 codes
     static constexpr int SLOT = TILE * ROW;   // one K or V tile (16 KB)
-    static constexpr int CTAS_PER_SM = G >= 8 ? 2 : 3;
-    static constexpr int NSLOT = CTAS_PER_SM == 2 ? 6 : 3;
+    static constexpr int CTAS_PER_SM = G >= 8 ? 2 : 4;
+    static constexpr int NSLOT = CTAS_PER_SM == 2 ? 6 : 2;
     // tile li (K of chunk li/2 when even, V when odd) sits in slot li % NSLOT
     static constexpr int QB = NPAD * ROW;     // Q operand (hi and lo rows): 16 rows of 128 codes
     static constexpr int PTERM = NPAD * ROW;  // one P term: 16 head rows of 128 token codes
@@ -80,7 +80,7 @@ struct TcFp8Cfg {
     // full[NSLOT] empty[NSLOT] s_full[2] s_free[2] p_full[2] o_full[2] o_free[2] red[2] mma_done
     static constexpr int NBARS = 2 * NSLOT + 13;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;   // tmem address, abort, last flag
-    static constexpr int KQ_OFF = MISC_OFF + 16;           // per-head power of two of q
+    static constexpr int KQ_OFF = MISC_OFF + 16;           // per-head logit factor (float)
     static constexpr int RED_OFF = KQ_OFF + 8 * 4;         // [2][4][16] chunk maxima, [4][16] sums
     static constexpr int PHYS_OFF = RED_OFF + (2 * 4 * NPAD + 4 * NPAD) * 4;
     static constexpr int SMEM_BYTES = PHYS_OFF + MAX_PART_BLOCKS * 4 + 1024;
@@ -94,6 +94,12 @@ struct TcFp8Cfg {
     static_assert(merge_scratch_bytes<G, D, THREADS>() <= NSLOT * SLOT, "merge scratch reuses the ring");
     static_assert(CTAS_PER_SM * (SMEM_BYTES + 1024) <= 228 * 1024, "CTAs per SM by shared memory");
     static_assert(CTAS_PER_SM * TMEM_COLS <= 512, "CTAs per SM by TMEM");
+    // An even ring keeps K tiles and V tiles in slots of their own, so a
+    // tile's slot was last used by the same product's previous tile, whose
+    // wait came first.  With an odd ring, K of chunk c would take the slot
+    // V of chunk c-2 held, and the issuer's parity test could not tell that
+    // barrier's awaited phase from the phase before it.
+    static_assert(NSLOT % 2 == 0, "K and V tiles in slots of their own");
 };
 
 // Two floats to two e4m3 codes (low byte first), round to nearest even,
@@ -128,23 +134,91 @@ __device__ __forceinline__ float warp_max(float v) {
     return r;
 }
 
-// 32 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
-        "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
-        "%30, %31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
-          "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
-          "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr)
-        : "memory");
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+// Columns [0, N) and [16, 16 + N) of this thread's TMEM lane from taddr, with
+// one wait for both loads (N = 1, 2, 4 or 8): the hi and lo accumulators of
+// the first N heads.
+template <int N>
+__device__ __forceinline__ void tmem_ld_hi_lo(uint32_t taddr, float (&hi)[N], float (&lo)[N]) {
+    static_assert(N == 1 || N == 2 || N == 4 || N == 8, "load shape");
+    uint32_t r[2 * N];
+    if constexpr (N == 1) {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%2];\n\t"
+            "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%1}, [%3];\n\t"
+            "tcgen05.wait::ld.sync.aligned;"
+            : "=r"(r[0]), "=r"(r[1])
+            : "r"(taddr), "r"(taddr + 16u)
+            : "memory");
+    } else if constexpr (N == 2) {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%4];\n\t"
+            "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%2, %3}, [%5];\n\t"
+            "tcgen05.wait::ld.sync.aligned;"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+            : "r"(taddr), "r"(taddr + 16u)
+            : "memory");
+    } else if constexpr (N == 4) {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%8];\n\t"
+            "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%4, %5, %6, %7}, [%9];\n\t"
+            "tcgen05.wait::ld.sync.aligned;"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+              "=r"(r[7])
+            : "r"(taddr), "r"(taddr + 16u)
+            : "memory");
+    } else if constexpr (N == 8) {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%16];\n\t"
+            "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%8, %9, %10, %11, %12, %13, %14, %15}, [%17];\n\t"
+            "tcgen05.wait::ld.sync.aligned;"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+              "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+              "=r"(r[14]), "=r"(r[15])
+            : "r"(taddr), "r"(taddr + 16u)
+            : "memory");
+    }
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+    for (int i = 0; i < N; ++i) {
+        hi[i] = __uint_as_float(r[i]);
+        lo[i] = __uint_as_float(r[N + i]);
+    }
+}
+
+// The first N columns of this thread's TMEM lane from taddr, waited for
+// (N = 2, 4, 8 or 16).
+template <int N>
+__device__ __forceinline__ void tmem_ld_first(uint32_t taddr, float (&v)[N]) {
+    static_assert(N == 2 || N == 4 || N == 8 || N == 16, "load shape");
+    if constexpr (N == 16) {
+        tmem_ld16(taddr, v);
+    } else {
+        uint32_t r[N];
+        if constexpr (N == 2) {
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];\n\t"
+                "tcgen05.wait::ld.sync.aligned;"
+                : "=r"(r[0]), "=r"(r[1])
+                : "r"(taddr)
+                : "memory");
+        } else if constexpr (N == 4) {
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];\n\t"
+                "tcgen05.wait::ld.sync.aligned;"
+                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                : "r"(taddr)
+                : "memory");
+        } else if constexpr (N == 8) {
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
+                "tcgen05.wait::ld.sync.aligned;"
+                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                  "=r"(r[6]), "=r"(r[7])
+                : "r"(taddr)
+                : "memory");
+        }
+#pragma unroll
+        for (int i = 0; i < N; ++i) v[i] = __uint_as_float(r[i]);
+    }
 }
 
 template <int BS, int G>
@@ -213,7 +287,7 @@ __global__ void __launch_bounds__(192, TcFp8Cfg<BS, G>::CTAS_PER_SM)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
     int* last_flag = reinterpret_cast<int*>(smem + C::MISC_OFF + 8);
-    int* kq = reinterpret_cast<int*>(smem + C::KQ_OFF);
+    float* qsk = reinterpret_cast<float*>(smem + C::KQ_OFF);  // [G]
     float* red_max = reinterpret_cast<float*>(smem + C::RED_OFF);  // [2][4][16]
     float* red_sum = red_max + 2 * 4 * C::NPAD;                   // [4][16]
     int* phys = reinterpret_cast<int*>(smem + C::PHYS_OFF);
@@ -294,7 +368,9 @@ __global__ void __launch_bounds__(192, TcFp8Cfg<BS, G>::CTAS_PER_SM)
         if (n >= 2 * G) val = make_uint4(0u, 0u, 0u, 0u);
         if (!(mx <= 3.402823466e38f)) val = make_uint4(0x7f7f7f7fu, 0x7f7f7f7fu, 0x7f7f7f7fu, 0x7f7f7f7fu);  // inf / NaN in q: NaN codes
         *reinterpret_cast<uint4*>(smem + C::Q_OFF + n * C::ROW + ((j ^ (n & 7)) * 16)) = val;
-        if (n < 2 * G && (n & 1) == 0 && j == 0) kq[n >> 1] = kexp;
+        // the logit of head n/2 is its S columns' sum times scale, k_scale and 2^-k
+        if (n < 2 * G && (n & 1) == 0 && j == 0)
+            qsk[n >> 1] = p.qscale * p.k_scales[g] * __uint_as_float((uint32_t)(127 - kexp) << 23);
         for (int u = t; u < 2 * C::PB / 16; u += 128)
             reinterpret_cast<uint4*>(smem + C::P_OFF)[u] = make_uint4(0u, 0u, 0u, 0u);
         fence_proxy_async_smem();
@@ -346,12 +422,7 @@ __global__ void __launch_bounds__(192, TcFp8Cfg<BS, G>::CTAS_PER_SM)
             unsigned long long t_last = globaltimer_ns();
             while (np < nchunks) {
                 bool progressed = false;
-                // With an odd ring, K of chunk nq takes the slot that V of chunk
-                // nq-2 held.  Until PV of chunk nq-2 has been issued (after the
-                // wait for that tile) the slot's barrier may still be one phase
-                // short, where the parity test of K(nq)'s phase passes as well:
-                // QK runs at most one chunk ahead of PV there.
-                if (nq < nchunks && (C::NSLOT % 2 == 0 || nq <= np + 1)) {
+                if (nq < nchunks) {
                     const int li = 2 * nq, st = li % C::NSLOT;
                     if (mbar_test(&full[st], (li / C::NSLOT) & 1) &&
                         (nq < 2 || mbar_test(&s_free[nq & 1], ((nq >> 1) - 1) & 1))) {
@@ -413,26 +484,24 @@ __global__ void __launch_bounds__(192, TcFp8Cfg<BS, G>::CTAS_PER_SM)
         const int q4 = warp & 3;            // TMEM lane quadrant of this warp
         const int r = q4 * 32 + lane;       // token row of S, dimension row of O
         const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
-        float m_run[G], l_run[G], acc[G], alpha_prev[G], qsk[G];
-        const float kscale = p.qscale * p.k_scales[g];
+        float m_run[G], l_run[G], acc[G], alpha_prev[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) {
             m_run[h] = -INFINITY;
             l_run[h] = 0.f;
             acc[h] = 0.f;
             alpha_prev[h] = 1.f;
-            qsk[h] = kscale * __uint_as_float((uint32_t)(127 - kq[h]) << 23);
         }
         auto fold = [&](int cc, const float* alpha) -> bool {
             if (!wait_all(&o_full[cc & 1], (cc >> 1) & 1)) return false;
             tc_fence_after();
-            float ov[32];
-            tmem_ld32(lane_addr + C::O_COL + (cc & 1) * 32, ov);
+            float oh[G], ol[G];
+            tmem_ld_hi_lo<G>(lane_addr + C::O_COL + (cc & 1) * 32, oh, ol);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&o_free[cc & 1]);
 #pragma unroll
-            for (int h = 0; h < G; ++h) acc[h] = fmaf(acc[h], alpha[h], fmaf(ov[16 + h], 0.0625f, ov[h]));
+            for (int h = 0; h < G; ++h) acc[h] = fmaf(acc[h], alpha[h], fmaf(ol[h], 0.0625f, oh[h]));
             return true;
         };
         bool ok = true;
@@ -442,8 +511,8 @@ __global__ void __launch_bounds__(192, TcFp8Cfg<BS, G>::CTAS_PER_SM)
                 break;
             }
             tc_fence_after();
-            float sv[16];
-            tmem_ld16(lane_addr + C::S_COL + (c & 1) * 16, sv);
+            float sv[2 * G];
+            tmem_ld_first<2 * G>(lane_addr + C::S_COL + (c & 1) * 16, sv);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_free[c & 1]);
