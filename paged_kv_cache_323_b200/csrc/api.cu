@@ -151,17 +151,19 @@ size_t workspace_bytes_for(long long num_seqs, long long num_heads, long long pa
 //    of the maximum length would still be split into more than 64 partitions
 //    and the grid keeps at least four waves of 3 CTAs per SM.
 //  * Tensor-core kernels: 4096 tokens, halved (down to 512) while the grid
-//    would have fewer than four waves of 2 CTAs per SM.  Their CTAs carry a
+//    would have fewer than 4 × 148 × 2 CTAs.  Their CTAs carry a
 //    fixed set-up and drain cost, so long partitions pay: on B200 the
 //    parallel-sampling GQA batch ran at 0.75 / 0.88 / 0.97 of peak with
 //    1024 / 2048 / 4096-token partitions.
 int auto_partition_tokens(long long num_seqs, long long num_kv_heads, long long max_ctx, bool tc,
                           bool fp8 = false) {
     if (tc) {
-        // The tensor-core kernels run 2 CTAs per SM, and a CTA's start (table
-        // and q fetch, first TMA round trip) and merge are a fixed cost: keep
-        // partitions as long as the grid still gives 4 waves (batch-8
-        // 128K-token GQA: 543 us at 4096 tokens, 565 us at 2048).
+        // The tensor-core kernels run 2 to 4 CTAs per SM, and a CTA's start
+        // (table and q fetch, first TMA round trip) and merge are a fixed
+        // cost: keep partitions as long as the grid still gives 4 waves of 2
+        // CTAs per SM (batch-8 128K-token GQA: 543 us at 4096 tokens, 565 us
+        // at 2048; the fp8 parallel-sampling batch at 4 CTAs per SM: 153 /
+        // 171 / 209 us at 4096 / 2048 / 1024).
         long long pt = kMaxPartitionTokens;
         const long long min_ctas = 4LL * 148 * 2;
         while (pt > kMinPartitionTokens && num_seqs * num_kv_heads * ((max_ctx + pt - 1) / pt) < min_ctas)
