@@ -212,7 +212,9 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(mhz)}
 
 
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, cuda: bool = True):
+    """One process per GPU under torchrun (NCCL); `cuda` False (the oracle arm
+    on a host without a GPU) joins the ranks over gloo instead."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -221,10 +223,13 @@ def dist_setup(n_gpus: int):
 
         import torch.distributed as dist
 
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
+        if cuda:
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+    elif cuda:
         torch.cuda.set_device(0)
     return world, rank, local
 
@@ -372,7 +377,9 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     name, make = WORKLOADS[args.workload]
-    w = make("cuda", DEFAULT_SEED[args.workload])
+    # the generator runs on the GPU where there is one (faster for the large
+    # pools); the timed work is the oracle on host cores either way
+    w = make("cuda" if torch.cuda.is_available() else "cpu", DEFAULT_SEED[args.workload])
     threads = cpu_threads()
     sub, n, _ = pick_sample(w, target_s=8.0 / max(1, args.steps), threads=threads)
     for _ in range(min(args.warmup, 1)):
@@ -640,7 +647,7 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    world, rank, local = dist_setup(args.gpus)
+    world, rank, local = dist_setup(args.gpus, cuda=args.impl != "reference" or torch.cuda.is_available())
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
