@@ -102,12 +102,24 @@ def _check(rc: int, where: str) -> None:
         raise PagedKVError(rc, where)
 
 
-def _stream(stream) -> int:
+def _stream(stream, device=None) -> int:
+    """cudaStream_t of `stream` (None: the current stream of `device`)."""
     if stream is None:
-        return torch.cuda.current_stream().cuda_stream
+        return torch.cuda.current_stream(device).cuda_stream
     if isinstance(stream, torch.cuda.Stream):
+        if device is not None and stream.device != device:
+            raise ValueError(f"stream is on {stream.device}, the tensors on {device}")
         return stream.cuda_stream
     return int(stream)
+
+
+def _device(*tensors) -> torch.device:
+    """The device of the first CUDA tensor given (else the current device):
+    the call runs there, and every other device tensor must be on it."""
+    for t in tensors:
+        if t is not None and t.is_cuda:
+            return t.device
+    return torch.device("cuda", torch.cuda.current_device())
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -120,14 +132,29 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
-def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
+def _dev(t: torch.Tensor, name: str, dtype=None, *, device=None, shape=None) -> int:
+    """Device pointer of a contiguous CUDA tensor, after checking its device,
+    element type and shape where given."""
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the other tensors on {device}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
     return t.data_ptr()
+
+
+def _tables(block_tables, context_lens, B: int) -> int:
+    """max_blocks_per_seq of a [B][max_blocks] table; context_lens must be [B]."""
+    if block_tables.dim() != 2 or block_tables.shape[0] != B:
+        raise ValueError(f"block_tables must be [{B}][max_blocks_per_seq], got {tuple(block_tables.shape)}")
+    if tuple(context_lens.shape) != (B,):
+        raise ValueError(f"context_lens must be [{B}], got {tuple(context_lens.shape)}")
+    return block_tables.shape[1]
 
 
 def paged_attention_workspace_size(num_seqs: int, num_heads: int, max_context: int, head_dim: int,
@@ -155,20 +182,24 @@ def paged_attention_decode_ex(out, q, k_cache, v_cache, block_tables, context_le
     N, Hkv, bs, D2 = k_cache.shape
     if D2 != D or tuple(out.shape) != (B, H, D) or tuple(v_cache.shape) != tuple(k_cache.shape):
         raise ValueError("shape mismatch between q, out and the caches")
-    maxb = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    maxb = _tables(block_tables, context_lens, B)
     if num_blocks is None:
         num_blocks = N
+    dev = _device(q)
+    code = _dtype_code(q)
+    args = (_dev(out, "out", q.dtype, device=dev), _dev(q, "q", device=dev),
+            _dev(k_cache, "k_cache", q.dtype, device=dev), _dev(v_cache, "v_cache", q.dtype, device=dev),
+            _dev(block_tables, "block_tables", torch.int32, device=dev),
+            _dev(context_lens, "context_lens", torch.int32, device=dev))
     need = paged_attention_workspace_size(B, H, maxb * bs, D, partition_tokens)
     if workspace is None and need > 0:
-        workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
-    ws_ptr = workspace.data_ptr() if workspace is not None else None
-    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    code = _dtype_code(q)
-    rc = lib.paged_attention_decode_ex(
-        _dev(out, "out", q.dtype), _dev(q, "q"), _dev(k_cache, "k_cache", q.dtype),
-        _dev(v_cache, "v_cache", q.dtype), _dev(block_tables, "block_tables", torch.int32),
-        _dev(context_lens, "context_lens", torch.int32), B, H, Hkv, D, bs, maxb, float(scale),
-        int(num_blocks), code, int(partition_tokens), ws_ptr, ws_bytes, _stream(stream))
+        workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
+    ws_ptr = _dev(workspace, "workspace", torch.uint8, device=dev) if workspace is not None else None
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    with torch.cuda.device(dev):
+        rc = lib.paged_attention_decode_ex(*args, B, H, Hkv, D, bs, maxb, float(scale),
+                                           int(num_blocks), code, int(partition_tokens), ws_ptr,
+                                           ws_bytes, _stream(stream, dev))
     _check(rc, "paged_attention_decode_ex")
 
 
@@ -182,19 +213,25 @@ def paged_attention_decode_fp8(out, q, k_cache, v_cache, k_scales, v_scales, blo
     N, Hkv, bs, D2 = k_cache.shape
     if D2 != D or tuple(out.shape) != (B, H, D) or tuple(v_cache.shape) != tuple(k_cache.shape):
         raise ValueError("shape mismatch between q, out and the caches")
-    maxb = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    maxb = _tables(block_tables, context_lens, B)
+    dev = _device(q)
+    args = (_dev(out, "out", torch.bfloat16, device=dev), _dev(q, "q", torch.bfloat16, device=dev),
+            _dev(k_cache, "k_cache", torch.float8_e4m3fn, device=dev),
+            _dev(v_cache, "v_cache", torch.float8_e4m3fn, device=dev),
+            _dev(k_scales, "k_scales", torch.float32, device=dev, shape=(Hkv,)),
+            _dev(v_scales, "v_scales", torch.float32, device=dev, shape=(Hkv,)),
+            _dev(block_tables, "block_tables", torch.int32, device=dev),
+            _dev(context_lens, "context_lens", torch.int32, device=dev))
     need = paged_attention_workspace_size(B, H, maxb * bs, D, partition_tokens)
     if workspace is None and need > 0:
-        workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
-    rc = lib.paged_attention_decode_fp8(
-        _dev(out, "out", torch.bfloat16), _dev(q, "q", torch.bfloat16),
-        _dev(k_cache, "k_cache", torch.float8_e4m3fn), _dev(v_cache, "v_cache", torch.float8_e4m3fn),
-        _dev(k_scales, "k_scales", torch.float32), _dev(v_scales, "v_scales", torch.float32),
-        _dev(block_tables, "block_tables", torch.int32),
-        _dev(context_lens, "context_lens", torch.int32), B, H, Hkv, D, bs, maxb, float(scale),
-        N if num_blocks is None else int(num_blocks), int(partition_tokens),
-        workspace.data_ptr() if workspace is not None else None,
-        workspace.numel() if workspace is not None else 0, _stream(stream))
+        workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
+    ws_ptr = _dev(workspace, "workspace", torch.uint8, device=dev) if workspace is not None else None
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    with torch.cuda.device(dev):
+        rc = lib.paged_attention_decode_fp8(*args, B, H, Hkv, D, bs, maxb, float(scale),
+                                            N if num_blocks is None else int(num_blocks),
+                                            int(partition_tokens), ws_ptr, ws_bytes,
+                                            _stream(stream, dev))
     _check(rc, "paged_attention_decode_fp8")
 
 
@@ -202,12 +239,20 @@ def kv_cache_append_fp8(k_cache, v_cache, k_scales, v_scales, k, v, slot_mapping
     """Quantise bf16 rows k, v [T][Hkv][D] into the fp8 pools."""
     T = slot_mapping.shape[0]
     N, Hkv, bs, D = k_cache.shape
-    rc = lib.kv_cache_append_fp8(
-        _dev(k_cache, "k_cache", torch.float8_e4m3fn), _dev(v_cache, "v_cache", torch.float8_e4m3fn),
-        _dev(k_scales, "k_scales", torch.float32), _dev(v_scales, "v_scales", torch.float32),
-        _dev(k, "k", torch.bfloat16) if T else None, _dev(v, "v", torch.bfloat16) if T else None,
-        _dev(slot_mapping, "slot_mapping", torch.int64) if T else None, T, Hkv, D, bs, N,
-        _stream(stream))
+    if tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("k_cache and v_cache must have the same shape")
+    if T and (tuple(k.shape) != (T, Hkv, D) or tuple(v.shape) != (T, Hkv, D)):
+        raise ValueError("k / v must be [num_tokens][num_kv_heads][head_dim]")
+    dev = _device(k_cache)
+    args = (_dev(k_cache, "k_cache", torch.float8_e4m3fn, device=dev),
+            _dev(v_cache, "v_cache", torch.float8_e4m3fn, device=dev),
+            _dev(k_scales, "k_scales", torch.float32, device=dev, shape=(Hkv,)),
+            _dev(v_scales, "v_scales", torch.float32, device=dev, shape=(Hkv,)),
+            _dev(k, "k", torch.bfloat16, device=dev) if T else None,
+            _dev(v, "v", torch.bfloat16, device=dev) if T else None,
+            _dev(slot_mapping, "slot_mapping", torch.int64, device=dev, shape=(T,)) if T else None)
+    with torch.cuda.device(dev):
+        rc = lib.kv_cache_append_fp8(*args, T, Hkv, D, bs, N, _stream(stream, dev))
     _check(rc, "kv_cache_append_fp8")
 
 
@@ -229,13 +274,17 @@ def paged_attention_decode_noalloc(out, q, k_cache, v_cache, block_tables, conte
     N, Hkv, bs, D2 = k_cache.shape
     if D2 != D or tuple(out.shape) != (B, H, D) or tuple(v_cache.shape) != tuple(k_cache.shape):
         raise ValueError("shape mismatch between q, out and the caches")
-    maxb = block_tables.shape[1] if block_tables.dim() == 2 else 0
-    rc = lib.paged_attention_decode_noalloc(
-        _dev(out, "out", q.dtype), _dev(q, "q"), _dev(k_cache, "k_cache", q.dtype),
-        _dev(v_cache, "v_cache", q.dtype), _dev(block_tables, "block_tables", torch.int32),
-        _dev(context_lens, "context_lens", torch.int32), B, H, Hkv, D, bs, maxb, float(scale),
-        N if num_blocks is None else int(num_blocks), _dtype_code(q), int(partition_tokens),
-        _stream(stream))
+    maxb = _tables(block_tables, context_lens, B)
+    dev = _device(q)
+    args = (_dev(out, "out", q.dtype, device=dev), _dev(q, "q", device=dev),
+            _dev(k_cache, "k_cache", q.dtype, device=dev), _dev(v_cache, "v_cache", q.dtype, device=dev),
+            _dev(block_tables, "block_tables", torch.int32, device=dev),
+            _dev(context_lens, "context_lens", torch.int32, device=dev))
+    with torch.cuda.device(dev):
+        rc = lib.paged_attention_decode_noalloc(*args, B, H, Hkv, D, bs, maxb, float(scale),
+                                                N if num_blocks is None else int(num_blocks),
+                                                _dtype_code(q), int(partition_tokens),
+                                                _stream(stream, dev))
     _check(rc, "paged_attention_decode_noalloc")
 
 
@@ -243,13 +292,19 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens,
                            stream=None) -> None:
     """bf16 form with the library-owned workspace (see include/pagedkv.h)."""
     B, H, D = q.shape
-    N, Hkv, bs, _ = k_cache.shape
-    rc = lib.paged_attention_decode(
-        _dev(out, "out", torch.bfloat16), _dev(q, "q", torch.bfloat16),
-        _dev(k_cache, "k_cache", torch.bfloat16), _dev(v_cache, "v_cache", torch.bfloat16),
-        _dev(block_tables, "block_tables", torch.int32),
-        _dev(context_lens, "context_lens", torch.int32), B, H, Hkv, D, bs, block_tables.shape[1],
-        float(scale), _stream(stream))
+    N, Hkv, bs, D2 = k_cache.shape
+    if D2 != D or tuple(out.shape) != (B, H, D) or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("shape mismatch between q, out and the caches")
+    maxb = _tables(block_tables, context_lens, B)
+    dev = _device(q)
+    args = (_dev(out, "out", torch.bfloat16, device=dev), _dev(q, "q", torch.bfloat16, device=dev),
+            _dev(k_cache, "k_cache", torch.bfloat16, device=dev),
+            _dev(v_cache, "v_cache", torch.bfloat16, device=dev),
+            _dev(block_tables, "block_tables", torch.int32, device=dev),
+            _dev(context_lens, "context_lens", torch.int32, device=dev))
+    with torch.cuda.device(dev):
+        rc = lib.paged_attention_decode(*args, B, H, Hkv, D, bs, maxb, float(scale),
+                                        _stream(stream, dev))
     _check(rc, "paged_attention_decode")
 
 
@@ -257,13 +312,17 @@ def kv_cache_append(k_cache, v_cache, k, v, slot_mapping, stream=None) -> None:
     """k, v: [T][Hkv][D]; slot_mapping int64 [T] (-1 = skip)."""
     T = slot_mapping.shape[0]
     N, Hkv, bs, D = k_cache.shape
+    if tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("k_cache and v_cache must have the same shape")
     if T and (tuple(k.shape) != (T, Hkv, D) or tuple(v.shape) != (T, Hkv, D)):
         raise ValueError("k / v must be [num_tokens][num_kv_heads][head_dim]")
-    rc = lib.kv_cache_append(
-        _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache", k_cache.dtype),
-        _dev(k, "k", k_cache.dtype) if T else None, _dev(v, "v", k_cache.dtype) if T else None,
-        _dev(slot_mapping, "slot_mapping", torch.int64) if T else None, T, Hkv, D, bs, N,
-        _dtype_code(k_cache), _stream(stream))
+    dev = _device(k_cache)
+    args = (_dev(k_cache, "k_cache", device=dev), _dev(v_cache, "v_cache", k_cache.dtype, device=dev),
+            _dev(k, "k", k_cache.dtype, device=dev) if T else None,
+            _dev(v, "v", k_cache.dtype, device=dev) if T else None,
+            _dev(slot_mapping, "slot_mapping", torch.int64, device=dev, shape=(T,)) if T else None)
+    with torch.cuda.device(dev):
+        rc = lib.kv_cache_append(*args, T, Hkv, D, bs, N, _dtype_code(k_cache), _stream(stream, dev))
     _check(rc, "kv_cache_append")
 
 
@@ -271,21 +330,28 @@ def copy_blocks(k_cache, v_cache, src_dst_pairs, stream=None) -> None:
     """src_dst_pairs: int64 [n][2] of (src, dst) physical blocks."""
     n = src_dst_pairs.shape[0]
     N, Hkv, bs, D = k_cache.shape
-    rc = lib.copy_blocks(
-        _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache", k_cache.dtype),
-        _dev(src_dst_pairs, "src_dst_pairs", torch.int64) if n else None, n, Hkv, D, bs, N,
-        _dtype_code(k_cache), _stream(stream))
+    if tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("k_cache and v_cache must have the same shape")
+    dev = _device(k_cache)
+    args = (_dev(k_cache, "k_cache", device=dev), _dev(v_cache, "v_cache", k_cache.dtype, device=dev),
+            _dev(src_dst_pairs, "src_dst_pairs", torch.int64, device=dev, shape=(n, 2)) if n else None)
+    with torch.cuda.device(dev):
+        rc = lib.copy_blocks(*args, n, Hkv, D, bs, N, _dtype_code(k_cache), _stream(stream, dev))
     _check(rc, "copy_blocks")
 
 
-def _reachable(t: torch.Tensor, name: str, dtype=None) -> int:
-    """Pointer of a device tensor or of a pinned host tensor (swap pools)."""
+def _reachable(t: torch.Tensor, name: str, dtype=None, *, device=None, shape=None) -> int:
+    """Pointer of a device tensor (on `device`) or of a pinned host tensor (swap pools)."""
     if not (t.is_cuda or t.is_pinned()):
         raise ValueError(f"{name} must be a CUDA tensor or pinned host memory")
+    if t.is_cuda and device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the other device tensors on {device}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
     return t.data_ptr()
 
 
@@ -297,11 +363,16 @@ def swap_blocks(dst_k, dst_v, src_k, src_v, src_dst_pairs, stream=None) -> None:
     Nd = dst_k.shape[0]
     if tuple(dst_k.shape[1:]) != (Hkv, bs, D):
         raise ValueError("source and destination pools must share the block layout")
-    rc = lib.swap_blocks(
-        _reachable(dst_k, "dst_k"), _reachable(dst_v, "dst_v", dst_k.dtype),
-        _reachable(src_k, "src_k", dst_k.dtype), _reachable(src_v, "src_v", dst_k.dtype),
-        _reachable(src_dst_pairs, "src_dst_pairs", torch.int64) if n else None, n, Hkv, D, bs, Ns,
-        Nd, _dtype_code(dst_k), _stream(stream))
+    if tuple(src_v.shape) != tuple(src_k.shape) or tuple(dst_v.shape) != tuple(dst_k.shape):
+        raise ValueError("K and V pools must have the same shape")
+    dev = _device(dst_k, src_k, src_dst_pairs)
+    args = (_reachable(dst_k, "dst_k", device=dev), _reachable(dst_v, "dst_v", dst_k.dtype, device=dev),
+            _reachable(src_k, "src_k", dst_k.dtype, device=dev),
+            _reachable(src_v, "src_v", dst_k.dtype, device=dev),
+            _reachable(src_dst_pairs, "src_dst_pairs", torch.int64, device=dev, shape=(n, 2))
+            if n else None)
+    with torch.cuda.device(dev):
+        rc = lib.swap_blocks(*args, n, Hkv, D, bs, Ns, Nd, _dtype_code(dst_k), _stream(stream, dev))
     _check(rc, "swap_blocks")
 
 
