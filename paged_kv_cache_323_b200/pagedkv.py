@@ -395,14 +395,17 @@ class BlockManager:
         if free_order is not None:
             order = np.ascontiguousarray(free_order, dtype=np.int32)
         self.block_size = block_size
+        # the instance keeps the library: at interpreter exit the module's
+        # globals may be cleared before this object is collected
+        self._lib = lib
         self._h = lib.pkv_bm_create(num_blocks, block_size, num_host_blocks,
                                     order.ctypes.data if order is not None else None)
         if not self._h:
             raise ValueError("pkv_bm_create rejected its arguments")
 
     def close(self) -> None:
-        if self._h:
-            lib.pkv_bm_destroy(self._h)
+        if getattr(self, "_h", None):
+            self._lib.pkv_bm_destroy(self._h)
             self._h = None
 
     def __del__(self):
