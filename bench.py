@@ -303,6 +303,7 @@ def compact_subset(w: wl.Workload, seqs):
 
 
 def oracle_sample_step(sub, scale, threads):
+    """One step of the oracle on a compact sample: (seconds, fp64 output rows)."""
     import oracle
 
     kc = sub["kc"].copy()
@@ -313,26 +314,40 @@ def oracle_sample_step(sub, scale, threads):
     if sub["k_scales"] is not None:  # fp8 cache
         oracle.kv_append_fp8(kc, vc, sub["k_scales"], sub["v_scales"], sub["k_new"], sub["v_new"],
                              sub["slots"])
-        oracle.paged_attention_fp8(sub["q"], kc, vc, sub["k_scales"], sub["v_scales"], sub["bt"],
-                                   sub["ctx"], scale)
-        return time.perf_counter() - t0
+        out = oracle.paged_attention_fp8(sub["q"], kc, vc, sub["k_scales"], sub["v_scales"],
+                                         sub["bt"], sub["ctx"], scale)
+        return time.perf_counter() - t0, out
     oracle.kv_append(kc, vc, sub["k_new"], sub["v_new"], sub["slots"])
-    oracle.paged_attention(sub["q"], kc, vc, sub["bt"], sub["ctx"], scale, nthreads=threads)
-    return time.perf_counter() - t0
+    out = oracle.paged_attention(sub["q"], kc, vc, sub["bt"], sub["ctx"], scale, nthreads=threads)
+    return time.perf_counter() - t0, out
 
 
 def pick_sample(w: wl.Workload, target_s: float, threads: int):
-    """Grow a seeded sample of sequences until one oracle step costs about target_s."""
+    """Grow a seeded sample of sequences until one oracle step costs about
+    target_s; returns (sample, sequences, seconds, the sample's output rows)."""
     rng = np.random.default_rng(1234)
     order = rng.permutation(w.num_seqs).tolist()
     n = min(len(order), max(1, threads))
     while True:
-        sub = compact_subset(w, sorted(order[:n]))
-        dt = oracle_sample_step(sub, w.scale, threads)
+        seqs = sorted(order[:n])
+        sub = compact_subset(w, seqs)
+        dt, out = oracle_sample_step(sub, w.scale, threads)
         if dt >= target_s / 4 or n >= len(order):
             break
         n = min(len(order), max(n + 1, int(n * min(8.0, target_s / 4 / max(dt, 1e-3)))))
-    return sub, n, dt
+    sub["seqs"] = seqs
+    return sub, n, dt, out
+
+
+# Parity bar of bf16 (and fp8-cache) outputs against the fp64 oracle:
+# |gpu - ref| <= 2e-2 + 1e-2 |ref| per element; fp32: |gpu - ref| <= 1e-5.
+def rows_match(gpu_rows: torch.Tensor, ref: np.ndarray, dtype: str) -> dict:
+    g = gpu_rows.detach().float().cpu().double().numpy().reshape(ref.shape)
+    err = np.abs(g - ref)
+    ok = bool(np.all(np.isfinite(g))) and (
+        bool(err.max() <= 1e-5) if dtype == "f32" else bool(np.all(err <= 2e-2 + 1e-2 * np.abs(ref))))
+    return {"rows": int(ref.shape[0] * ref.shape[1]), "max_abs_err": float(err.max()), "ok": ok,
+            "bar": "max abs 1e-5" if dtype == "f32" else "|gpu - ref| <= 2e-2 + 1e-2 |ref|"}
 
 
 def measure_swap(pk, w, stream, nblocks: int = 1024, reps: int = 5) -> dict:
@@ -381,10 +396,10 @@ def run_reference(args, world, rank):
     # pools); the timed work is the oracle on host cores either way
     w = make("cuda" if torch.cuda.is_available() else "cpu", DEFAULT_SEED[args.workload])
     threads = cpu_threads()
-    sub, n, _ = pick_sample(w, target_s=8.0 / max(1, args.steps), threads=threads)
+    sub, n, _, _ = pick_sample(w, target_s=8.0 / max(1, args.steps), threads=threads)
     for _ in range(min(args.warmup, 1)):
         oracle_sample_step(sub, w.scale, threads)
-    times = [oracle_sample_step(sub, w.scale, threads) for _ in range(args.steps)]
+    times = [oracle_sample_step(sub, w.scale, threads)[0] for _ in range(args.steps)]
     t = sum(times) / len(times)
     value = sub["kv_bytes"] / t / 1e9
     sample = f"{n} of {w.num_seqs} sequences (seeded), all heads, per step"
@@ -401,91 +416,102 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
-def run_gpu(args, world, rank, local):
-    from paged_kv_cache_323_b200 import pagedkv as pk
+# Configurations measured beside the headline in the default run: the
+# parallel-sampling GQA batch, the long-context split-K batch and the
+# prefix-sharing block-size sweep.
+DEFAULT_CONFIGS = ("gqa_sampling", "long_context", "prefix_bs8", "prefix_bs16", "prefix_bs32")
+L2_FLUSH_BYTES = 512 << 20  # written before each cold step: four times the 126 MB L2
 
-    name, make = WORKLOADS[args.workload]
-    w = make("cuda", rank_seed(args.workload, rank))
-    dev = torch.device("cuda", torch.cuda.current_device())
-    t = {
+
+def device_inputs(w, dev) -> dict:
+    return {
         "q": w.q, "k_cache": w.k_cache, "v_cache": w.v_cache, "k_new": w.k_new, "v_new": w.v_new,
         "bt": torch.from_numpy(w.block_tables).to(dev),
         "ctx": torch.from_numpy(w.context_lens).to(dev),
         "slots": torch.from_numpy(w.slot_mapping).to(dev),
         "pairs": torch.from_numpy(w.cow_pairs).to(dev),
     }
-    out = torch.empty_like(w.q)
-    ws_bytes = pk.paged_attention_workspace_size(w.num_seqs, w.num_heads,
-                                                 w.max_blocks_per_seq * w.block_size, w.head_dim,
-                                                 args.partition_tokens)
-    ws = torch.zeros(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
 
-    fp8 = w.dtype == "fp8"
-    if fp8:
-        ks = torch.from_numpy(w.k_scales).to(dev)
-        vs = torch.from_numpy(w.v_scales).to(dev)
 
-    def step(q, k_new, v_new, bt, ctx, slots):
+class Step:
+    """One pass of the hot path on a workload through the binding: the
+    copy-on-write copies (if any), the append, the decode with a caller
+    workspace.  Calling it with a set of per-step inputs (q, new K/V, slots,
+    tables, lengths) writes the decode output into ``self.out``."""
+
+    def __init__(self, pk, w, t, dev, partition_tokens):
+        self.pk, self.w, self.t, self.pt = pk, w, t, partition_tokens
+        self.out = torch.empty_like(w.q)
+        self.ws_bytes = pk.paged_attention_workspace_size(
+            w.num_seqs, w.num_heads, w.max_blocks_per_seq * w.block_size, w.head_dim,
+            partition_tokens)
+        self.ws = torch.zeros(max(self.ws_bytes, 1), dtype=torch.uint8, device=dev)
+        self.fp8 = w.dtype == "fp8"
+        if self.fp8:
+            self.ks = torch.from_numpy(w.k_scales).to(dev)
+            self.vs = torch.from_numpy(w.v_scales).to(dev)
+        self.dev_args = (t["q"], t["k_new"], t["v_new"], t["bt"], t["ctx"], t["slots"])
+
+    def __call__(self, q, k_new, v_new, bt, ctx, slots, out=None):
+        pk, w, t = self.pk, self.w, self.t
+        out = self.out if out is None else out
+        ws = self.ws if self.ws_bytes else None
         if len(w.cow_pairs):
             pk.copy_blocks(t["k_cache"], t["v_cache"], t["pairs"])
-        if fp8:
-            pk.kv_cache_append_fp8(t["k_cache"], t["v_cache"], ks, vs, k_new, v_new, slots)
-            pk.paged_attention_decode_fp8(out, q, t["k_cache"], t["v_cache"], ks, vs, bt, ctx,
-                                          w.scale, num_blocks=w.num_blocks,
-                                          partition_tokens=args.partition_tokens,
-                                          workspace=ws if ws_bytes else None)
+        if self.fp8:
+            pk.kv_cache_append_fp8(t["k_cache"], t["v_cache"], self.ks, self.vs, k_new, v_new, slots)
+            pk.paged_attention_decode_fp8(out, q, t["k_cache"], t["v_cache"], self.ks, self.vs, bt,
+                                          ctx, w.scale, num_blocks=w.num_blocks,
+                                          partition_tokens=self.pt, workspace=ws)
             return
         pk.kv_cache_append(t["k_cache"], t["v_cache"], k_new, v_new, slots)
         pk.paged_attention_decode_ex(out, q, t["k_cache"], t["v_cache"], bt, ctx, w.scale,
-                                     num_blocks=w.num_blocks,
-                                     partition_tokens=args.partition_tokens,
-                                     workspace=ws if ws_bytes else None)
+                                     num_blocks=w.num_blocks, partition_tokens=self.pt,
+                                     workspace=ws)
 
-    dev_args = (t["q"], t["k_new"], t["v_new"], t["bt"], t["ctx"], t["slots"])
-    for _ in range(args.warmup):
-        step(*dev_args)
-    torch.cuda.synchronize()
-    code = pk.get_device_error()
-    if code != 0:
-        raise RuntimeError(f"device error word {code} after warm-up")
 
-    # ------------------------------------------------ device-resident timing
-    # The headline region runs the steps bare.  Per-kernel durations come from
-    # a second region of the same steps in which the library brackets every
-    # launch with CUDA events on its stream (those events cost a few percent
-    # of the step, so they stay out of the headline).
-    clocks = ClockSampler(torch.cuda.current_device())
-    barrier(world)
-    torch.cuda.synchronize()
-    clocks.start()
-    launches0 = pk.launch_count()
+def timed_region(step, steps, world, stream) -> float:
+    """Exactly `steps` steps between a barrier + synchronize on both sides,
+    timed by CUDA events on the launching stream; the slowest rank's ms."""
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
     ev0.record(stream)
-    for _ in range(args.steps):
-        step(*dev_args)
+    for _ in range(steps):
+        step(*step.dev_args)
     ev1.record(stream)
     torch.cuda.synchronize()
-    launches = pk.launch_count() - launches0
     barrier(world)
-    ms = max_over_ranks(world, ev0.elapsed_time(ev1))
+    return max_over_ranks(world, ev0.elapsed_time(ev1))
 
+
+def repeated_regions(step, steps, world, stream, min_s: float):
+    """The timed region repeated until the repeats span at least `min_s`
+    seconds (every rank runs the same number); returns the ms of each."""
+    first = timed_region(step, steps, world, stream)
+    reps = int(min(200, max(1, -(-min_s * 1e3 // max(first, 1e-3)))))
+    reps = int(max_over_ranks(world, float(reps)))
+    return [first] + [timed_region(step, steps, world, stream) for _ in range(reps - 1)]
+
+
+def profiled_region(pk, step, steps, world, stream):
+    """The same steps with the library's per-launch events on (they cost a
+    few percent, so this region stays out of the headline): the mean device
+    time of each kernel and per-step percentiles."""
     pk.profile_reset()
     pk.profile_enable(True)
-    step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-    ev0.record(stream)
+    step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    barrier(world)
+    torch.cuda.synchronize()
     step_ev[0].record(stream)
-    for i in range(args.steps):
-        step(*dev_args)
+    for i in range(steps):
+        step(*step.dev_args)
         step_ev[i + 1].record(stream)
-    ev1.record(stream)
     torch.cuda.synchronize()
     pk.profile_enable(False)
-    step_ms = sorted(step_ev[i].elapsed_time(step_ev[i + 1]) for i in range(args.steps))
-    clock_info = clocks.stop()
     barrier(world)
-    ms_profiled = max_over_ranks(world, ev0.elapsed_time(ev1))
+    step_ms = sorted(step_ev[i].elapsed_time(step_ev[i + 1]) for i in range(steps))
     per_kernel = {}
     for kind, kname in ((pk.KERNEL_DECODE, "decode"), (pk.KERNEL_APPEND, "kv_append"),
                         (pk.KERNEL_COPY_BLOCKS, "copy_blocks")):
@@ -493,19 +519,146 @@ def run_gpu(args, world, rank, local):
         if n:
             per_kernel[kname] = {"launches": n, "avg_us": kms / n * 1e3}
     pk.profile_reset()
+    pct = {"p10": step_ms[len(step_ms) // 10], "p50": step_ms[len(step_ms) // 2],
+           "p90": step_ms[(9 * len(step_ms)) // 10]}
+    return per_kernel, pct
+
+
+def cold_l2_steps(step, steps, stream, flush) -> float:
+    """Median ms of single steps, each timed alone right after a 512 MB write
+    (outside its events) has pushed every earlier byte out of L2."""
+    times = []
+    for _ in range(steps):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step(*step.dev_args)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times)
+
+
+def waste_of(w) -> dict:
+    wst = w.padded_slot_waste()
+    return {"per_sequence": wst["per_sequence_unused"] / max(1, wst["per_sequence_allocated"]),
+            "physical": wst["physical_unused"] / max(1, wst["physical_allocated"])}
+
+
+def partition_of(pk, w, partition_tokens) -> int:
+    return pk.paged_attention_partition_tokens(
+        w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.block_size,
+        w.max_blocks_per_seq * w.block_size,
+        {"f32": pk.PKV_F32, "bf16": pk.PKV_BF16, "fp8": pk.PKV_FP8_E4M3}[w.dtype], partition_tokens)
+
+
+def oracle_check(w, step, target_s: float, threads: int) -> dict:
+    """CPU baseline of a configuration: the oracle as it stands, timed on
+    this host's cores over a seeded sample of the batch, and its rows
+    compared with the GPU step's rows for the same sequences."""
+    sub, n, dt, ref = pick_sample(w, target_s=target_s, threads=threads)
+    got = step.out.index_select(0, torch.tensor(sub["seqs"], device=step.out.device))
+    return {"value": sub["kv_bytes"] / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} of {w.num_seqs} sequences (seeded), all heads, one step in {dt:.2f} s",
+            "parity": rows_match(got, ref, w.dtype)}
+
+
+def measure_config(pk, key, args, world, rank, stream, peak, flush) -> dict:
+    """One configuration of the default run's `configs` map."""
+    name, make = WORKLOADS[key]
+    w = make("cuda", rank_seed(key, rank))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    step = Step(pk, w, device_inputs(w, dev), dev, args.partition_tokens)
+    for _ in range(args.warmup):
+        step(*step.dev_args)
+    torch.cuda.synchronize()
+    code = pk.get_device_error()
+    if code != 0:
+        raise RuntimeError(f"{key}: device error word {code} after warm-up")
+    runs = repeated_regions(step, args.steps, world, stream, min_s=args.min_region_s / 2)
+    ms = statistics.median(runs) / args.steps
+    per_kernel, pct = profiled_region(pk, step, args.steps, world, stream)
+    cold_ms = max_over_ranks(world, cold_l2_steps(step, min(args.steps, 10), stream, flush))
+    logical, unique = w.kv_bytes_logical(), w.kv_bytes_unique()
+    dec_us = per_kernel.get("decode", {}).get("avg_us")
+    fam = decode_kernel_family(w)
+    traffic = committed_traffic("decode", key, kernel_source_sha(fam))
+    shared = unique < logical
+    e = {
+        "workload": name, "kernel": fam, "partition_tokens": partition_of(pk, w, args.partition_tokens),
+        "step_us": ms * 1e3, "step_us_pct": {k: v * 1e3 for k, v in pct.items()},
+        "step_us_cold_l2": cold_ms * 1e3, "decode_us": dec_us,
+        "tokens_per_s": world * w.num_seqs / (ms / 1e3),
+        "kv_bytes_per_step": {"logical": logical, "unique": unique},
+        # logical: every sequence's context bytes; unique: each physical block once
+        "kv_gbs_logical": job_value(world, logical, ms), "kv_gbs_unique": job_value(world, unique, ms),
+        "pct_of_peak_hbm": 100.0 * job_value(world, logical, ms) / peak,
+        "decode_kernel": None if dec_us is None else {
+            "logical_gbs": logical / (dec_us * 1e-6) / 1e9,
+            "frac_logical": logical / (dec_us * 1e-6) / 1e9 / peak,
+            "unique_gbs": unique / (dec_us * 1e-6) / 1e9,
+            "dram_gbs": None if traffic is None else traffic / (dec_us * 1e-6) / 1e9,
+            "frac_dram": None if traffic is None else traffic / (dec_us * 1e-6) / 1e9 / peak,
+            "dram_bytes_per_launch": traffic},
+        "l2": ("warm: steps back to back; the shared prefix blocks stay in L2 across sequences"
+               if shared else "warm: steps back to back; the KV read per step is larger than L2")
+              + "; step_us_cold_l2 flushes L2 (512 MB write) before each step",
+        "padded_slot_waste": waste_of(w),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        e["cpu_baseline"] = oracle_check(w, step, target_s=1.5, threads=cpu_threads())
+    del step, w
+    torch.cuda.empty_cache()
+    return e
+
+
+def run_gpu(args, world, rank, local):
+    from paged_kv_cache_323_b200 import pagedkv as pk
+
+    pk.set_longest_first(not args.index_order)
+    name, make = WORKLOADS[args.workload]
+    w = make("cuda", rank_seed(args.workload, rank))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    step = Step(pk, w, device_inputs(w, dev), dev, args.partition_tokens)
+    for _ in range(args.warmup):
+        step(*step.dev_args)
+    torch.cuda.synchronize()
+    code = pk.get_device_error()
+    if code != 0:
+        raise RuntimeError(f"device error word {code} after warm-up")
+
+    # ------------------------------------------------ device-resident timing
+    # The headline region runs exactly `steps` steps bare; it is repeated
+    # until the repeats span half a second (so the clock sampler sees the
+    # load) and the median repeat is reported.  Per-kernel durations come
+    # from a second region of the same steps in which the library brackets
+    # every launch with CUDA events on its stream.
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    launches0 = pk.launch_count()
+    runs = repeated_regions(step, args.steps, world, stream, min_s=args.min_region_s)
+    launches = (pk.launch_count() - launches0) // len(runs)
+    ms = statistics.median(runs)
+    per_kernel, pct = profiled_region(pk, step, args.steps, world, stream)
+    clock_info = clocks.stop()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    cold_ms = max_over_ranks(world, cold_l2_steps(step, min(args.steps, 20), stream, flush))
 
     # -------------------------------------------- end to end from host memory
     # Every step uploads its inputs (q, new K/V, slots, tables, lengths) from
     # pinned host memory and reads its output back.  Uploads and read-backs
-    # run on a copy stream with double-buffered device staging, so step i+1's
-    # upload and step i-1's read-back overlap step i's kernels; the KV pool
-    # stays resident (it is the cache itself).
+    # run on copy streams with double-buffered device staging, so step i+1's
+    # upload and step i-1's read-back overlap step i's kernels: the figure is
+    # pipelined throughput, not the latency of one step.  The KV pool stays
+    # resident (it is the cache itself).
     names = ("q", "k_new", "v_new", "bt", "ctx", "slots")
     host = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True).copy_(v)
-            for k, v in zip(names, dev_args)}
-    staged = [{k: torch.empty_like(v) for k, v in zip(names, dev_args)} for _ in range(2)]
-    outs = [torch.empty_like(out) for _ in range(2)]
-    out_host = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
+            for k, v in zip(names, step.dev_args)}
+    staged = [{k: torch.empty_like(v) for k, v in zip(names, step.dev_args)} for _ in range(2)]
+    outs = [torch.empty_like(step.out) for _ in range(2)]
+    out_host = [torch.empty(step.out.shape, dtype=step.out.dtype, pin_memory=True) for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = out_host[0].numel() * out_host[0].element_size()
     up_stream = torch.cuda.Stream()    # host -> device
@@ -521,8 +674,6 @@ def run_gpu(args, world, rank, local):
             ev_up[b].record(up_stream)
 
     def e2e_run(n):
-        nonlocal out
-        keep = out
         upload(0)
         for i in range(n):
             b = i % 2
@@ -533,9 +684,8 @@ def run_gpu(args, world, rank, local):
             stream.wait_event(ev_up[b])
             if i >= 2:
                 stream.wait_event(ev_back[b])  # outs[b] was read back
-            out = outs[b]
             sb = staged[b]
-            step(sb["q"], sb["k_new"], sb["v_new"], sb["bt"], sb["ctx"], sb["slots"])
+            step(sb["q"], sb["k_new"], sb["v_new"], sb["bt"], sb["ctx"], sb["slots"], out=outs[b])
             ev_used[b].record(stream)
             down_stream.wait_event(ev_used[b])
             with torch.cuda.stream(down_stream):
@@ -543,9 +693,10 @@ def run_gpu(args, world, rank, local):
                 ev_back[b].record(down_stream)
         stream.wait_stream(up_stream)
         stream.wait_stream(down_stream)
-        out = keep
 
     e2e_run(args.warmup)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     ev0.record(stream)
@@ -554,22 +705,17 @@ def run_gpu(args, world, rank, local):
     torch.cuda.synchronize()
     barrier(world)
     ms_e2e = max_over_ranks(world, ev0.elapsed_time(ev1))
-    if not torch.equal(out_host[(args.steps - 1) % 2], out.cpu()):
+    if not torch.equal(out_host[(args.steps - 1) % 2], step.out.cpu()):
         raise RuntimeError("end-to-end output differs from the device-resident run")
     code = pk.get_device_error()
     if code != 0:
         raise RuntimeError(f"device error word {code} after the timed steps")
 
-    if rank != 0:
-        return
+    peak, peak_src = measured_peak()
     kv_bytes = w.kv_bytes_logical()
     kv_unique = w.kv_bytes_unique()
-    wst = w.padded_slot_waste()
-    waste = {"per_sequence": wst["per_sequence_unused"] / max(1, wst["per_sequence_allocated"]),
-             "physical": wst["physical_unused"] / max(1, wst["physical_allocated"])}
-    step_s = ms / args.steps / 1e3
-    value = job_value(world, kv_bytes, ms / args.steps)
-    peak, peak_src = measured_peak()
+    step_ms = ms / args.steps
+    value = job_value(world, kv_bytes, step_ms)
     part = per_kernel.get("decode")
     roofline = None
     if part:
@@ -581,58 +727,69 @@ def run_gpu(args, world, rank, local):
                     else "fallback 6650 GB/s"}
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": name, "num_seqs_per_gpu": w.num_seqs, "num_heads": w.num_heads,
                    "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
                    "block_size": w.block_size, "kv_bytes_per_step_per_gpu": kv_bytes,
                    "kv_bytes_unique_per_step_per_gpu": kv_unique,
-                   "padded_slot_waste": waste,
-                   "partition_tokens": pk.paged_attention_partition_tokens(
-                       w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.block_size,
-                       w.max_blocks_per_seq * w.block_size,
-                       {"f32": pk.PKV_F32, "bf16": pk.PKV_BF16, "fp8": pk.PKV_FP8_E4M3}[w.dtype],
-                       args.partition_tokens),
+                   "padded_slot_waste": waste_of(w),
+                   "partition_tokens": partition_of(pk, w, args.partition_tokens),
                    "accumulate": "f32",
-                   "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush",
+                   "schedule": "index order" if args.index_order else "longest first",
+                   "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush; "
+                         "step_us_cold_l2 flushes L2 before each step",
                    "parallelism": f"{world} independent batches, one per GPU"},
-        "tokens_per_s": world * w.num_seqs / step_s,
+        "timing": {"repeats": len(runs), "steps_per_repeat": args.steps,
+                   "region_s": sum(runs) / 1e3, "statistic": "median repeat",
+                   "repeat_ms_per_step": {"min": min(runs) / args.steps,
+                                          "max": max(runs) / args.steps}},
+        "tokens_per_s": world * w.num_seqs / (step_ms / 1e3),
         # shared blocks counted once (equal to `value` when nothing is shared)
-        "unique_kv_gbs": job_value(world, kv_unique, ms / args.steps),
+        "unique_kv_gbs": job_value(world, kv_unique, step_ms),
         "pct_of_peak_hbm": 100.0 * value / peak,
         "per_kernel_us": per_kernel,
-        "ms_per_step_profiled": ms_profiled / args.steps,
-        "ms_per_step_profiled_pct": {"p10": step_ms[len(step_ms) // 10],
-                                     "p50": step_ms[len(step_ms) // 2],
-                                     "p90": step_ms[(9 * len(step_ms)) // 10]},
+        "ms_per_step_profiled_pct": pct,
+        "step_us_cold_l2": cold_ms * 1e3,
         "roofline": roofline,
         "gpu_launches": launches,
         "e2e": {"value": job_value(world, kv_bytes, ms_e2e / args.steps), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": ms_e2e / args.steps},
+                "ms_per_step": ms_e2e / args.steps,
+                "mode": "pipelined: each step's uploads and read-back run on copy streams and "
+                        "overlap the neighbouring steps' kernels (throughput, not one step's latency)"},
         "clocks": clock_info,
     }
     if world == 1:
         line["swap"] = measure_swap(pk, w, stream)
     if world == 1 and not args.no_cpu_baseline:
         # the oracle as it stands, on this host's cores: a seeded sample of the
-        # batch, stepped repeatedly for about 10 s of CPU time
+        # batch, stepped repeatedly for about 10 s of CPU time; its rows are
+        # also compared with the GPU step's
         threads = cpu_threads()
-        sub, n, _ = pick_sample(w, target_s=10.0, threads=threads)
-        steps, spent = 0, 0.0
-        while spent < 10.0 and steps < 1000:
-            spent += oracle_sample_step(sub, w.scale, threads)
-            steps += 1
-        line["cpu_baseline"] = {"value": sub["kv_bytes"] * steps / spent / 1e9, "unit": "GB/s",
+        sub, n, _, ref = pick_sample(w, target_s=10.0, threads=threads)
+        got = step.out.index_select(0, torch.tensor(sub["seqs"], device=dev))
+        steps_run, spent = 0, 0.0
+        while spent < 10.0 and steps_run < 1000:
+            spent += oracle_sample_step(sub, w.scale, threads)[0]
+            steps_run += 1
+        line["cpu_baseline"] = {"value": sub["kv_bytes"] * steps_run / spent / 1e9, "unit": "GB/s",
                                 "cores": threads, "kind": "oracle",
                                 "sample": f"{n} of {w.num_seqs} sequences (seeded), all heads; "
-                                          f"{steps} steps in {spent:.1f} s"}
+                                          f"{steps_run} steps in {spent:.1f} s",
+                                "parity": rows_match(got, ref, w.dtype)}
         # and on one core, over a smaller sample (about 3 s)
-        sub1, n1, _ = pick_sample(w, target_s=3.0, threads=1)
-        t1 = oracle_sample_step(sub1, w.scale, 1)
+        sub1, n1, t1, _ = pick_sample(w, target_s=3.0, threads=1)
         line["cpu_baseline"]["value_1_core"] = sub1["kv_bytes"] / t1 / 1e9
         line["cpu_baseline"]["sample_1_core"] = f"{n1} of {w.num_seqs} sequences (seeded), one step"
-    print(json.dumps(line), flush=True)
+    configs = [] if args.no_configs or args.workload != "mha" else list(DEFAULT_CONFIGS)
+    if configs:
+        del step, staged, outs, w
+        torch.cuda.empty_cache()
+        line["configs"] = {k: measure_config(pk, k, args, world, rank, stream, peak, flush)
+                           for k in configs}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
 
 
 def main():
@@ -644,6 +801,13 @@ def main():
     ap.add_argument("--workload", default="mha", choices=sorted(WORKLOADS))
     ap.add_argument("--partition-tokens", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--index-order", action="store_true",
+                    help="run the decode grid in index order instead of longest first")
+    ap.add_argument("--min-region-s", type=float, default=0.5,
+                    help="repeat the timed region of K steps until the repeats span this long")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="headline workload only (the default mha run also measures "
+                         + ", ".join(DEFAULT_CONFIGS) + ")")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -68,7 +68,7 @@ typedef enum {
     PKV_ERR_INVALID = -2,       /* an argument is out of its documented range */
     PKV_ERR_UNSUPPORTED = -3,   /* a valid shape this build has no kernel for */
     PKV_ERR_CUDA = -4,          /* the CUDA runtime reported an error */
-    PKV_ERR_WORKSPACE = -5,     /* split-K workspace missing or too small */
+    PKV_ERR_WORKSPACE = -5,     /* decode workspace missing or too small */
     PKV_ERR_DEVICE_BOUNDS = -6, /* device word: a table entry, slot or length was out of range */
     PKV_ERR_TIMEOUT = -7,       /* device word: a bounded wait in a kernel ran out */
     PKV_ERR_OUT_OF_BLOCKS = -8  /* block manager: the free list cannot cover the request */
@@ -92,11 +92,23 @@ typedef enum {
  * every sequence s and query head h, out[s][h] = softmax(scale * q[s][h] .
  * K_s^T) V_s where K_s, V_s are the first context_lens[s] tokens of the
  * sequence gathered through block_tables (int32 [num_seqs][max_blocks_per_seq],
- * row-major).  This form takes bf16 data, does not range-check table entries
- * against the pool size (only against 0), partitions long contexts
- * automatically, and uses a workspace the library allocates and keeps per
- * device (grown with cudaMalloc when needed, so do not call it inside CUDA
- * graph capture on a new size).  Returns PKV_OK or a pkv_status.
+ * row-major).  This form takes bf16 data and partitions long contexts
+ * automatically.
+ *   - Pool bounds: its argument list carries no pool size, so table entries
+ *     are checked only against 0.  An entry at or past the end of the pool
+ *     is NOT detected: the kernel reads whatever device memory lies there,
+ *     which can fault the context.  Use paged_attention_decode_ex, whose
+ *     num_blocks turns such entries into device faults (block skipped, error
+ *     word set).
+ *   - Workspace: the library keeps one decode workspace per (device,
+ *     stream), so calls on different streams never share one.  It is grown
+ *     stream-ordered on the call's stream (cudaMallocAsync, zero fill, then
+ *     cudaFreeAsync of the old buffer), which neither synchronises nor
+ *     disturbs earlier launches on that stream.  A call made while the
+ *     stream is being captured into a CUDA graph that would have to grow it
+ *     returns PKV_ERR_WORKSPACE; inside capture, use paged_attention_decode_ex
+ *     with a caller workspace.  The buffers live until the process exits.
+ * Returns PKV_OK or a pkv_status.
  */
 PKV_API int paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
                            const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
@@ -117,13 +129,26 @@ PKV_API int paged_attention_decode(void* out, const void* q, const void* k_cache
  *   workspace         device memory of at least
  *                     paged_attention_workspace_size(num_seqs, num_heads,
  *                     max_blocks_per_seq*block_size, head_dim, partition_tokens)
- *                     bytes, 256-byte aligned, owned by the caller; may be
- *                     NULL when that size is 0.  It holds the partial results
- *                     and one merge counter per (sequence, kv head): it must
- *                     be zero-filled (e.g. cudaMemset) before its first use,
- *                     and every completed call leaves the counters at zero
- *                     again, so it can be reused without clearing.  Two calls
- *                     in flight at once must not share it.
+ *                     bytes, 256-byte aligned, owned by the caller.  It holds
+ *                     one split-K merge counter per (sequence, kv head) at its
+ *                     start, in a region nothing else uses, then the launch's
+ *                     schedule, then the partial results of split sequences.
+ *                     The schedule orders the grid's (sequence, partition)
+ *                     units longest first, written by a one-CTA planning
+ *                     kernel that the decode kernel follows as a programmatic
+ *                     dependent launch; it changes which SM runs a unit and
+ *                     when, never the arithmetic, so outputs are the same bits
+ *                     with or without it.  Zero-fill the workspace (e.g.
+ *                     cudaMemset) once before its first use.  Every call
+ *                     leaves the counters it used at zero again -- a call
+ *                     whose kernel stopped on PKV_ERR_TIMEOUT too -- so the
+ *                     same buffer serves later calls of any shape without
+ *                     clearing.  (A batch of more than 65536 (sequence, kv
+ *                     head) units also uses counters past that region; the
+ *                     call clears those itself, on `stream`, before its
+ *                     kernel.)  When no sequence is split, workspace may be
+ *                     NULL: the grid then runs in index order, unplanned.  Two
+ *                     calls in flight at once must not share a workspace.
  */
 PKV_API int paged_attention_decode_ex(void* out, const void* q, const void* k_cache, const void* v_cache,
                               const int32_t* block_tables, const int32_t* context_lens,
@@ -171,9 +196,10 @@ PKV_API int kv_cache_append_fp8(void* k_cache, void* v_cache, const float* k_sca
                                 const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
                                 int head_dim, int block_size, int num_blocks, void* stream);
 
-/* Bytes of split-K workspace paged_attention_decode_ex needs; 0 when every
- * sequence fits one partition.  With partition_tokens 0 the result covers
- * any automatic choice. */
+/* Bytes of workspace paged_attention_decode_ex uses (the merge counters'
+ * region, the schedule and, when sequences are split, the partial results);
+ * 0 only for num_seqs <= 0.  With partition_tokens 0 the result covers any
+ * automatic choice. */
 PKV_API size_t paged_attention_workspace_size(int num_seqs, int num_heads, int max_context, int head_dim,
                                       int partition_tokens);
 
@@ -222,8 +248,10 @@ PKV_API int copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_pai
  *     size chosen) exceeds PKV_NOALLOC_SCRATCH_BYTES returns
  *     PKV_ERR_WORKSPACE without launching anything; a larger partition_tokens
  *     lowers the need.
- *   - The first call on a device looks up the array's device address there
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Each call looks up the array's device address on the current device
+ *     (cudaGetSymbolAddress, which allocates nothing), so the address is
+ *     right after a device reset too.  The first call on a device may load
+ *     the library's device code there: make it before any stream capture.
  *   - All calls share the array and it keeps the last call's contents; each
  *     call clears the merge counters on its stream before its kernel.  Calls
  *     whose kernels overlap on the GPU (other streams, other threads) race on
@@ -257,7 +285,10 @@ PKV_API int swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void*
                         int dtype, void* stream);
 
 /* Synchronise `stream`, then return in *code the current device's error word
- * (PKV_OK, PKV_ERR_DEVICE_BOUNDS or PKV_ERR_TIMEOUT) and clear it. */
+ * (PKV_OK, PKV_ERR_DEVICE_BOUNDS or PKV_ERR_TIMEOUT) and clear it.  After
+ * PKV_ERR_TIMEOUT the outputs of the decode launch that timed out are not
+ * meaningful (they are finite: a stopped partition counts as empty), while
+ * the pools, the workspaces and the context stay valid for later calls. */
 PKV_API int pkv_get_device_error(void* stream, int* code);
 
 /* Self-test of the failure path: launches one warp that waits, with the
@@ -266,6 +297,29 @@ PKV_API int pkv_get_device_error(void* stream, int* code);
  * PKV_ERR_TIMEOUT (read it with pkv_get_device_error).  Nothing traps and the
  * context stays usable. */
 PKV_API int pkv_selftest_bounded_wait(int timeout_us, void* stream);
+
+/* Failure-path test hook: the limit, in microseconds, of the bounded waits
+ * inside the decode kernels' pipelines (1 .. 1e6; 0 restores the default of
+ * one second).  A limit far below a load's latency makes a real decode give
+ * up, which is how the timeout path (PKV_ERR_TIMEOUT, a stopped CTA's turn on
+ * its merge counter) is tested without a fault.  The wait that lets a
+ * stopped CTA's own copies land keeps its one-second bound.  Process-wide;
+ * read by each decode call at launch.  Returns the previous limit in
+ * microseconds, or PKV_ERR_INVALID. */
+PKV_API int pkv_set_wait_limit_us(int microseconds);
+
+/* Debug builds.  libpagedkv_debug.so is this library compiled with
+ * -DPKV_DEBUG: every index the kernels derive from the inputs (schedule
+ * entries, units, copy sources and destinations, workspace and output rows)
+ * is checked right before its use, and a failed check records
+ * PKV_ERR_DEVICE_BOUNDS in the error word and its source line, then skips the
+ * access instead of reading or writing out of bounds.  pkv_debug_build()
+ * returns 1 in that build, 0 in the release one.  pkv_debug_failed_line()
+ * synchronises `stream`, then returns in *line the source line of the first
+ * failed check since the last read (0: none; always 0 in release builds) and
+ * clears it. */
+PKV_API int pkv_debug_build(void);
+PKV_API int pkv_debug_failed_line(void* stream, int* line);
 
 /* Static English text of a status code. */
 PKV_API const char* pkv_status_string(int status);
@@ -287,6 +341,12 @@ PKV_API int pkv_profile_reset(void);
  * kernel that serves every other shape.  Both compute the same attention;
  * returns the previous setting.  Process-wide. */
 PKV_API int pkv_set_tensor_core_gqa(int enable);
+
+/* Schedule of the decode grid: 1 (default) orders the (sequence,
+ * partition) units longest first whenever the call has a workspace (see
+ * paged_attention_decode_ex), 0 runs them in index order.  Both give the same
+ * bits; only the time differs.  Process-wide; returns the previous setting. */
+PKV_API int pkv_set_longest_first(int enable);
 
 /* Kernels launched by this library in this process so far (all kinds). */
 PKV_API unsigned long long pkv_launch_count(void);

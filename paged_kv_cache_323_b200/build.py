@@ -1,7 +1,10 @@
 """Build libpagedkv.so in-tree: nvcc for sm_100a only, one object per .cu,
-compiled in parallel, linked with the static CUDA runtime.
+compiled in parallel, linked with the static CUDA runtime.  --debug builds
+libpagedkv_debug.so instead: the same sources with -DPKV_DEBUG, whose kernels
+check every derived index before its use (see pkv_debug_build in
+include/pagedkv.h).
 
-    python -m paged_kv_cache_323_b200.build [--force] [--verbose-ptxas]
+    python -m paged_kv_cache_323_b200.build [--force] [--verbose-ptxas] [--debug]
 """
 from __future__ import annotations
 
@@ -17,6 +20,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpagedkv.so")
+LIB_DEBUG = os.path.join(PKG, "libpagedkv_debug.so")
 SOURCES = ["api.cu", "decode_f32.cu", "decode_bf16.cu", "decode_fp8.cu", "decode_tc.cu", "decode_tc_fp8.cu",
            "noalloc.cu",
            "block_manager.cpp"]
@@ -39,28 +43,30 @@ def _inputs() -> list[str]:
             + [os.path.abspath(__file__)])
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
-    extra = ["-Xptxas", "-v"] if verbose_ptxas else []
+def build(force: bool = False, verbose_ptxas: bool = False, debug: bool = False) -> str:
+    lib = LIB_DEBUG if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
+    out_dir = os.path.join(BUILD, "debug") if debug else BUILD
+    os.makedirs(out_dir, exist_ok=True)
+    extra = (["-Xptxas", "-v"] if verbose_ptxas else []) + (["-DPKV_DEBUG"] if debug else [])
 
     def compile_one(src: str) -> str:
-        obj = os.path.join(BUILD, os.path.splitext(src)[0] + ".o")
+        obj = os.path.join(out_dir, os.path.splitext(src)[0] + ".o")
         if src.endswith(".cpp"):  # host-only C++: the host compiler through nvcc's flags
             cmd = [nvcc(), "-x", "c++", "-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler",
                    "-fvisibility=hidden", "-c", os.path.join(CSRC, src), "-o", obj]
         else:
             cmd = [nvcc()] + NVCC_FLAGS + extra + ["-c", os.path.join(CSRC, src), "-o", obj]
         p = subprocess.run(cmd, capture_output=True, text=True)
-        log = os.path.join(BUILD, src + ".log")
+        log = os.path.join(out_dir, src + ".log")
         with open(log, "w") as f:
             f.write(" ".join(cmd) + "\n" + p.stdout + p.stderr)
         if p.returncode != 0:
@@ -70,19 +76,20 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
 
     with ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
         objs = list(ex.map(compile_one, SOURCES))
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [nvcc()] + ARCH + ["-shared", "-o", tmp] + objs + ["-cudart", "static"]
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose-ptxas", action="store_true")
+    ap.add_argument("--debug", action="store_true", help="build libpagedkv_debug.so (-DPKV_DEBUG)")
     a = ap.parse_args()
-    print(build(force=a.force, verbose_ptxas=a.verbose_ptxas))
+    print(build(force=a.force, verbose_ptxas=a.verbose_ptxas, debug=a.debug))
 
 
 if __name__ == "__main__":

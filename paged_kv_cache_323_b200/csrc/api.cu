@@ -15,11 +15,13 @@
 #include "../../include/pagedkv.h"
 #include "kv_ops.cuh"
 #include "launch.h"
+#include "plan.cuh"
 
-// One error word per device (a __device__ variable exists once per device
-// context).  Kernels receive its device address; pkv_get_device_error reads
-// and clears it.
-__device__ int g_pkv_device_error;
+// One error record per device (a __device__ variable exists once per device
+// context): [0] the first device fault's status, [1] the source line of the
+// first failed index check (debug builds only).  Kernels receive its device
+// address; pkv_get_device_error reads and clears [0], pkv_debug_failed_line [1].
+__device__ int g_pkv_device_error[2];
 
 namespace {
 
@@ -28,16 +30,21 @@ constexpr int kAutoPartitionTokens = 1024;
 constexpr int kMinPartitionTokens = 512;  // bounds the automatic choice from below
 constexpr int kMaxPartitionTokens = 4096;
 
-struct DeviceState {
-    int* err = nullptr;     // device address of g_pkv_device_error
-    void* ws = nullptr;     // library-owned split-K workspace
-    size_t ws_bytes = 0;
+// Library-owned split-K workspace of paged_attention_decode: one buffer per
+// (device, stream), grown stream-ordered on that stream.
+struct StreamWorkspace {
+    int dev;
+    cudaStream_t stream;
+    void* ptr;
+    size_t bytes;
 };
 
 std::mutex g_mu;
-DeviceState g_dev[kMaxDevices];
+std::vector<StreamWorkspace> g_stream_ws;
 std::atomic<int> g_tc_gqa{1};  // tensor-core kernel for grouped-query heads where it applies
+std::atomic<int> g_longest_first{1};  // plan the decode grid longest first when there is a workspace
 std::atomic<unsigned long long> g_launches{0};
+std::atomic<unsigned long long> g_wait_ns{pkv::kWaitTimeoutNs};  // decode pipeline wait limit
 
 // ---------------------------------------------------------- profiler
 struct ProfRecord {
@@ -69,21 +76,24 @@ int current_device(int* dev) {
     return PKV_OK;
 }
 
+// Device address of the current device's error word.  Looked up on every
+// call (a symbol lookup, no allocation), so it stays right if the caller
+// resets the device and a new context takes the old one's place.
 int error_word(int dev, int** out) {
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (g_dev[dev].err == nullptr) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_pkv_device_error) != cudaSuccess) return PKV_ERR_CUDA;
-        g_dev[dev].err = static_cast<int*>(p);
+    (void)dev;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_pkv_device_error) != cudaSuccess || p == nullptr) {
+        cudaGetLastError();
+        return PKV_ERR_CUDA;
     }
-    *out = g_dev[dev].err;
+    *out = static_cast<int*>(p);
     return PKV_OK;
 }
 
-// Launch one kernel through `fn`, counting it and (when profiling) bracketing
-// it with events on its own stream.
+// Launch `kernels` kernels through `fn`, counting them and (when profiling)
+// bracketing them with one pair of events on their stream.
 template <class Fn>
-int launch(int kind, cudaStream_t st, Fn&& fn) {
+int launch(int kind, cudaStream_t st, Fn&& fn, int kernels = 1) {
     cudaEvent_t a = nullptr, b = nullptr;
     int dev = 0;
     bool prof = false;
@@ -100,7 +110,7 @@ int launch(int kind, cudaStream_t st, Fn&& fn) {
     if (prof) cudaEventRecord(a, st);
     cudaError_t e = fn();
     if (e == cudaSuccess) e = cudaGetLastError();
-    g_launches.fetch_add(1);
+    g_launches.fetch_add((unsigned long long)kernels);
     if (prof) {
         cudaEventRecord(b, st);
         std::lock_guard<std::mutex> lk(g_prof_mu);
@@ -125,19 +135,37 @@ bool decode_shape_supported(int head_dim, int block_size, int group) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Split-K workspace: [B][H][P][D] fp32 partial outputs, [B][H][P] (m, l)
-// pairs, then one int counter per (sequence, head) slot (used per kv head).
+// Decode workspace.  First the split-K merge counters, one int per
+// (sequence, kv head), in a region of at least kFixedCounterSlots slots at
+// offset 0 that nothing else is ever written to; then the longest-first
+// schedule of the launch ([B * P] ints); then, when sequences are split, the
+// fp32 partial outputs [B][H][P][D] and the (m, l) pairs [B][H][P]; each
+// region 256-byte aligned.  Every launch, complete or stopped by a timeout,
+// leaves the counters it used at zero, so the first kFixedCounterSlots
+// counters are zero between calls whatever shape each call has.  A batch
+// with more (sequence, kv head) units than that uses counters past the fixed
+// region, where an earlier call may have left other data: decode_impl clears
+// that part on every such call.
+constexpr long long kFixedCounterSlots = 65536;
+
 struct WorkspaceLayout {
-    size_t o_off, ml_off, cnt_off, total;
+    size_t cnt_off, plan_off, o_off, ml_off, total;
 };
 
 WorkspaceLayout workspace_layout(long long num_seqs, long long num_heads, long long parts, long long D) {
-    WorkspaceLayout w{0, 0, 0, 0};
-    if (parts <= 1) return w;
-    w.o_off = 0;
-    w.ml_off = align256(size_t(num_seqs) * num_heads * parts * D * sizeof(float));
-    w.cnt_off = w.ml_off + align256(size_t(num_seqs) * num_heads * parts * sizeof(float2));
-    w.total = w.cnt_off + align256(size_t(num_seqs) * num_heads * sizeof(int));
+    WorkspaceLayout w{0, 0, 0, 0, 0};
+    if (num_seqs <= 0 || parts <= 0) return w;
+    const long long slots = num_seqs * num_heads > kFixedCounterSlots ? num_seqs * num_heads
+                                                                      : kFixedCounterSlots;
+    w.cnt_off = 0;
+    w.plan_off = align256(size_t(slots) * sizeof(int));
+    w.o_off = w.plan_off + align256(size_t(num_seqs) * parts * sizeof(int));
+    w.ml_off = w.o_off;
+    w.total = w.o_off;
+    if (parts > 1) {
+        w.ml_off = w.o_off + align256(size_t(num_seqs) * num_heads * parts * D * sizeof(float));
+        w.total = w.ml_off + align256(size_t(num_seqs) * num_heads * parts * sizeof(float2));
+    }
     return w;
 }
 
@@ -213,9 +241,9 @@ extern "C" void pkv_internal_decode_scratch(int num_seqs, int num_heads, int num
     const long long parts = (max_ctx + pt - 1) / pt;
     const WorkspaceLayout w = workspace_layout(num_seqs, num_heads, parts, head_dim);
     *total = w.total;
-    if (w.total > 0) {
+    if (w.total > 0 && parts > 1) {
         *cnt_off = w.cnt_off;
-        *cnt_bytes = size_t(num_seqs) * num_heads * sizeof(int);
+        *cnt_bytes = size_t(num_seqs) * num_kv_heads * sizeof(int);
     }
 }
 
@@ -281,7 +309,9 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     const long long grid = parts * num_kv_heads * (long long)num_seqs;
     if (grid > INT_MAX || (long long)num_seqs * num_heads > INT_MAX) return PKV_ERR_INVALID;
     const size_t need = workspace_bytes_for(num_seqs, num_heads, parts, head_dim);
-    if (need > 0) {
+    // Split-K needs the workspace.  Without a split it only holds the
+    // longest-first schedule: a NULL workspace then runs in index order.
+    if (parts > 1 || workspace != nullptr) {
         if (workspace == nullptr || workspace_bytes < need ||
             (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
             return PKV_ERR_WORKSPACE;
@@ -300,9 +330,22 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     p.context_lens = context_lens;
     const WorkspaceLayout wl = workspace_layout(num_seqs, num_heads, parts, head_dim);
     char* wsb = static_cast<char*>(workspace);
-    p.ws_o = need > 0 ? reinterpret_cast<float*>(wsb + wl.o_off) : nullptr;
-    p.ws_ml = need > 0 ? reinterpret_cast<float2*>(wsb + wl.ml_off) : nullptr;
-    p.counters = need > 0 ? reinterpret_cast<int*>(wsb + wl.cnt_off) : nullptr;
+    const bool split = parts > 1;
+    p.ws_o = split ? reinterpret_cast<float*>(wsb + wl.o_off) : nullptr;
+    p.ws_ml = split ? reinterpret_cast<float2*>(wsb + wl.ml_off) : nullptr;
+    p.counters = split ? reinterpret_cast<int*>(wsb + wl.cnt_off) : nullptr;
+    int* order = workspace != nullptr && g_longest_first.load() != 0
+                     ? reinterpret_cast<int*>(wsb + wl.plan_off)
+                     : nullptr;
+    p.order = order;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const long long units = (long long)num_seqs * num_kv_heads;
+    if (split && units > kFixedCounterSlots) {
+        // counters past the fixed region may hold an earlier call's partials
+        if (cudaMemsetAsync(wsb + wl.cnt_off + kFixedCounterSlots * sizeof(int), 0,
+                            size_t(units - kFixedCounterSlots) * sizeof(int), st) != cudaSuccess)
+            return PKV_ERR_CUDA;
+    }
     p.k_scales = fp8 ? k_scales : nullptr;
     p.v_scales = fp8 ? v_scales : nullptr;
     p.err = err;
@@ -314,16 +357,24 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     p.partition_tokens = pt;
     p.num_partitions = (int)parts;
     p.qscale = scale * 1.4426950408889634f;  // log2(e): softmax runs in base 2
+    p.wait_ns = g_wait_ns.load();
 
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool use_tc = g_tc_gqa.load() != 0 &&
                         pkv::decode_tc_supported(kv_dtype, head_dim, block_size, group, pt);
+    // the schedule first (one CTA), then the decode grid as its programmatic
+    // dependent: counted and profiled together as the decode
     return launch(PKV_KERNEL_DECODE, st, [&] {
+        if (order != nullptr) {
+            pkv::plan_kernel<<<1, pkv::kPlanThreads, 0, st>>>(context_lens, num_seqs, (int)parts, pt,
+                                                            (int)max_ctx, order, err);
+            const cudaError_t e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+        }
         if (use_tc) return pkv::launch_decode_tc(p, kv_dtype, block_size, group, grid, st);
         if (fp8) return pkv::launch_decode_partition_fp8(p, head_dim, block_size, group, grid, st);
         return dtype == PKV_F32 ? pkv::launch_decode_partition_f32(p, head_dim, block_size, group, grid, st)
                                 : pkv::launch_decode_partition_bf16(p, head_dim, block_size, group, grid, st);
-    });
+    }, order != nullptr ? 2 : 1);
 }
 
 }  // namespace
@@ -367,20 +418,33 @@ int paged_attention_decode(void* out, const void* q, const void* k_cache, const 
     if (max_ctx > INT_MAX) return PKV_ERR_INVALID;
     const size_t need = paged_attention_workspace_size(num_seqs, num_heads, (int)max_ctx, head_dim, 0);
     void* ws = nullptr;
-    if (need > 0) {
+    if (need > 0) {  // always: the workspace holds the schedule
         int dev = 0;
         if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
+        cudaStream_t st = static_cast<cudaStream_t>(stream);
         std::lock_guard<std::mutex> lk(g_mu);
-        DeviceState& d = g_dev[dev];
-        if (d.ws_bytes < need) {
-            if (d.ws) cudaFree(d.ws);  // synchronises: no launch still reads the old buffer
-            d.ws = nullptr;
-            d.ws_bytes = 0;
-            if (cudaMalloc(&d.ws, need) != cudaSuccess) return PKV_ERR_CUDA;
-            if (cudaMemset(d.ws, 0, need) != cudaSuccess) return PKV_ERR_CUDA;  // merge counters start at 0
-            d.ws_bytes = need;
+        StreamWorkspace* d = nullptr;
+        for (StreamWorkspace& e : g_stream_ws)
+            if (e.dev == dev && e.stream == st) d = &e;
+        if (d == nullptr) {
+            g_stream_ws.push_back(StreamWorkspace{dev, st, nullptr, 0});
+            d = &g_stream_ws.back();
         }
-        ws = d.ws;
+        if (d->bytes < need) {
+            // grow on the call's stream: calls on it are ordered, so the old
+            // buffer is released only after the launches that read it
+            cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+            if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return PKV_ERR_CUDA;
+            if (cap != cudaStreamCaptureStatusNone) return PKV_ERR_WORKSPACE;
+            size_t grow = need + need / 4;
+            void* fresh = nullptr;
+            if (cudaMallocAsync(&fresh, grow, st) != cudaSuccess) return PKV_ERR_CUDA;
+            if (cudaMemsetAsync(fresh, 0, grow, st) != cudaSuccess) return PKV_ERR_CUDA;  // counters start at 0
+            if (d->ptr != nullptr && cudaFreeAsync(d->ptr, st) != cudaSuccess) return PKV_ERR_CUDA;
+            d->ptr = fresh;
+            d->bytes = grow;
+        }
+        ws = d->ptr;
     }
     return paged_attention_decode_ex(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs,
                                      num_heads, num_kv_heads, head_dim, block_size,
@@ -573,6 +637,29 @@ int pkv_selftest_bounded_wait(int timeout_us, void* stream) {
     return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
+int pkv_debug_build(void) {
+#ifdef PKV_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+int pkv_debug_failed_line(void* stream, int* line) {
+    if (!line) return PKV_ERR_NULL;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PKV_ERR_CUDA;
+    int dev = 0;
+    if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
+    int* err = nullptr;
+    if (error_word(dev, &err) != PKV_OK) return PKV_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, err + 1, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return PKV_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpy(err + 1, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return PKV_ERR_CUDA;
+    *line = v;
+    return PKV_OK;
+}
+
 int pkv_get_device_error(void* stream, int* code) {
     if (!code) return PKV_ERR_NULL;
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PKV_ERR_CUDA;
@@ -640,6 +727,17 @@ int pkv_profile_reset(void) {
 }
 
 unsigned long long pkv_launch_count(void) { return g_launches.load(); }
+
+int pkv_set_wait_limit_us(int microseconds) {
+    if (microseconds < 0 || microseconds > 1000000) return PKV_ERR_INVALID;
+    const unsigned long long ns =
+        microseconds == 0 ? pkv::kWaitTimeoutNs : 1000ull * (unsigned long long)microseconds;
+    return (int)(g_wait_ns.exchange(ns) / 1000ull);
+}
+
+int pkv_set_longest_first(int enable) {
+    return g_longest_first.exchange(enable != 0 ? 1 : 0);
+}
 
 int pkv_set_tensor_core_gqa(int enable) {
     return g_tc_gqa.exchange(enable != 0 ? 1 : 0);

@@ -22,6 +22,25 @@ __device__ __forceinline__ void set_error(int* err, int code) {
     if (err != nullptr) atomicCAS(err, 0, code);
 }
 
+// Debug builds (-DPKV_DEBUG) check every index derived from the inputs
+// (schedule entries, units, copy sources and destinations, workspace and
+// output rows) right before its use: a failed check records
+// PKV_ERR_DEVICE_BOUNDS in err[0] and the source line in err[1] (the first
+// failure wins), and the caller skips the access, so the build reports a
+// bad index where a release build would read or write out of bounds.  In
+// release builds PKV_DCHECK is the constant true and compiles away.
+#ifdef PKV_DEBUG
+static __device__ __noinline__ void debug_fail(int* err, int line) {
+    if (err != nullptr) {
+        atomicCAS(err, 0, PKV_ERR_DEVICE_BOUNDS);
+        atomicCAS(err + 1, 0, line);
+    }
+}
+#define PKV_DCHECK(err, cond) ((cond) ? true : (::pkv::debug_fail((err), __LINE__), false))
+#else
+#define PKV_DCHECK(err, cond) true
+#endif
+
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -96,6 +115,22 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, u
             "r"(smem_addr(dst_smem)),
         "l"(src_gmem), "r"(bytes), "r"(smem_addr(bar))
         : "memory");
+}
+
+// ------------------------------------------ 16-byte async copies (LDGSTS)
+// One 16-byte global -> shared copy that bypasses L1 (both addresses 16-byte
+// aligned).  Completion is tracked per thread: see cp_async_arrive_noinc.
+__device__ __forceinline__ void cp_async16(void* dst_smem, const void* src_gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst_smem)),
+                 "l"(src_gmem)
+                 : "memory");
+}
+
+// Arrive on `bar` once every cp.async this thread issued so far has landed.
+// The arrival counts toward the barrier's expected count (set at init).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
 }
 
 // ------------------------------------------------------- element types

@@ -135,10 +135,9 @@ __global__ void __launch_bounds__(DecodeCfg<T, TKV, D, BS, G>::THREADS,
 
     const int P = p.num_partitions;
     const int Hkv = p.num_kv_heads;
-    const long long bid = blockIdx.x;
-    const int part = (int)(bid % P);
-    const int g = (int)((bid / P) % Hkv);
-    const int s = (int)(bid / ((long long)P * Hkv));
+    const Unit unit = decode_unit(p, false);
+    if (unit.s < 0) return;  // a schedule entry out of range (debug builds)
+    const int part = unit.part, g = unit.g, s = unit.s;
     const int ctx = p.context_lens[s];
     const int max_ctx = p.max_blocks_per_seq * BS;
 
@@ -174,7 +173,9 @@ __global__ void __launch_bounds__(DecodeCfg<T, TKV, D, BS, G>::THREADS,
 
     if (tid == 0) {
         for (int i = 0; i < C::NST; ++i) {
-            mbar_init(&full[i], 1);
+            // stages of small blocks complete when every producer lane's
+            // 16-byte copies have landed; larger ones on the bulk copies' bytes
+            mbar_init(&full[i], BS >= C::ST ? 1 : 32);
             mbar_init(&empty[i], C::NHS);
         }
         *abort_flag = 0;
@@ -213,6 +214,8 @@ __global__ void __launch_bounds__(DecodeCfg<T, TKV, D, BS, G>::THREADS,
         // ------------------------------------------------------ producer
         const char* kbase = static_cast<const char*>(p.k_cache);
         const char* vbase = static_cast<const char*>(p.v_cache);
+        const long long pool_bytes = (long long)p.num_blocks * Hkv * C::SLICE;  // debug checks
+        (void)pool_bytes;
         if constexpr (BS >= C::ST) {
             // One lane issues every copy (16 rows of one block, the whole
             // block when bs = 16): spreading two copies over the warp measured
@@ -221,7 +224,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, TKV, D, BS, G>::THREADS,
                 for (int j = 0; j < nstg; ++j) {
                     const int st = j % C::NST;
                     if (j >= C::NST) {
-                        if (!mbar_wait_bounded(&empty[st], ((j / C::NST) - 1) & 1, abort_flag)) {
+                        if (!mbar_wait_bounded(&empty[st], ((j / C::NST) - 1) & 1, abort_flag, p.wait_ns)) {
                             set_error(p.err, PKV_ERR_TIMEOUT);
                             *abort_flag = 1;
                             break;
@@ -229,9 +232,9 @@ __global__ void __launch_bounds__(DecodeCfg<T, TKV, D, BS, G>::THREADS,
                     }
                     unsigned char* dst = stages + st * C::STAGE;
                     const int e = phys[j * C::ST / BS];
-                    if (e >= 0) {
-                        const long long off =
-                            (((long long)e * Hkv + g) * BS + (j * C::ST) % BS) * C::ROWB;
+                    const long long off =
+                        (((long long)e * Hkv + g) * BS + (j * C::ST) % BS) * C::ROWB;
+                    if (e >= 0 && PKV_DCHECK(p.err, off + C::STAGE_K <= pool_bytes && st < C::NST)) {
                         mbar_arrive_expect_tx(&full[st], 2 * C::STAGE_K);
                         bulk_g2s(dst, kbase + off, C::STAGE_K, &full[st]);
                         bulk_g2s(dst + C::STAGE_K, vbase + off, C::STAGE_K, &full[st]);
@@ -242,15 +245,23 @@ __global__ void __launch_bounds__(DecodeCfg<T, TKV, D, BS, G>::THREADS,
                 }
             }
         } else {
-            // Whole blocks stacked row after row, several per stage: lane 0
-            // waits for the slot and registers the byte count, then lane 2b
-            // copies block b's K slice and lane 2b+1 its V slice, so the
-            // stage's copies issue side by side.
+            // Whole blocks stacked row after row, several per stage (blocks
+            // of 2 KB or less).  Bulk copies this small are paced by their
+            // count, not their bytes, so the whole warp moves them with
+            // 16-byte async copies instead: consecutive lanes take
+            // consecutive 16-byte pieces of a block's K slice, then its V
+            // slice, so each warp instruction reads 512 contiguous bytes.
+            // Every lane then arrives on the stage's barrier when its own
+            // copies have landed (32 arrivals complete the stage).
+            constexpr int PIECES = C::SLICE / 16;           // 16-byte pieces of one slice
+            constexpr int PER_LANE = 2 * C::BPS * PIECES / 32;
+            static_assert((2 * C::BPS * PIECES) % 32 == 0 && PIECES % 32 == 0,
+                          "a warp instruction stays inside one slice");
             for (int j = 0; j < nstg; ++j) {
                 const int st = j % C::NST;
                 bool ready = true;
                 if (lane == 0 && j >= C::NST)
-                    ready = mbar_wait_bounded(&empty[st], ((j / C::NST) - 1) & 1, abort_flag);
+                    ready = mbar_wait_bounded(&empty[st], ((j / C::NST) - 1) & 1, abort_flag, p.wait_ns);
                 if (!__shfl_sync(0xffffffffu, ready, 0)) {
                     if (lane == 0) {
                         set_error(p.err, PKV_ERR_TIMEOUT);
@@ -258,22 +269,26 @@ __global__ void __launch_bounds__(DecodeCfg<T, TKV, D, BS, G>::THREADS,
                     }
                     break;
                 }
-                const int b = lane >> 1;
-                const int jb = j * C::BPS + b;
-                const int e = (lane < 2 * C::BPS && jb < nblk) ? phys[jb] : -1;
-                const int nload = __popc(__ballot_sync(0xffffffffu, e >= 0));
-                if (lane == 0) {
-                    if (nload > 0)
-                        mbar_arrive_expect_tx(&full[st], (uint32_t)(nload * C::SLICE));
-                    else
-                        mbar_arrive(&full[st]);
+                int e[C::BPS];
+#pragma unroll
+                for (int b = 0; b < C::BPS; ++b) {
+                    const int jb = j * C::BPS + b;
+                    e[b] = jb < nblk ? phys[jb] : -1;
                 }
-                __syncwarp();  // the byte count is registered before any copy lands
-                if (e >= 0) {
-                    const long long off = ((long long)e * Hkv + g) * C::SLICE;
-                    unsigned char* dst = stages + st * C::STAGE + (lane & 1) * C::STAGE_K + b * C::SLICE;
-                    bulk_g2s(dst, ((lane & 1) ? vbase : kbase) + off, C::SLICE, &full[st]);
+                unsigned char* dst = stages + st * C::STAGE;
+#pragma unroll
+                for (int i = 0; i < PER_LANE; ++i) {
+                    const int c = i * 32 + lane;                 // piece of the stage
+                    const int kv = c / (C::BPS * PIECES);        // 0: K rows, 1: V rows
+                    const int b = (c / PIECES) % C::BPS;         // block within the stage
+                    const int piece = c % PIECES;
+                    const long long off = ((long long)e[b] * Hkv + g) * C::SLICE + piece * 16;
+                    if (e[b] >= 0 && PKV_DCHECK(p.err, off + 16 <= pool_bytes && st < C::NST)) {
+                        cp_async16(dst + kv * C::STAGE_K + b * C::SLICE + piece * 16,
+                                   (kv ? vbase : kbase) + off);
+                    }
                 }
+                cp_async_arrive_noinc(&full[st]);
                 issued = j + 1;
             }
         }
@@ -301,7 +316,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, TKV, D, BS, G>::THREADS,
         for (int j = bl; j < nstg; j += C::NBL) {
             const int st = j % C::NST;
             // every lane waits (bounded); the warp leaves together if any lane gave up
-            const bool ready = mbar_wait_bounded(&full[st], (j / C::NST) & 1, abort_flag);
+            const bool ready = mbar_wait_bounded(&full[st], (j / C::NST) & 1, abort_flag, p.wait_ns);
             if (!__all_sync(0xffffffffu, ready)) {
                 if (lane == 0) {
                     set_error(p.err, PKV_ERR_TIMEOUT);
@@ -445,6 +460,8 @@ __global__ void __launch_bounds__(DecodeCfg<T, TKV, D, BS, G>::THREADS,
                 }
             }
         }
+        __syncthreads();
+        abort_merge_turn<T, D, G>(p, s, g, part, nparts, reinterpret_cast<int*>(smem + C::FLAG_OFF) + 1);
         return;
     }
 
@@ -484,6 +501,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, TKV, D, BS, G>::THREADS,
         }
         O *= vsc;
         const long long sh = sh0 + hg;
+        if (!PKV_DCHECK(p.err, sh < (long long)p.num_seqs * H && part < P)) continue;
         if (nparts == 1) {
             Elem<T>::store(static_cast<T*>(p.out) + sh * D + d, L > 0.f ? O / L : 0.f);
         } else {

@@ -6,6 +6,8 @@
 
 #include <math.h>
 
+#include <utility>
+
 #include "common.cuh"
 
 namespace pkv {
@@ -20,6 +22,9 @@ struct DecodeParams {
     float* ws_o;    // [B][H][P][D] unnormalised partial outputs
     float2* ws_ml;  // [B][H][P] (running max in log2 units, running sum)
     int* counters;  // [B][Hkv] partitions finished, zero between launches
+    // longest-first schedule written by plan_kernel just before this launch
+    // ([B * P] entries s * P + part), or null for index order
+    const int* order;
     const float* k_scales;  // fp8 caches: per-kv-head dequantisation scales (else null)
     const float* v_scales;
     int* err;
@@ -31,7 +36,67 @@ struct DecodeParams {
     int partition_tokens;
     int num_partitions;  // partitions per sequence in the grid
     float qscale;        // scale * log2(e)
+    // limit of the pipeline's bounded waits (ns of %globaltimer); the drain
+    // after an abort always waits up to kWaitTimeoutNs
+    unsigned long long wait_ns;
 };
+
+// Launch a decode kernel.  When the launch follows a planning grid
+// (p.order set), it is a programmatic dependent launch: its CTAs may start
+// while the plan still runs and wait for it in decode_unit.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_decode_kernel(void (*kern)(KArgs...), unsigned grid, unsigned threads,
+                                        size_t smem, cudaStream_t st, bool after_plan,
+                                        Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = after_plan ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// Which (sequence, kv head, partition) this CTA runs.  With a schedule
+// (p.order) the CTA first waits for the planning grid that wrote it (a no-op
+// without one in flight), then takes pair order[b / Hkv] and kv head
+// b % Hkv.  Without one: partition fastest, or, when `partition_major` (the
+// tensor-core kernels with at most 4 partitions per sequence), all first
+// partitions, then all second ones, and so on.
+struct Unit {
+    int s, g, part;
+};
+
+__device__ __forceinline__ Unit decode_unit(const DecodeParams& p, bool partition_major) {
+    const int P = p.num_partitions;
+    const int Hkv = p.num_kv_heads;
+    const long long bid = blockIdx.x;
+    Unit u;
+    if (p.order != nullptr) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        const int pair = p.order[bid / Hkv];
+        u.g = (int)(bid % Hkv);
+        u.s = pair / P;
+        u.part = pair % P;
+    } else if (partition_major) {
+        const long long units = (long long)p.num_seqs * Hkv;
+        u.part = (int)(bid / units);
+        u.g = (int)((bid % units) % Hkv);
+        u.s = (int)((bid % units) / Hkv);
+    } else {
+        u.part = (int)(bid % P);
+        u.g = (int)((bid / P) % Hkv);
+        u.s = (int)(bid / ((long long)P * Hkv));
+    }
+    if (!PKV_DCHECK(p.err, u.s >= 0 && u.s < p.num_seqs && u.g >= 0 && u.g < Hkv && u.part >= 0 &&
+                               u.part < P))
+        u.s = -1;  // the CTA exits
+    return u;
+}
 
 // Split-K merge, fused into the decode kernels: called by every thread of a
 // partition CTA after the CTA wrote its (m, l, o) for the group's G heads to
@@ -56,10 +121,14 @@ __device__ __forceinline__ void fused_merge(const DecodeParams& p, int s, int g,
     __threadfence();
     __syncthreads();
     if (tid == 0) {
-        const unsigned old = atomicInc(
-            reinterpret_cast<unsigned*>(p.counters) + (long long)s * p.num_kv_heads + g,
-            (unsigned)(nparts - 1));
-        *last_flag = old == (unsigned)(nparts - 1);
+        *last_flag = 0;
+        if (PKV_DCHECK(p.err, nparts <= P && (long long)s * p.num_kv_heads + g <
+                                                 (long long)p.num_seqs * p.num_kv_heads)) {
+            const unsigned old = atomicInc(
+                reinterpret_cast<unsigned*>(p.counters) + (long long)s * p.num_kv_heads + g,
+                (unsigned)(nparts - 1));
+            *last_flag = old == (unsigned)(nparts - 1);
+        }
     }
     __syncthreads();
     if (!*last_flag) return;
@@ -129,6 +198,7 @@ __device__ __forceinline__ void fused_merge(const DecodeParams& p, int s, int g,
         }
         const float L = red[2 * hg + 1];
         const float inv = L > 0.f ? 1.f / L : 0.f;
+        if (!PKV_DCHECK(p.err, sh0 + hg < (long long)p.num_seqs * p.num_heads)) continue;
         T* dst = static_cast<T*>(p.out) + (sh0 + hg) * D + col * 4;
         Elem<T>::store(dst + 0, t.x * inv);
         Elem<T>::store(dst + 1, t.y * inv);
@@ -141,6 +211,40 @@ template <typename T, int D, int G>
 __device__ __forceinline__ void zero_rows(const DecodeParams& p, int s, int g) {
     T* out = static_cast<T*>(p.out) + ((long long)s * p.num_heads + (long long)g * G) * D;
     for (int i = threadIdx.x; i < G * D; i += blockDim.x) Elem<T>::store(out + i, 0.f);
+}
+
+// The end of a partition CTA whose bounded wait ran out (called by every
+// thread, after the CTA's own copies and MMAs have landed).  It still takes
+// its one turn on the (s, g) merge counter, so the counter wraps back to zero
+// exactly as on a complete launch and the workspace stays valid for later
+// calls: it posts an empty partial (m = -inf, l = 0, o = 0), which the merge
+// weighs by zero, and if it arrives last it writes zero rows instead of
+// merging.  A sequence with one partition has no counter; its rows are
+// zeroed.  The outputs of a launch that timed out are not meaningful, but
+// they are finite and the error word says PKV_ERR_TIMEOUT.
+template <typename T, int D, int G>
+__device__ __forceinline__ void abort_merge_turn(const DecodeParams& p, int s, int g, int part,
+                                                 int nparts, int* last_flag) {
+    if (nparts == 1) {
+        zero_rows<T, D, G>(p, s, g);
+        return;
+    }
+    const int P = p.num_partitions;
+    const long long sh0 = (long long)s * p.num_heads + (long long)g * G;
+    if (!PKV_DCHECK(p.err, part < P && sh0 + G <= (long long)p.num_seqs * p.num_heads)) return;
+    for (int i = threadIdx.x; i < G * D; i += blockDim.x)
+        p.ws_o[((sh0 + i / D) * P + part) * D + i % D] = 0.f;
+    if (threadIdx.x < G) p.ws_ml[(sh0 + threadIdx.x) * P + part] = make_float2(-INFINITY, 0.f);
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const unsigned old = atomicInc(
+            reinterpret_cast<unsigned*>(p.counters) + (long long)s * p.num_kv_heads + g,
+            (unsigned)(nparts - 1));
+        *last_flag = old == (unsigned)(nparts - 1);
+    }
+    __syncthreads();
+    if (*last_flag) zero_rows<T, D, G>(p, s, g);
 }
 
 }  // namespace pkv

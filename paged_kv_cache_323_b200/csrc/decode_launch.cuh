@@ -25,8 +25,8 @@ cudaError_t launch_partition_inst(const DecodeParams& p, long long grid, cudaStr
         if (e != cudaSuccess) return e;
         configured.fetch_or(bit);
     }
-    kern<<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, st>>>(p);
-    return cudaGetLastError();
+    return launch_decode_kernel(kern, static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, st,
+                                p.order != nullptr, p);
 }
 
 template <typename T, typename TKV, int D, int BS>

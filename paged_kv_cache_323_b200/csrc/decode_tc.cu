@@ -66,8 +66,8 @@ cudaError_t launch_inst(const DecodeParams& p, const CUtensorMap& mk, const CUte
         if (e != cudaSuccess) return e;
         configured.fetch_or(bit);
     }
-    kern<<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, st>>>(p, mk, mv);
-    return cudaGetLastError();
+    return launch_decode_kernel(kern, static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, st,
+                                p.order != nullptr, p, mk, mv);
 }
 
 template <int BS>

@@ -206,26 +206,15 @@ __global__ void __launch_bounds__(192, 2)
     unsigned char* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
 
     const int P = p.num_partitions;
-    const int Hkv = p.num_kv_heads;
-    const long long bid = blockIdx.x;
-    // Launch order.  With a few partitions per sequence (the grid is sized
-    // for the longest, so many CTAs lie past a shorter sequence's end)
-    // partition-major: all first partitions, then all second ones, and so on,
-    // so the CTAs that exit at once come last instead of taking SM slots
-    // between real work.  With many (long contexts) partition-fastest, so that
-    // a unit's partitions finish together and its merge is not left for the
-    // last wave.
-    int part, g, s;
-    if (P <= 4) {
-        const long long units = (long long)p.num_seqs * Hkv;
-        part = (int)(bid / units);
-        g = (int)((bid % units) % Hkv);
-        s = (int)((bid % units) / Hkv);
-    } else {
-        part = (int)(bid % P);
-        g = (int)((bid / P) % Hkv);
-        s = (int)(bid / ((long long)P * Hkv));
-    }
+    // Launch order: the longest-first schedule when there is one.  Without
+    // it, with a few partitions per sequence (the grid is sized for the
+    // longest, so many CTAs lie past a shorter sequence's end)
+    // partition-major, so the CTAs that exit at once come last instead of
+    // taking SM slots between real work; with many (long contexts)
+    // partition-fastest, so that a unit's partitions finish together.
+    const Unit unit = decode_unit(p, P <= 4);
+    if (unit.s < 0) return;  // a schedule entry out of range (debug builds)
+    const int part = unit.part, g = unit.g, s = unit.s;
     const int ctx = p.context_lens[s];
     const int max_ctx = p.max_blocks_per_seq * BS;
     if (ctx < 0 || ctx > max_ctx) {
@@ -343,7 +332,7 @@ __global__ void __launch_bounds__(192, 2)
             const CUtensorMap* map = (li & 1) ? &tmv : &tmk;
             const int st = li % C::NSLOT;
             if (li >= C::NSLOT) {
-                const bool ready = mbar_wait_bounded(&empty[st], ((li / C::NSLOT) - 1) & 1, abort_flag);
+                const bool ready = mbar_wait_bounded(&empty[st], ((li / C::NSLOT) - 1) & 1, abort_flag, p.wait_ns);
                 if (!__all_sync(0xffffffffu, ready)) {
                     if (lane == 0) {
                         set_error(p.err, PKV_ERR_TIMEOUT);
@@ -355,7 +344,10 @@ __global__ void __launch_bounds__(192, 2)
             const int jb0 = c * C::BPT;
             const int j = jb0 + lane;
             const int e = (lane < C::BPT && j < nblk) ? phys[j] : -1;
-            const int nload = __popc(__ballot_sync(0xffffffffu, e >= 0));
+            const bool load = e >= 0 && PKV_DCHECK(p.err, e < p.num_blocks && g < p.num_kv_heads &&
+                                                              st < C::NSLOT &&
+                                                              (lane + 1) * BS * C::ROW <= C::HALF);
+            const int nload = __popc(__ballot_sync(0xffffffffu, load));
             if (lane == 0) {
                 if (nload > 0)
                     mbar_arrive_expect_tx(&full[st], (uint32_t)(nload * BS * 2 * C::ROW));
@@ -363,7 +355,7 @@ __global__ void __launch_bounds__(192, 2)
                     mbar_arrive(&full[st]);
             }
             __syncwarp();  // the expected byte count is registered before any copy lands
-            if (e >= 0) {
+            if (load) {
                 unsigned char* dst = smem + st * C::SLOT + lane * BS * C::ROW;
                 tma_load_4d(dst, map, 0, 0, g, e, &full[st]);
                 tma_load_4d(dst + C::HALF, map, 64, 0, g, e, &full[st]);
@@ -375,7 +367,7 @@ __global__ void __launch_bounds__(192, 2)
         if (lane == 0) {
             const uint32_t q_base = smem_addr(smem + C::Q_OFF);
             auto wait_or_abort = [&](uint64_t* bar, uint32_t parity) -> bool {
-                if (mbar_wait_bounded(bar, parity, abort_flag)) return true;
+                if (mbar_wait_bounded(bar, parity, abort_flag, p.wait_ns)) return true;
                 set_error(p.err, PKV_ERR_TIMEOUT);
                 *abort_flag = 1;
                 return false;
@@ -429,7 +421,7 @@ __global__ void __launch_bounds__(192, 2)
         const int r = q4 * 32 + lane;       // token row of S, dimension row of O
         const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
         auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
-            const bool ok = mbar_wait_bounded(bar, parity, abort_flag);
+            const bool ok = mbar_wait_bounded(bar, parity, abort_flag, p.wait_ns);
             if (__all_sync(0xffffffffu, ok)) return true;
             if (lane == 0) {
                 set_error(p.err, PKV_ERR_TIMEOUT);
@@ -543,6 +535,7 @@ __global__ void __launch_bounds__(192, 2)
                 const long long sh0 = (long long)s * H + (long long)g * G;
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
+                    if (!PKV_DCHECK(p.err, sh0 + h < (long long)p.num_seqs * H && part < P)) continue;
                     const float L = (red_sum[h] + red_sum[C::NPAD + h]) +
                                     (red_sum[2 * C::NPAD + h] + red_sum[3 * C::NPAD + h]);
                     if (nparts == 1) {
@@ -578,6 +571,7 @@ __global__ void __launch_bounds__(192, 2)
         __syncthreads();
         tc_fence_after();
         if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+        abort_merge_turn<T, D, G>(p, s, g, part, nparts, last_flag);
         return;
     }
     tc_fence_after();

@@ -233,26 +233,15 @@ __global__ void __launch_bounds__(192, TcFp8Cfg<BS, G>::CTAS_PER_SM)
     unsigned char* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
 
     const int P = p.num_partitions;
-    const int Hkv = p.num_kv_heads;
-    const long long bid = blockIdx.x;
-    // Launch order.  With a few partitions per sequence (the grid is sized
-    // for the longest, so many CTAs lie past a shorter sequence's end)
-    // partition-major: all first partitions, then all second ones, and so on,
-    // so the CTAs that exit at once come last instead of taking SM slots
-    // between real work.  With many (long contexts) partition-fastest, so that
-    // a unit's partitions finish together and its merge is not left for the
-    // last wave.
-    int part, g, s;
-    if (P <= 4) {
-        const long long units = (long long)p.num_seqs * Hkv;
-        part = (int)(bid / units);
-        g = (int)((bid % units) % Hkv);
-        s = (int)((bid % units) / Hkv);
-    } else {
-        part = (int)(bid % P);
-        g = (int)((bid / P) % Hkv);
-        s = (int)(bid / ((long long)P * Hkv));
-    }
+    // Launch order: the longest-first schedule when there is one.  Without
+    // it, with a few partitions per sequence (the grid is sized for the
+    // longest, so many CTAs lie past a shorter sequence's end)
+    // partition-major, so the CTAs that exit at once come last instead of
+    // taking SM slots between real work; with many (long contexts)
+    // partition-fastest, so that a unit's partitions finish together.
+    const Unit unit = decode_unit(p, P <= 4);
+    if (unit.s < 0) return;  // a schedule entry out of range (debug builds)
+    const int part = unit.part, g = unit.g, s = unit.s;
     const int ctx = p.context_lens[s];
     const int max_ctx = p.max_blocks_per_seq * BS;
     if (ctx < 0 || ctx > max_ctx) {
@@ -382,7 +371,7 @@ __global__ void __launch_bounds__(192, TcFp8Cfg<BS, G>::CTAS_PER_SM)
 
     // a bounded wait taken by a whole warp; the warp leaves together if any lane gave up
     auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
-        const bool ok = mbar_wait_bounded(bar, parity, abort_flag);
+        const bool ok = mbar_wait_bounded(bar, parity, abort_flag, p.wait_ns);
         if (__all_sync(0xffffffffu, ok)) return true;
         if (lane == 0) {
             set_error(p.err, PKV_ERR_TIMEOUT);
@@ -403,7 +392,10 @@ __global__ void __launch_bounds__(192, TcFp8Cfg<BS, G>::CTAS_PER_SM)
             if (li >= C::NSLOT && !wait_all(&empty[st], ((li / C::NSLOT) - 1) & 1)) break;
             const int j = c * C::BPT + lane;
             const int e = (lane < C::BPT && j < nblk) ? phys[j] : -1;
-            const int nload = __popc(__ballot_sync(0xffffffffu, e >= 0));
+            const bool load = e >= 0 && PKV_DCHECK(p.err, e < p.num_blocks && g < p.num_kv_heads &&
+                                                              st < C::NSLOT &&
+                                                              (lane + 1) * BS * C::ROW <= C::SLOT);
+            const int nload = __popc(__ballot_sync(0xffffffffu, load));
             if (lane == 0) {
                 if (nload > 0)
                     mbar_arrive_expect_tx(&full[st], (uint32_t)(nload * BS * C::ROW));
@@ -411,7 +403,7 @@ __global__ void __launch_bounds__(192, TcFp8Cfg<BS, G>::CTAS_PER_SM)
                     mbar_arrive(&full[st]);
             }
             __syncwarp();  // the expected byte count is registered before any copy lands
-            if (e >= 0) tma_load_4d(smem + st * C::SLOT + lane * BS * C::ROW, map, 0, 0, g, e, &full[st]);
+            if (load) tma_load_4d(smem + st * C::SLOT + lane * BS * C::ROW, map, 0, 0, g, e, &full[st]);
             issued = li + 1;
         }
     } else if (warp == 1) {
@@ -471,7 +463,7 @@ __global__ void __launch_bounds__(192, TcFp8Cfg<BS, G>::CTAS_PER_SM)
                     t_last = globaltimer_ns();
                 } else {
                     if (*abort_flag) break;
-                    if (globaltimer_ns() - t_last > kWaitTimeoutNs) {
+                    if (globaltimer_ns() - t_last > p.wait_ns) {
                         set_error(p.err, PKV_ERR_TIMEOUT);
                         *abort_flag = 1;
                         break;
@@ -607,6 +599,7 @@ __global__ void __launch_bounds__(192, TcFp8Cfg<BS, G>::CTAS_PER_SM)
                 const float vsc = p.v_scales[g] * 0.00390625f;
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
+                    if (!PKV_DCHECK(p.err, sh0 + h < (long long)p.num_seqs * H && part < P)) continue;
                     const float L = (red_sum[h] + red_sum[C::NPAD + h]) +
                                     (red_sum[2 * C::NPAD + h] + red_sum[3 * C::NPAD + h]);
                     const float O = acc[h] * vsc;
@@ -642,6 +635,7 @@ __global__ void __launch_bounds__(192, TcFp8Cfg<BS, G>::CTAS_PER_SM)
         __syncthreads();
         tc_fence_after();
         if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+        abort_merge_turn<T, D, G>(p, s, g, part, nparts, last_flag);
         return;
     }
     tc_fence_after();

@@ -14,18 +14,19 @@
 // exits.  No call here allocates or frees memory.
 //
 // The host never uses the array's name as an address (in host code it is
-// only a stand-in symbol): the device address is looked up once per device
-// with cudaGetSymbolAddress, with that device current, on the first call
-// made on it.  Every call shares the array and it keeps the previous call's
-// contents, so each call clears the merge counters (the only part that must
-// start at zero) with cudaMemsetAsync on its stream before the kernel runs.
+// only a stand-in symbol): every call looks up the device address with
+// cudaGetSymbolAddress, with the caller's device current.  The lookup
+// allocates nothing, and doing it per call keeps the address right if the
+// device is reset and a new context replaces the old one.  Every call shares
+// the array and it keeps the previous call's contents, so each call clears
+// the merge counters (the only part that must start at zero) with
+// cudaMemsetAsync on its stream before the kernel runs.
 // Two calls whose kernels overlap on the GPU -- on different streams, or on
 // different host threads -- race on the array and corrupt each other's
 // results; callers must order them.
 #include <cuda_runtime.h>
 
 #include <climits>
-#include <mutex>
 
 #include "../../include/pagedkv.h"
 
@@ -35,21 +36,16 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[PKV_NOALLOC_SCRATCH_BYTES];
 
-std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices];  // device address of g_noalloc_scratch, per device
-
-// Look up (once per device) the device address of the scratch array.
+// The device address of the scratch array on the current device.
 int scratch_address(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKV_ERR_CUDA;
-    std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (g_scratch_addr[dev] == nullptr) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-            return PKV_ERR_CUDA;
-        g_scratch_addr[dev] = p;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+        cudaGetLastError();
+        return PKV_ERR_CUDA;
     }
-    *out = g_scratch_addr[dev];
+    *out = p;
     return PKV_OK;
 }
 

@@ -14,12 +14,16 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libpagedkv.so")
+# PKV_LIBRARY=debug loads the build whose kernels check every derived index
+# (python -m paged_kv_cache_323_b200.build --debug)
+DEBUG = os.environ.get("PKV_LIBRARY", "") == "debug"
+LIB_PATH = os.path.join(_HERE, "libpagedkv_debug.so" if DEBUG else "libpagedkv.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_323_b200.build` "
-        "(nvcc, sm_100a); the decode path has no other implementation")
+        f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_323_b200.build"
+        f"{' --debug' if DEBUG else ''}` (nvcc, sm_100a); the decode path has no other "
+        "implementation")
 
 lib = ctypes.CDLL(LIB_PATH)
 
@@ -73,12 +77,16 @@ SIGNATURES = {
     "pkv_bm_get_stats": (_I, [_P, _P]),
     "pkv_get_device_error": (_I, [_P, ctypes.POINTER(_I)]),
     "pkv_selftest_bounded_wait": (_I, [_I, _P]),
+    "pkv_set_wait_limit_us": (_I, [_I]),
+    "pkv_debug_build": (_I, []),
+    "pkv_debug_failed_line": (_I, [_P, ctypes.POINTER(_I)]),
     "pkv_status_string": (ctypes.c_char_p, [_I]),
     "pkv_profile_enable": (_I, [_I]),
     "pkv_profile_read": (_I, [_I, ctypes.POINTER(ctypes.c_longlong), ctypes.POINTER(ctypes.c_double)]),
     "pkv_profile_reset": (_I, []),
     "pkv_launch_count": (ctypes.c_ulonglong, []),
     "pkv_set_tensor_core_gqa": (_I, [_I]),
+    "pkv_set_longest_first": (_I, [_I]),
     "pkv_version": (_I, []),
 }
 for _name, (_res, _args) in SIGNATURES.items():
@@ -148,6 +156,32 @@ def _dev(t: torch.Tensor, name: str, dtype=None, *, device=None, shape=None) -> 
     return t.data_ptr()
 
 
+# Split-K workspaces the binding keeps for calls that pass none: one zeroed
+# uint8 buffer per (device index, stream handle), grown when a call needs
+# more.  Each buffer is allocated on its own stream, so torch's allocator
+# reuses the memory of a replaced one only after the work queued on that
+# stream before the replacement.  Calls on one stream are ordered, so
+# sharing the buffer between them is safe; different streams get different
+# buffers.
+_workspaces: dict = {}
+
+
+def _torch_stream(stream_handle: int, dev: torch.device):
+    if stream_handle == torch.cuda.current_stream(dev).cuda_stream:
+        return torch.cuda.current_stream(dev)
+    return torch.cuda.ExternalStream(stream_handle, device=dev)
+
+
+def _workspace_for(need: int, dev: torch.device, stream_handle: int) -> torch.Tensor:
+    key = (dev.index, stream_handle)
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < need:
+        with torch.cuda.stream(_torch_stream(stream_handle, dev)):
+            ws = torch.zeros(need + need // 4, dtype=torch.uint8, device=dev)
+        _workspaces[key] = ws
+    return ws
+
+
 def _tables(block_tables, context_lens, B: int) -> int:
     """max_blocks_per_seq of a [B][max_blocks] table; context_lens must be [B]."""
     if block_tables.dim() != 2 or block_tables.shape[0] != B:
@@ -177,7 +211,8 @@ def paged_attention_decode_ex(out, q, k_cache, v_cache, block_tables, context_le
     """out, q: [B][H][D]; caches: [N][Hkv][bs][D]; block_tables int32 [B][maxb];
     context_lens int32 [B].  ``workspace`` is a zero-initialised uint8 CUDA
     tensor of at least :func:`paged_attention_workspace_size` bytes, reusable
-    across calls (a fresh zeroed one is allocated here when None)."""
+    across calls of any shape; when None, a buffer this module keeps per
+    (device, stream) is used."""
     B, H, D = q.shape
     N, Hkv, bs, D2 = k_cache.shape
     if D2 != D or tuple(out.shape) != (B, H, D) or tuple(v_cache.shape) != tuple(k_cache.shape):
@@ -192,14 +227,15 @@ def paged_attention_decode_ex(out, q, k_cache, v_cache, block_tables, context_le
             _dev(block_tables, "block_tables", torch.int32, device=dev),
             _dev(context_lens, "context_lens", torch.int32, device=dev))
     need = paged_attention_workspace_size(B, H, maxb * bs, D, partition_tokens)
+    st = _stream(stream, dev)
     if workspace is None and need > 0:
-        workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
+        workspace = _workspace_for(need, dev, st)
     ws_ptr = _dev(workspace, "workspace", torch.uint8, device=dev) if workspace is not None else None
     ws_bytes = workspace.numel() if workspace is not None else 0
     with torch.cuda.device(dev):
         rc = lib.paged_attention_decode_ex(*args, B, H, Hkv, D, bs, maxb, float(scale),
                                            int(num_blocks), code, int(partition_tokens), ws_ptr,
-                                           ws_bytes, _stream(stream, dev))
+                                           ws_bytes, st)
     _check(rc, "paged_attention_decode_ex")
 
 
@@ -223,15 +259,15 @@ def paged_attention_decode_fp8(out, q, k_cache, v_cache, k_scales, v_scales, blo
             _dev(block_tables, "block_tables", torch.int32, device=dev),
             _dev(context_lens, "context_lens", torch.int32, device=dev))
     need = paged_attention_workspace_size(B, H, maxb * bs, D, partition_tokens)
+    st = _stream(stream, dev)
     if workspace is None and need > 0:
-        workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
+        workspace = _workspace_for(need, dev, st)
     ws_ptr = _dev(workspace, "workspace", torch.uint8, device=dev) if workspace is not None else None
     ws_bytes = workspace.numel() if workspace is not None else 0
     with torch.cuda.device(dev):
         rc = lib.paged_attention_decode_fp8(*args, B, H, Hkv, D, bs, maxb, float(scale),
                                             N if num_blocks is None else int(num_blocks),
-                                            int(partition_tokens), ws_ptr, ws_bytes,
-                                            _stream(stream, dev))
+                                            int(partition_tokens), ws_ptr, ws_bytes, st)
     _check(rc, "paged_attention_decode_fp8")
 
 
@@ -478,9 +514,25 @@ def get_device_error(stream=None) -> int:
     return code.value
 
 
+def debug_failed_line(stream=None) -> int:
+    """Source line of the first failed index check of a debug build (0: none)."""
+    line = ctypes.c_int(0)
+    _check(lib.pkv_debug_failed_line(_stream(stream), ctypes.byref(line)), "pkv_debug_failed_line")
+    return line.value
+
+
 def selftest_bounded_wait(timeout_us: int, stream=None) -> None:
     """Launch a wait that runs out after timeout_us (see include/pagedkv.h)."""
     _check(lib.pkv_selftest_bounded_wait(int(timeout_us), _stream(stream)), "pkv_selftest_bounded_wait")
+
+
+def set_wait_limit_us(microseconds: int) -> int:
+    """Failure-path test hook: limit of the decode kernels' pipeline waits
+    (0 restores the one-second default); returns the previous limit."""
+    rc = int(lib.pkv_set_wait_limit_us(int(microseconds)))
+    if rc < 0:
+        raise PagedKVError(rc, "pkv_set_wait_limit_us")
+    return rc
 
 
 def profile_enable(on: bool = True) -> None:
@@ -507,3 +559,9 @@ def set_tensor_core_gqa(enable: bool) -> bool:
     where a tensor-core one applies (bf16 caches with grouped query heads,
     fp8 caches); returns the previous setting."""
     return bool(lib.pkv_set_tensor_core_gqa(1 if enable else 0))
+
+
+def set_longest_first(enable: bool) -> bool:
+    """Order the decode grid longest first (True, the default) or by index
+    (False); both give the same bits.  Returns the previous setting."""
+    return bool(lib.pkv_set_longest_first(1 if enable else 0))

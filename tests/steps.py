@@ -66,6 +66,28 @@ def gpu_step(w: wl.Workload, t: dict | None = None, partition_tokens: int = 0,
     return t["out"], t["k_cache"], t["v_cache"]
 
 
+def _fp8_attention(q, kc, vc, w: wl.Workload) -> np.ndarray:
+    """The oracle's fp8 attention over the batch, run as one call per slice of
+    sequences on a pool of host threads (each call is independent and the
+    ctypes call releases the GIL; the arithmetic is the oracle's own)."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
+    B = q.shape[0]
+    nthreads = max(1, min(B, os.cpu_count() or 1))
+    bounds = np.linspace(0, B, nthreads + 1).astype(int)
+
+    def part(i):
+        a, b = bounds[i], bounds[i + 1]
+        if a == b:
+            return np.zeros((0,) + q.shape[1:], dtype=np.float64)
+        return oracle.paged_attention_fp8(q[a:b], kc, vc, w.k_scales, w.v_scales,
+                                          w.block_tables[a:b], w.context_lens[a:b], w.scale)
+
+    with ThreadPoolExecutor(nthreads) as ex:
+        return np.concatenate(list(ex.map(part, range(nthreads))), axis=0)
+
+
 def oracle_step(w: wl.Workload):
     """The same step on host copies; returns (out fp64, k pool, v pool) as numpy."""
     kc = wl.to_numpy_bits(w.k_cache).copy()
@@ -75,8 +97,7 @@ def oracle_step(w: wl.Workload):
     if w.dtype == "fp8":
         oracle.kv_append_fp8(kc, vc, w.k_scales, w.v_scales, wl.to_numpy_bits(w.k_new),
                              wl.to_numpy_bits(w.v_new), w.slot_mapping)
-        out = oracle.paged_attention_fp8(wl.to_numpy_bits(w.q), kc, vc, w.k_scales, w.v_scales,
-                                         w.block_tables, w.context_lens, w.scale)
+        out = _fp8_attention(wl.to_numpy_bits(w.q), kc, vc, w)
         return out, kc, vc
     oracle.kv_append(kc, vc, wl.to_numpy_bits(w.k_new), wl.to_numpy_bits(w.v_new), w.slot_mapping)
     out = oracle.paged_attention(wl.to_numpy_bits(w.q), kc, vc, w.block_tables, w.context_lens,
@@ -108,13 +129,14 @@ def assert_pool_equal(gpu: torch.Tensor, ref: np.ndarray, what: str):
 def subset(w: wl.Workload, seqs, pool_device_k=None, pool_device_v=None) -> wl.Workload:
     """The step restricted to the sequences ``seqs``, on a compact pool that
     holds only the blocks they reference (and copy-on-write sources), taken
-    from the workload's pre-step pool.  Used to check sampled outputs of
-    full-size workloads against the oracle."""
+    from the workload's pre-step pool (``meta["blocks"]`` lists them in pool
+    order).  Used to check full-size workloads against the oracle."""
     seqs = [int(s) for s in seqs]
+    pos = {s: i for i, s in enumerate(seqs)}
     kpool = w.k_cache if pool_device_k is None else pool_device_k
     vpool = w.v_cache if pool_device_v is None else pool_device_v
     bs = w.block_size
-    sel_pairs = [i for i, s in enumerate(w.pair_seq.tolist()) if s in seqs]
+    sel_pairs = [i for i, s in enumerate(w.pair_seq.tolist()) if s in pos]
     blocks = set()
     for s in seqs:
         nb = -(-int(w.context_lens[s]) // bs)
@@ -134,7 +156,7 @@ def subset(w: wl.Workload, seqs, pool_device_k=None, pool_device_v=None) -> wl.W
     for i, s in enumerate(seqs):
         nb = -(-int(w.context_lens[s]) // bs)
         bt[i, :nb] = [remap[int(x)] for x in w.block_tables[s][:nb]]
-    toks = [i for i, s in enumerate(w.token_seq.tolist()) if s in seqs]
+    toks = [i for i, s in enumerate(w.token_seq.tolist()) if s in pos]
     slots = np.asarray([remap[int(w.slot_mapping[i]) // bs] * bs + int(w.slot_mapping[i]) % bs
                         for i in toks], dtype=np.int64)
     tok_idx = torch.tensor(toks, dtype=torch.long)
@@ -146,10 +168,29 @@ def subset(w: wl.Workload, seqs, pool_device_k=None, pool_device_v=None) -> wl.W
         num_kv_heads=w.num_kv_heads, head_dim=w.head_dim, block_size=bs, num_blocks=len(order),
         max_blocks_per_seq=w.max_blocks_per_seq, scale=w.scale,
         context_lens=w.context_lens[seqs].copy(), block_tables=bt, cow_pairs=pairs,
-        slot_mapping=slots, token_seq=np.asarray([seqs.index(int(w.token_seq[i])) for i in toks],
+        slot_mapping=slots, token_seq=np.asarray([pos[int(w.token_seq[i])] for i in toks],
                                                  dtype=np.int32),
-        pair_seq=np.asarray([seqs.index(int(w.pair_seq[i])) for i in sel_pairs], dtype=np.int32),
+        pair_seq=np.asarray([pos[int(w.pair_seq[i])] for i in sel_pairs], dtype=np.int32),
         q=w.q.index_select(0, seq_idx.to(w.q.device)).cpu(), k_cache=k_sub, v_cache=v_sub,
         k_new=w.k_new.index_select(0, tok_idx.to(w.k_new.device)).cpu(),
-        v_new=w.v_new.index_select(0, tok_idx.to(w.v_new.device)).cpu(), meta={},
-        k_scales=w.k_scales, v_scales=w.v_scales)
+        v_new=w.v_new.index_select(0, tok_idx.to(w.v_new.device)).cpu(),
+        meta={"blocks": order}, k_scales=w.k_scales, v_scales=w.v_scales)
+
+
+def full_size_check(w: wl.Workload, partition_tokens: int = 0) -> float:
+    """Every output row of a full-size step, element by element, and every
+    pool block the step reads or writes, byte for byte.  The oracle runs on
+    a compact host copy of the blocks the batch references (all sequences);
+    the GPU runs the whole workload in place."""
+    sub = subset(w, range(w.num_seqs))  # taken before the GPU step changes the pools
+    ref, kref, vref = oracle_step(sub)
+    out, kc, vc = gpu_step(w, partition_tokens=partition_tokens)
+    idx = torch.tensor(sub.meta["blocks"], dtype=torch.long, device=kc.device)
+    if kc.dtype == torch.float8_e4m3fn:
+        k_used = kc.view(torch.uint8).index_select(0, idx).view(torch.float8_e4m3fn)
+        v_used = vc.view(torch.uint8).index_select(0, idx).view(torch.float8_e4m3fn)
+    else:
+        k_used, v_used = kc.index_select(0, idx), vc.index_select(0, idx)
+    assert_pool_equal(k_used, kref, "k pool (referenced blocks)")
+    assert_pool_equal(v_used, vref, "v pool (referenced blocks)")
+    return assert_close(out, ref, "bf16" if w.dtype == "fp8" else w.dtype)

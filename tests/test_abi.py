@@ -86,12 +86,14 @@ def test_decode_validation(pk):
 
 def test_workspace_size(pk):
     ws = pk.paged_attention_workspace_size
-    assert ws(4, 8, 512, 128, 0) == 0  # one partition
-    assert ws(4, 8, 512, 128, 512) == 0
-    n = ws(4, 8, 513, 128, 0)  # two partitions
-    assert n >= 4 * 8 * 2 * (128 + 2) * 4
+    one = ws(4, 8, 512, 128, 0)  # one partition: the merge counters' region and the schedule
+    assert one == ws(4, 8, 512, 128, 512) and one >= 65536 * 4 + 4 * 4
+    n = ws(4, 8, 513, 128, 0)  # two partitions: plus the partial results
+    assert n >= one + 4 * 8 * 2 * (128 + 2) * 4
     assert ws(4, 8, 4096, 128, 256) >= 4 * 8 * 16 * 128 * 4
     assert ws(0, 8, 4096, 128, 0) == 0
+    # the counters' region grows with batches of more than 65536 (sequence, head) units
+    assert ws(1024, 128, 512, 128, 0) >= 1024 * 128 * 4
 
 
 def test_append_and_copy_validation(pk):

@@ -48,7 +48,24 @@ def test_compact_subset_reproduces_rows(make):
 def test_pick_sample_bounds_the_work():
     w = wl.gqa_sampling(groups=4, samples=2, prompt_median=100, prompt_max=200, heads=4,
                         kv_heads=2, head_dim=64)
-    sub, n, dt = bench.pick_sample(w, target_s=0.0, threads=1)  # any work is enough
-    assert n == 1 and len(sub["ctx"]) == 1 and dt >= 0
-    sub, n, _ = bench.pick_sample(w, target_s=1e9, threads=2)  # never enough: every sequence
+    sub, n, dt, out = bench.pick_sample(w, target_s=0.0, threads=1)  # any work is enough
+    assert n == 1 and len(sub["ctx"]) == 1 and dt >= 0 and out.shape[0] == 1
+    sub, n, _, out = bench.pick_sample(w, target_s=1e9, threads=2)  # never enough: every sequence
     assert n == w.num_seqs and len(sub["ctx"]) == w.num_seqs
+    # the rows it returns are the oracle's rows of those sequences in the full step
+    ref, _, _ = oracle_step(w)
+    assert sub["seqs"] == list(range(w.num_seqs)) and np.array_equal(out, ref)
+
+
+def test_rows_match_bar():
+    """The bench's per-row parity verdict applies the spec bars."""
+    import torch
+
+    ref = np.zeros((2, 3, 4))
+    ok = bench.rows_match(torch.full((2, 3, 4), 0.019, dtype=torch.bfloat16), ref, "bf16")
+    assert ok["ok"] and ok["rows"] == 6
+    assert not bench.rows_match(torch.full((2, 3, 4), 0.03), ref, "bf16")["ok"]
+    assert not bench.rows_match(torch.full((2, 3, 4), 2e-5), ref, "f32")["ok"]
+    nan = torch.zeros((2, 3, 4))
+    nan[1, 2, 3] = float("nan")
+    assert not bench.rows_match(nan, ref, "bf16")["ok"]

@@ -13,7 +13,7 @@ import pytest
 import torch
 
 from paged_kv_cache_323_b200 import workload as wl
-from steps import assert_close, assert_pool_equal, gpu_step, oracle_step, subset, to_device
+from steps import assert_close, assert_pool_equal, full_size_check, gpu_step, oracle_step, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -111,12 +111,9 @@ def test_tc_fp8_permutation_bit_identical(tc_mode):
     lambda: wl.gqa_sampling(device="cuda", dtype="fp8"),
     lambda: wl.long_context(device="cuda", dtype="fp8"),
 ], ids=["gqa_sampling", "long_context"])
-def test_tc_fp8_full_size_sampled(tc_mode, make):
-    w = make()
-    seqs = sorted({0, w.num_seqs // 3, w.num_seqs - 1, int(np.argmax(w.context_lens))})
-    ref, _, _ = oracle_step(subset(w, seqs))
-    out, _, _ = gpu_step(w)
-    assert_close(out[torch.tensor(seqs, device=out.device)], ref, "bf16")
+def test_tc_fp8_full_size(tc_mode, make):
+    """Every row of the full-size fp8 workloads (256 x 32, 8 x 64)."""
+    full_size_check(make())
 
 
 @pytest.mark.parametrize("pt", [0, 1024])
