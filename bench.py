@@ -486,12 +486,19 @@ def timed_region(step, steps, world, stream) -> float:
     return max_over_ranks(world, ev0.elapsed_time(ev1))
 
 
+def repeat_count(world: int, first_ms: float, min_s: float, cap: int = 200) -> int:
+    """Repeats of the timed region so that they span at least `min_s`
+    seconds, given the first one took `first_ms`; the same on every rank
+    (the largest any rank needs), since each repeat holds barriers."""
+    reps = int(min(cap, max(1, -(-min_s * 1e3 // max(first_ms, 1e-3)))))
+    return int(max_over_ranks(world, float(reps)))
+
+
 def repeated_regions(step, steps, world, stream, min_s: float):
     """The timed region repeated until the repeats span at least `min_s`
     seconds (every rank runs the same number); returns the ms of each."""
     first = timed_region(step, steps, world, stream)
-    reps = int(min(200, max(1, -(-min_s * 1e3 // max(first, 1e-3)))))
-    reps = int(max_over_ranks(world, float(reps)))
+    reps = repeat_count(world, first, min_s)
     return [first] + [timed_region(step, steps, world, stream) for _ in range(reps - 1)]
 
 

@@ -47,9 +47,14 @@ def _worker(rank, world, port, out_path):
     out, _, _ = oracle_step(w)
     local_ms = 10.0 + rank  # rank 1 is the slower one
     ms = bench.max_over_ranks(world, local_ms)
+    # the timed region's repeat count: every rank runs the same number (the
+    # largest any rank needs), here 0.5 s of 1 ms regions on rank 0 and of
+    # 2 ms regions on rank 1, so 500 capped at 200 on both
+    reps = bench.repeat_count(world, 1.0 + rank, 0.5)
+    reps_small = bench.repeat_count(world, 100.0 * (rank + 1), 0.5)  # 5 on rank 0, 3 on rank 1
     value = bench.job_value(world, w.kv_bytes_logical(), ms)
     gathered = [None] * world
-    dist.all_gather_object(gathered, (seed, float(out.sum()), w.kv_bytes_logical()))
+    dist.all_gather_object(gathered, (seed, float(out.sum()), w.kv_bytes_logical(), reps, reps_small))
     if rank == 0:
         torch.save({"ms": ms, "value": value, "gathered": gathered}, out_path)
     dist.barrier()
@@ -61,8 +66,9 @@ def test_two_gloo_ranks(tmp_path):
     mp.spawn(_worker, args=(2, _free_port(), out_path), nprocs=2, join=True)
     r = torch.load(out_path)
     assert r["ms"] == 11.0  # the slowest rank decides
-    (s0, sum0, b0), (s1, sum1, b1) = r["gathered"]
+    (s0, sum0, b0, n0, m0), (s1, sum1, b1, n1, m1) = r["gathered"]
     assert s0 != s1 and sum0 != sum1  # distinct batches per rank
+    assert n0 == n1 == 200 and m0 == m1 == 5  # ranks agree on the timed regions they run
     assert abs(r["value"] - 2 * b0 / 11e-3 / 1e9) < 1e-9  # weak scaling: world x bytes / max time
 
 
