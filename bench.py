@@ -70,6 +70,12 @@ WORKLOADS = {
                          lambda dev, seed: wl.gqa_sampling(seed=seed, device=dev, dtype="fp8")),
     "long_context_fp8": ("long_context_b8_h64_kv8_d128_bs32_ctxU32768-131072_fp8e4m3_cache",
                          lambda dev, seed: wl.long_context(seed=seed, device=dev, dtype="fp8")),
+    # head_dim 64 over an fp8 cache (the CUDA-core kernel)
+    "mha_d64_fp8": ("mha_decode_b64_h32_kv32_d64_bs16_ctxU128-2048_fp8e4m3_cache",
+                    lambda dev, seed: wl.mha(seed=seed, device=dev, head_dim=64, dtype="fp8")),
+    "mha_d64_fp8_small": ("mha_decode_b16_h32_kv32_d64_bs16_ctxU128-2048_fp8e4m3_cache_pool4096",
+                          lambda dev, seed: wl.mha(seed=seed, device=dev, num_seqs=16, num_blocks=4096,
+                                                   head_dim=64, dtype="fp8")),
     "mha_bs8_small": ("mha_decode_b16_h32_kv32_d128_bs8_ctxU128-2048_bf16_pool8192",
                       lambda dev, seed: wl.mha(seed=seed, device=dev, num_seqs=16, num_blocks=8192,
                                                block_size=8)),
@@ -80,7 +86,8 @@ WORKLOADS = {
 DEFAULT_SEED = {"mha": 2, "gqa_sampling": 3, "long_context": 4, "prefix_bs8": 5, "prefix_bs16": 5,
                 "prefix_bs32": 5, "tiny": 1, "mha_small": 2, "mha_bs8": 2, "mha_bs32": 2,
                 "mha_contig_bs8": 2, "mha_contig_bs16": 2, "mha_contig_bs32": 2, "mha_fp8": 2,
-                "mha_fp8_small": 2, "mha_bs8_small": 2, "gqa_sampling_fp8": 3, "long_context_fp8": 4}
+                "mha_fp8_small": 2, "mha_bs8_small": 2, "gqa_sampling_fp8": 3, "long_context_fp8": 4,
+                "mha_d64_fp8": 2, "mha_d64_fp8_small": 2}
 
 
 def measured_peak():
@@ -623,7 +630,8 @@ def measure_config(pk, key, args, world, rank, stream, peak, flush) -> dict:
 def run_gpu(args, world, rank, local):
     from paged_kv_cache_323_b200 import pagedkv as pk
 
-    pk.set_longest_first(not args.index_order)
+    pk.set_longest_first(args.schedule)
+    pk.set_tensor_core_gqa(not args.cuda_cores)
     name, make = WORKLOADS[args.workload]
     w = make("cuda", rank_seed(args.workload, rank))
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -743,7 +751,9 @@ def run_gpu(args, world, rank, local):
                    "padded_slot_waste": waste_of(w),
                    "partition_tokens": partition_of(pk, w, args.partition_tokens),
                    "accumulate": "f32",
-                   "schedule": "index order" if args.index_order else "longest first",
+                   "schedule": {0: "index order", 1: "longest first where it pays",
+                                2: "longest first"}[args.schedule],
+                   "kernel": "cuda_core" if args.cuda_cores else decode_kernel_family(w),
                    "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush; "
                          "step_us_cold_l2 flushes L2 before each step",
                    "parallelism": f"{world} independent batches, one per GPU"},
@@ -808,8 +818,11 @@ def main():
     ap.add_argument("--workload", default="mha", choices=sorted(WORKLOADS))
     ap.add_argument("--partition-tokens", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--index-order", action="store_true",
-                    help="run the decode grid in index order instead of longest first")
+    ap.add_argument("--cuda-cores", action="store_true",
+                    help="decode on the CUDA-core kernel even where a tensor-core one applies")
+    ap.add_argument("--schedule", type=int, default=1, choices=[0, 1, 2],
+                    help="decode grid schedule: 0 index order, 1 longest first where it pays "
+                         "(default), 2 longest first always")
     ap.add_argument("--min-region-s", type=float, default=0.5,
                     help="repeat the timed region of K steps until the repeats span this long")
     ap.add_argument("--no-configs", action="store_true",

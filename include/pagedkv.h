@@ -133,12 +133,13 @@ PKV_API int paged_attention_decode(void* out, const void* q, const void* k_cache
  *                     one split-K merge counter per (sequence, kv head) at its
  *                     start, in a region nothing else uses, then the launch's
  *                     schedule, then the partial results of split sequences.
- *                     The schedule orders the grid's (sequence, partition)
- *                     units longest first, written by a one-CTA planning
- *                     kernel that the decode kernel follows as a programmatic
- *                     dependent launch; it changes which SM runs a unit and
- *                     when, never the arithmetic, so outputs are the same bits
- *                     with or without it.  Zero-fill the workspace (e.g.
+ *                     The schedule, where one is planned (see
+ *                     pkv_set_longest_first), orders the grid's (sequence,
+ *                     partition) units longest first; a one-CTA planning
+ *                     kernel writes it and the decode kernel follows as a
+ *                     programmatic dependent launch.  It changes which SM runs
+ *                     a unit and when, never the arithmetic, so outputs are
+ *                     the same bits with or without it.  Zero-fill the workspace (e.g.
  *                     cudaMemset) once before its first use.  Every call
  *                     leaves the counters it used at zero again -- a call
  *                     whose kernel stopped on PKV_ERR_TIMEOUT too -- so the
@@ -342,11 +343,14 @@ PKV_API int pkv_profile_reset(void);
  * returns the previous setting.  Process-wide. */
 PKV_API int pkv_set_tensor_core_gqa(int enable);
 
-/* Schedule of the decode grid: 1 (default) orders the (sequence,
- * partition) units longest first whenever the call has a workspace (see
- * paged_attention_decode_ex), 0 runs them in index order.  Both give the same
- * bits; only the time differs.  Process-wide; returns the previous setting. */
-PKV_API int pkv_set_longest_first(int enable);
+/* Schedule of the decode grid (calls with a workspace; see
+ * paged_attention_decode_ex): 1 (default) plans longest first where that
+ * pays -- the tensor-core kernels with 2 to 4 partitions per sequence, whose
+ * index order would leave the partitions only long sequences have for the
+ * end of the launch -- and runs every other launch in index order; 2 plans
+ * every launch; 0 none.  All give the same bits; only the time differs.
+ * Process-wide; returns the previous mode, or PKV_ERR_INVALID. */
+PKV_API int pkv_set_longest_first(int mode);
 
 /* Kernels launched by this library in this process so far (all kinds). */
 PKV_API unsigned long long pkv_launch_count(void);

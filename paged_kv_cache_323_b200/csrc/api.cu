@@ -42,7 +42,9 @@ struct StreamWorkspace {
 std::mutex g_mu;
 std::vector<StreamWorkspace> g_stream_ws;
 std::atomic<int> g_tc_gqa{1};  // tensor-core kernel for grouped-query heads where it applies
-std::atomic<int> g_longest_first{1};  // plan the decode grid longest first when there is a workspace
+// Longest-first schedule of the decode grid: 0 never, 1 where it pays (the
+// tensor-core kernels with 2 to 4 partitions per sequence), 2 always.
+std::atomic<int> g_longest_first{1};
 std::atomic<unsigned long long> g_launches{0};
 std::atomic<unsigned long long> g_wait_ns{pkv::kWaitTimeoutNs};  // decode pipeline wait limit
 
@@ -138,7 +140,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // Decode workspace.  First the split-K merge counters, one int per
 // (sequence, kv head), in a region of at least kFixedCounterSlots slots at
 // offset 0 that nothing else is ever written to; then the longest-first
-// schedule of the launch ([B * P] ints); then, when sequences are split, the
+// schedule of the launch ([B * P] int2); then, when sequences are split, the
 // fp32 partial outputs [B][H][P][D] and the (m, l) pairs [B][H][P]; each
 // region 256-byte aligned.  Every launch, complete or stopped by a timeout,
 // leaves the counters it used at zero, so the first kFixedCounterSlots
@@ -159,7 +161,7 @@ WorkspaceLayout workspace_layout(long long num_seqs, long long num_heads, long l
                                                                       : kFixedCounterSlots;
     w.cnt_off = 0;
     w.plan_off = align256(size_t(slots) * sizeof(int));
-    w.o_off = w.plan_off + align256(size_t(num_seqs) * parts * sizeof(int));
+    w.o_off = w.plan_off + align256(size_t(num_seqs) * parts * sizeof(int2));
     w.ml_off = w.o_off;
     w.total = w.o_off;
     if (parts > 1) {
@@ -306,6 +308,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     const int pt = resolve_partition_tokens(num_seqs, num_heads, num_kv_heads, head_dim,
                                             block_size, max_ctx, kv_dtype, partition_tokens);
     const long long parts = (max_ctx + pt - 1) / pt;
+    const bool use_tc = g_tc_gqa.load() != 0 &&
+                        pkv::decode_tc_supported(kv_dtype, head_dim, block_size, group, pt);
     const long long grid = parts * num_kv_heads * (long long)num_seqs;
     if (grid > INT_MAX || (long long)num_seqs * num_heads > INT_MAX) return PKV_ERR_INVALID;
     const size_t need = workspace_bytes_for(num_seqs, num_heads, parts, head_dim);
@@ -334,9 +338,19 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     p.ws_o = split ? reinterpret_cast<float*>(wsb + wl.o_off) : nullptr;
     p.ws_ml = split ? reinterpret_cast<float2*>(wsb + wl.ml_off) : nullptr;
     p.counters = split ? reinterpret_cast<int*>(wsb + wl.cnt_off) : nullptr;
-    int* order = workspace != nullptr && g_longest_first.load() != 0
-                     ? reinterpret_cast<int*>(wsb + wl.plan_off)
-                     : nullptr;
+    // The schedule pays where index order leaves the longest work for last:
+    // the tensor-core kernels run 2 to 4 partitions per sequence
+    // partition-major, so the later partitions, which only the longest
+    // sequences have, come at the end of the launch (parallel-sampling batch:
+    // 257 -> 250 us bf16, 154 -> 145 us fp8).  Elsewhere it does not: with
+    // one partition per sequence and nearly equal lengths (a shared-prefix
+    // batch) longest first starts the CTAs in synchronised waves that read
+    // the shared blocks in step (+4 %), and the planning kernel itself costs
+    // about 4 us per launch.
+    const int sched = g_longest_first.load();
+    const bool plan = workspace != nullptr &&
+                      (sched == 2 || (sched == 1 && use_tc && parts >= 2 && parts <= 4));
+    int2* order = plan ? reinterpret_cast<int2*>(wsb + wl.plan_off) : nullptr;
     p.order = order;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const long long units = (long long)num_seqs * num_kv_heads;
@@ -359,8 +373,6 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     p.qscale = scale * 1.4426950408889634f;  // log2(e): softmax runs in base 2
     p.wait_ns = g_wait_ns.load();
 
-    const bool use_tc = g_tc_gqa.load() != 0 &&
-                        pkv::decode_tc_supported(kv_dtype, head_dim, block_size, group, pt);
     // the schedule first (one CTA), then the decode grid as its programmatic
     // dependent: counted and profiled together as the decode
     return launch(PKV_KERNEL_DECODE, st, [&] {
@@ -735,8 +747,9 @@ int pkv_set_wait_limit_us(int microseconds) {
     return (int)(g_wait_ns.exchange(ns) / 1000ull);
 }
 
-int pkv_set_longest_first(int enable) {
-    return g_longest_first.exchange(enable != 0 ? 1 : 0);
+int pkv_set_longest_first(int mode) {
+    if (mode < 0 || mode > 2) return PKV_ERR_INVALID;
+    return g_longest_first.exchange(mode);
 }
 
 int pkv_set_tensor_core_gqa(int enable) {

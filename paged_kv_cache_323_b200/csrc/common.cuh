@@ -117,22 +117,6 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, u
         : "memory");
 }
 
-// ------------------------------------------ 16-byte async copies (LDGSTS)
-// One 16-byte global -> shared copy that bypasses L1 (both addresses 16-byte
-// aligned).  Completion is tracked per thread: see cp_async_arrive_noinc.
-__device__ __forceinline__ void cp_async16(void* dst_smem, const void* src_gmem) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst_smem)),
-                 "l"(src_gmem)
-                 : "memory");
-}
-
-// Arrive on `bar` once every cp.async this thread issued so far has landed.
-// The arrival counts toward the barrier's expected count (set at init).
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar))
-                 : "memory");
-}
-
 // ------------------------------------------------------- element types
 template <typename T>
 struct Elem;

@@ -138,20 +138,20 @@ __global__ void __launch_bounds__(DecodeCfg<T, TKV, D, BS, G>::THREADS,
     const Unit unit = decode_unit(p, false);
     if (unit.s < 0) return;  // a schedule entry out of range (debug builds)
     const int part = unit.part, g = unit.g, s = unit.s;
-    const int ctx = p.context_lens[s];
+    const int ctx = unit.ctx;
     const int max_ctx = p.max_blocks_per_seq * BS;
 
     if (ctx < 0 || ctx > max_ctx) {  // not a valid sequence: zero row, report once
         if (part == 0) {
             if (threadIdx.x == 0) set_error(p.err, PKV_ERR_DEVICE_BOUNDS);
-            zero_rows<T, D, G>(p, s, g);
+            zero_rows<T, D, G>(p, (long long)s * p.num_heads + (long long)g * G);
         }
         return;
     }
     const int PT = p.partition_tokens;
     const int nparts = (ctx + PT - 1) / PT;
     if (part >= nparts) {
-        if (ctx == 0 && part == 0) zero_rows<T, D, G>(p, s, g);  // nothing attended
+        if (ctx == 0 && part == 0) zero_rows<T, D, G>(p, (long long)s * p.num_heads + (long long)g * G);  // nothing attended
         return;
     }
     const int tok0 = part * PT;
@@ -173,9 +173,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, TKV, D, BS, G>::THREADS,
 
     if (tid == 0) {
         for (int i = 0; i < C::NST; ++i) {
-            // stages of small blocks complete when every producer lane's
-            // 16-byte copies have landed; larger ones on the bulk copies' bytes
-            mbar_init(&full[i], BS >= C::ST ? 1 : 32);
+            mbar_init(&full[i], 1);
             mbar_init(&empty[i], C::NHS);
         }
         *abort_flag = 0;
@@ -245,18 +243,10 @@ __global__ void __launch_bounds__(DecodeCfg<T, TKV, D, BS, G>::THREADS,
                 }
             }
         } else {
-            // Whole blocks stacked row after row, several per stage (blocks
-            // of 2 KB or less).  Bulk copies this small are paced by their
-            // count, not their bytes, so the whole warp moves them with
-            // 16-byte async copies instead: consecutive lanes take
-            // consecutive 16-byte pieces of a block's K slice, then its V
-            // slice, so each warp instruction reads 512 contiguous bytes.
-            // Every lane then arrives on the stage's barrier when its own
-            // copies have landed (32 arrivals complete the stage).
-            constexpr int PIECES = C::SLICE / 16;           // 16-byte pieces of one slice
-            constexpr int PER_LANE = 2 * C::BPS * PIECES / 32;
-            static_assert((2 * C::BPS * PIECES) % 32 == 0 && PIECES % 32 == 0,
-                          "a warp instruction stays inside one slice");
+            // Whole blocks stacked row after row, several per stage: lane 0
+            // waits for the slot and registers the byte count, then lane 2b
+            // copies block b's K slice and lane 2b+1 its V slice, so the
+            // stage's copies issue side by side.
             for (int j = 0; j < nstg; ++j) {
                 const int st = j % C::NST;
                 bool ready = true;
@@ -269,26 +259,23 @@ __global__ void __launch_bounds__(DecodeCfg<T, TKV, D, BS, G>::THREADS,
                     }
                     break;
                 }
-                int e[C::BPS];
-#pragma unroll
-                for (int b = 0; b < C::BPS; ++b) {
-                    const int jb = j * C::BPS + b;
-                    e[b] = jb < nblk ? phys[jb] : -1;
+                const int b = lane >> 1;
+                const int jb = j * C::BPS + b;
+                const int e = (lane < 2 * C::BPS && jb < nblk) ? phys[jb] : -1;
+                const long long off = ((long long)e * Hkv + g) * C::SLICE;
+                const bool load = e >= 0 && PKV_DCHECK(p.err, off + C::SLICE <= pool_bytes && st < C::NST);
+                const int nload = __popc(__ballot_sync(0xffffffffu, load));
+                if (lane == 0) {
+                    if (nload > 0)
+                        mbar_arrive_expect_tx(&full[st], (uint32_t)(nload * C::SLICE));
+                    else
+                        mbar_arrive(&full[st]);
                 }
-                unsigned char* dst = stages + st * C::STAGE;
-#pragma unroll
-                for (int i = 0; i < PER_LANE; ++i) {
-                    const int c = i * 32 + lane;                 // piece of the stage
-                    const int kv = c / (C::BPS * PIECES);        // 0: K rows, 1: V rows
-                    const int b = (c / PIECES) % C::BPS;         // block within the stage
-                    const int piece = c % PIECES;
-                    const long long off = ((long long)e[b] * Hkv + g) * C::SLICE + piece * 16;
-                    if (e[b] >= 0 && PKV_DCHECK(p.err, off + 16 <= pool_bytes && st < C::NST)) {
-                        cp_async16(dst + kv * C::STAGE_K + b * C::SLICE + piece * 16,
-                                   (kv ? vbase : kbase) + off);
-                    }
+                __syncwarp();  // the byte count is registered before any copy lands
+                if (load) {
+                    unsigned char* dst = stages + st * C::STAGE + (lane & 1) * C::STAGE_K + b * C::SLICE;
+                    bulk_g2s(dst, ((lane & 1) ? vbase : kbase) + off, C::SLICE, &full[st]);
                 }
-                cp_async_arrive_noinc(&full[st]);
                 issued = j + 1;
             }
         }
@@ -461,7 +448,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, TKV, D, BS, G>::THREADS,
             }
         }
         __syncthreads();
-        abort_merge_turn<T, D, G>(p, s, g, part, nparts, reinterpret_cast<int*>(smem + C::FLAG_OFF) + 1);
+        abort_merge_turn<T, D, G>(p, s, g, (long long)s * p.num_heads + (long long)g * G, part, nparts, reinterpret_cast<int*>(smem + C::FLAG_OFF) + 1);
         return;
     }
 

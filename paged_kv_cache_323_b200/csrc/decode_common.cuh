@@ -23,8 +23,9 @@ struct DecodeParams {
     float2* ws_ml;  // [B][H][P] (running max in log2 units, running sum)
     int* counters;  // [B][Hkv] partitions finished, zero between launches
     // longest-first schedule written by plan_kernel just before this launch
-    // ([B * P] entries s * P + part), or null for index order
-    const int* order;
+    // ([B * P] entries {s * P + part, context length of s}), or null for
+    // index order
+    const int2* order;
     const float* k_scales;  // fp8 caches: per-kv-head dequantisation scales (else null)
     const float* v_scales;
     int* err;
@@ -68,7 +69,7 @@ inline cudaError_t launch_decode_kernel(void (*kern)(KArgs...), unsigned grid, u
 // tensor-core kernels with at most 4 partitions per sequence), all first
 // partitions, then all second ones, and so on.
 struct Unit {
-    int s, g, part;
+    int s, g, part, ctx;  // ctx: the sequence's context length
 };
 
 __device__ __forceinline__ Unit decode_unit(const DecodeParams& p, bool partition_major) {
@@ -78,10 +79,11 @@ __device__ __forceinline__ Unit decode_unit(const DecodeParams& p, bool partitio
     Unit u;
     if (p.order != nullptr) {
         asm volatile("griddepcontrol.wait;" ::: "memory");
-        const int pair = p.order[bid / Hkv];
+        const int2 e = p.order[bid / Hkv];
         u.g = (int)(bid % Hkv);
-        u.s = pair / P;
-        u.part = pair % P;
+        u.s = e.x / P;
+        u.part = e.x % P;
+        u.ctx = e.y;
     } else if (partition_major) {
         const long long units = (long long)p.num_seqs * Hkv;
         u.part = (int)(bid / units);
@@ -95,6 +97,8 @@ __device__ __forceinline__ Unit decode_unit(const DecodeParams& p, bool partitio
     if (!PKV_DCHECK(p.err, u.s >= 0 && u.s < p.num_seqs && u.g >= 0 && u.g < Hkv && u.part >= 0 &&
                                u.part < P))
         u.s = -1;  // the CTA exits
+    else if (p.order == nullptr)
+        u.ctx = p.context_lens[u.s];
     return u;
 }
 
@@ -207,9 +211,11 @@ __device__ __forceinline__ void fused_merge(const DecodeParams& p, int s, int g,
     }
 }
 
+// Zero the G output rows of D values from query head row sh0 (= s * H + the
+// CTA's first query head) on.
 template <typename T, int D, int G>
-__device__ __forceinline__ void zero_rows(const DecodeParams& p, int s, int g) {
-    T* out = static_cast<T*>(p.out) + ((long long)s * p.num_heads + (long long)g * G) * D;
+__device__ __forceinline__ void zero_rows(const DecodeParams& p, long long sh0) {
+    T* out = static_cast<T*>(p.out) + sh0 * D;
     for (int i = threadIdx.x; i < G * D; i += blockDim.x) Elem<T>::store(out + i, 0.f);
 }
 
@@ -223,14 +229,13 @@ __device__ __forceinline__ void zero_rows(const DecodeParams& p, int s, int g) {
 // zeroed.  The outputs of a launch that timed out are not meaningful, but
 // they are finite and the error word says PKV_ERR_TIMEOUT.
 template <typename T, int D, int G>
-__device__ __forceinline__ void abort_merge_turn(const DecodeParams& p, int s, int g, int part,
-                                                 int nparts, int* last_flag) {
+__device__ __forceinline__ void abort_merge_turn(const DecodeParams& p, int s, int g, long long sh0,
+                                                 int part, int nparts, int* last_flag) {
     if (nparts == 1) {
-        zero_rows<T, D, G>(p, s, g);
+        zero_rows<T, D, G>(p, sh0);
         return;
     }
     const int P = p.num_partitions;
-    const long long sh0 = (long long)s * p.num_heads + (long long)g * G;
     if (!PKV_DCHECK(p.err, part < P && sh0 + G <= (long long)p.num_seqs * p.num_heads)) return;
     for (int i = threadIdx.x; i < G * D; i += blockDim.x)
         p.ws_o[((sh0 + i / D) * P + part) * D + i % D] = 0.f;
@@ -244,7 +249,7 @@ __device__ __forceinline__ void abort_merge_turn(const DecodeParams& p, int s, i
         *last_flag = old == (unsigned)(nparts - 1);
     }
     __syncthreads();
-    if (*last_flag) zero_rows<T, D, G>(p, s, g);
+    if (*last_flag) zero_rows<T, D, G>(p, sh0);
 }
 
 }  // namespace pkv

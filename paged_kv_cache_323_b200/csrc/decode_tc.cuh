@@ -215,19 +215,19 @@ __global__ void __launch_bounds__(192, 2)
     const Unit unit = decode_unit(p, P <= 4);
     if (unit.s < 0) return;  // a schedule entry out of range (debug builds)
     const int part = unit.part, g = unit.g, s = unit.s;
-    const int ctx = p.context_lens[s];
+    const int ctx = unit.ctx;
     const int max_ctx = p.max_blocks_per_seq * BS;
     if (ctx < 0 || ctx > max_ctx) {
         if (part == 0) {
             if (threadIdx.x == 0) set_error(p.err, PKV_ERR_DEVICE_BOUNDS);
-            zero_rows<T, D, G>(p, s, g);
+            zero_rows<T, D, G>(p, (long long)s * p.num_heads + (long long)g * G);
         }
         return;
     }
     const int PT = p.partition_tokens;
     const int nparts = (ctx + PT - 1) / PT;
     if (part >= nparts) {
-        if (ctx == 0 && part == 0) zero_rows<T, D, G>(p, s, g);
+        if (ctx == 0 && part == 0) zero_rows<T, D, G>(p, (long long)s * p.num_heads + (long long)g * G);
         return;
     }
     const int tok0 = part * PT;
@@ -571,7 +571,7 @@ __global__ void __launch_bounds__(192, 2)
         __syncthreads();
         tc_fence_after();
         if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
-        abort_merge_turn<T, D, G>(p, s, g, part, nparts, last_flag);
+        abort_merge_turn<T, D, G>(p, s, g, (long long)s * p.num_heads + (long long)g * G, part, nparts, last_flag);
         return;
     }
     tc_fence_after();

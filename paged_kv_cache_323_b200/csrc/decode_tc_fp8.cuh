@@ -27,26 +27,28 @@
 //    contiguous in a token's row).  The probabilities p in [0, 1] are split
 //    the same way at scale 256: 256 p = hi + lo / 16, so every p keeps 8
 //    significant bits (as a bf16 P would) down to 2^-14, and errs by under
-//    2^-22 below that.  hi and lo go to two accumulators, O_hi and O_lo,
-//    combined as O_hi + O_lo / 16 when the chunk is folded; the running sums
-//    add the same represented values.  V rows that are not tokens of the
+//    2^-22 below that.  P^T holds both terms as rows (2h: hi, 2h + 1: lo), so
+//    one PV product gives O_hi and O_lo in columns 2h and 2h + 1, combined as
+//    O_hi + O_lo / 16 when the chunk is folded; the running sums add the same
+//    represented values.  V rows that are not tokens of the
 //    partition are zeroed before PV (they may hold NaN codes).
 //
 // One CTA per (sequence, kv head, partition), 192 threads:
 //  * warp 0 -- producer: per 128-token chunk, one TMA copy per block of the K
 //    tile, then of the V tile, into a ring of 16 KB slots, K tiles in the
 //    even slots and V tiles in the odd ones; no multicast.  Up to 4 query
-//    heads per kv head: two slots, so that four CTAs share an SM and their
-//    per-chunk chains overlap.  8 query heads need more registers (two CTAs
-//    per SM): six slots.
-//  * warp 1 -- TMEM owner (128 columns) and, lane 0, MMA issuer: QK^T (M=128,
-//    N=16, four K=32 steps) and PV (M=128, N=16, four K=32 steps per term),
-//    each issued as soon as its operands are ready (the issuer polls both,
-//    so neither waits behind the other).
+//    heads per CTA: two slots, so that five (up to 2 heads) or four CTAs
+//    share an SM and their per-chunk chains overlap.  8 query heads need
+//    more registers (two CTAs per SM): six slots.
+//  * warp 1 -- TMEM owner (64 columns) and, lane 0, MMA issuer: QK^T (M=128,
+//    N=16, four K=32 steps) and PV (M=128, N=16, four K=32 steps, both p
+//    terms at once), each issued as soon as its operands are ready (the
+//    issuer polls both, so neither waits behind the other).
 //  * warps 2-5 -- softmax, as in the bf16 kernel: thread r owns TMEM lane r
 //    (token r of S, dimension r of O); S, P and O are double-buffered.
 // Every wait is bounded; on timeout the CTA records the error, lets its copies
 // and MMAs land, frees TMEM and returns.
+
 #pragma once
 
 #include "decode_tc.cuh"
@@ -59,20 +61,24 @@ struct TcFp8Cfg {
     static constexpr int D = 128;
     static constexpr int TILE = 128;          // tokens per chunk
     static constexpr int BPT = TILE / BS;     // blocks per chunk
-    static constexpr int NPAD = 16;           // MMA N: 2G columns used by QK, G by PV
+    static constexpr int NPAD = 16;           // MMA N: 2GT columns used by QK, G by PV
     static constexpr int ROW = 128;           // bytes of a swizzled row: 128 codes
     static constexpr int SLOT = TILE * ROW;   // one K or V tile (16 KB)
-    static constexpr int CTAS_PER_SM = G >= 8 ? 2 : 4;
+    // CTAs per SM: more CTAs overlap more per-chunk chains (2 -> 3 -> 4 on
+    // batch-64 MHA: 122.5 / 115.0 / 112.0 us); up to 2 query heads fit the
+    // 64 registers of 5, 4 heads the 80 of 4, 8 heads need 2.
+    static constexpr int CTAS_PER_SM = G >= 8 ? 2 : (G >= 4 ? 4 : 5);
     static constexpr int NSLOT = CTAS_PER_SM == 2 ? 6 : 2;
     // tile li (K of chunk li/2 when even, V when odd) sits in slot li % NSLOT
     static constexpr int QB = NPAD * ROW;     // Q operand (hi and lo rows): 16 rows of 128 codes
-    static constexpr int PTERM = NPAD * ROW;  // one P term: 16 head rows of 128 token codes
-    static constexpr int PB = 2 * PTERM;      // one P buffer: the hi and lo terms
+    // one P buffer: P^T rows 2h (hi term) and 2h + 1 (lo term) of query head
+    // h, 128 token codes each; one PV product yields both O terms
+    static constexpr int PB = NPAD * ROW;
     static constexpr int MAX_PART_BLOCKS = 4096 / BS;
     static constexpr int THREADS = 192;
-    static constexpr uint32_t TMEM_COLS = 128;
+    static constexpr uint32_t TMEM_COLS = 64;
     static constexpr uint32_t S_COL = 0;      // two S buffers at columns 0 and 16
-    static constexpr uint32_t O_COL = 32;     // two O buffers (hi 16 + lo 16 columns) at 32 and 64
+    static constexpr uint32_t O_COL = 32;     // two O buffers at 32 and 48: column 2h hi, 2h + 1 lo
     // shared-memory map, offsets from a 1024-byte aligned base
     static constexpr int Q_OFF = NSLOT * SLOT;
     static constexpr int P_OFF = Q_OFF + QB;
@@ -90,7 +96,7 @@ struct TcFp8Cfg {
 
     static_assert(TILE % BS == 0 && (BS * ROW) % 1024 == 0, "blocks stack on swizzle atoms");
     static_assert(2 * G <= NPAD && G <= 8, "hi and lo columns of every head fit the MMA N");
-    static_assert(Q_OFF % 1024 == 0 && P_OFF % 1024 == 0 && PTERM % 1024 == 0, "operand alignment");
+    static_assert(Q_OFF % 1024 == 0 && P_OFF % 1024 == 0 && PB % 1024 == 0, "operand alignment");
     static_assert(merge_scratch_bytes<G, D, THREADS>() <= NSLOT * SLOT, "merge scratch reuses the ring");
     static_assert(CTAS_PER_SM * (SMEM_BYTES + 1024) <= 228 * 1024, "CTAs per SM by shared memory");
     static_assert(CTAS_PER_SM * TMEM_COLS <= 512, "CTAs per SM by TMEM");
@@ -132,56 +138,6 @@ __device__ __forceinline__ float warp_max(float v) {
     float r;
     asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
     return r;
-}
-
-// Columns [0, N) and [16, 16 + N) of this thread's TMEM lane from taddr, with
-// one wait for both loads (N = 1, 2, 4 or 8): the hi and lo accumulators of
-// the first N heads.
-template <int N>
-__device__ __forceinline__ void tmem_ld_hi_lo(uint32_t taddr, float (&hi)[N], float (&lo)[N]) {
-    static_assert(N == 1 || N == 2 || N == 4 || N == 8, "load shape");
-    uint32_t r[2 * N];
-    if constexpr (N == 1) {
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%2];\n\t"
-            "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%1}, [%3];\n\t"
-            "tcgen05.wait::ld.sync.aligned;"
-            : "=r"(r[0]), "=r"(r[1])
-            : "r"(taddr), "r"(taddr + 16u)
-            : "memory");
-    } else if constexpr (N == 2) {
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%4];\n\t"
-            "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%2, %3}, [%5];\n\t"
-            "tcgen05.wait::ld.sync.aligned;"
-            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-            : "r"(taddr), "r"(taddr + 16u)
-            : "memory");
-    } else if constexpr (N == 4) {
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%8];\n\t"
-            "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%4, %5, %6, %7}, [%9];\n\t"
-            "tcgen05.wait::ld.sync.aligned;"
-            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-              "=r"(r[7])
-            : "r"(taddr), "r"(taddr + 16u)
-            : "memory");
-    } else if constexpr (N == 8) {
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%16];\n\t"
-            "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%8, %9, %10, %11, %12, %13, %14, %15}, [%17];\n\t"
-            "tcgen05.wait::ld.sync.aligned;"
-            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-              "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-              "=r"(r[14]), "=r"(r[15])
-            : "r"(taddr), "r"(taddr + 16u)
-            : "memory");
-    }
-#pragma unroll
-    for (int i = 0; i < N; ++i) {
-        hi[i] = __uint_as_float(r[i]);
-        lo[i] = __uint_as_float(r[N + i]);
-    }
 }
 
 // The first N columns of this thread's TMEM lane from taddr, waited for
@@ -242,19 +198,19 @@ __global__ void __launch_bounds__(192, TcFp8Cfg<BS, G>::CTAS_PER_SM)
     const Unit unit = decode_unit(p, P <= 4);
     if (unit.s < 0) return;  // a schedule entry out of range (debug builds)
     const int part = unit.part, g = unit.g, s = unit.s;
-    const int ctx = p.context_lens[s];
+    const int ctx = unit.ctx;
     const int max_ctx = p.max_blocks_per_seq * BS;
     if (ctx < 0 || ctx > max_ctx) {
         if (part == 0) {
             if (threadIdx.x == 0) set_error(p.err, PKV_ERR_DEVICE_BOUNDS);
-            zero_rows<T, D, G>(p, s, g);
+            zero_rows<T, D, G>(p, (long long)s * p.num_heads + (long long)g * G);
         }
         return;
     }
     const int PTOK = p.partition_tokens;
     const int nparts = (ctx + PTOK - 1) / PTOK;
     if (part >= nparts) {
-        if (ctx == 0 && part == 0) zero_rows<T, D, G>(p, s, g);
+        if (ctx == 0 && part == 0) zero_rows<T, D, G>(p, (long long)s * p.num_heads + (long long)g * G);
         return;
     }
     const int tok0 = part * PTOK;
@@ -320,12 +276,13 @@ __global__ void __launch_bounds__(192, TcFp8Cfg<BS, G>::CTAS_PER_SM)
         // rows past 2G; thread t writes 16 codes (dims 16j .. 16j+15) of row t / 8.
         const int t = tid - 64;
         const int n = t >> 3, j = t & 7;
+        const int hq = n >> 1;  // query head within the group
         float qv[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) qv[e] = 0.f;
         if (n < 2 * G) {
             const uint4* qrow = reinterpret_cast<const uint4*>(
-                static_cast<const T*>(p.q) + ((long long)s * p.num_heads + g * G + (n >> 1)) * D + j * 16);
+                static_cast<const T*>(p.q) + ((long long)s * p.num_heads + g * G + hq) * D + j * 16);
             Elem<T>::unpack(qrow[0], qv);
             Elem<T>::unpack(qrow[1], qv + 8);
         }
@@ -359,7 +316,7 @@ __global__ void __launch_bounds__(192, TcFp8Cfg<BS, G>::CTAS_PER_SM)
         *reinterpret_cast<uint4*>(smem + C::Q_OFF + n * C::ROW + ((j ^ (n & 7)) * 16)) = val;
         // the logit of head n/2 is its S columns' sum times scale, k_scale and 2^-k
         if (n < 2 * G && (n & 1) == 0 && j == 0)
-            qsk[n >> 1] = p.qscale * p.k_scales[g] * __uint_as_float((uint32_t)(127 - kexp) << 23);
+            qsk[hq] = p.qscale * p.k_scales[g] * __uint_as_float((uint32_t)(127 - kexp) << 23);
         for (int u = t; u < 2 * C::PB / 16; u += 128)
             reinterpret_cast<uint4*>(smem + C::P_OFF)[u] = make_uint4(0u, 0u, 0u, 0u);
         fence_proxy_async_smem();
@@ -441,16 +398,15 @@ __global__ void __launch_bounds__(192, TcFp8Cfg<BS, G>::CTAS_PER_SM)
                         tc_fence_after();
                         const uint32_t v_base = smem_addr(smem + st * C::SLOT);
                         const uint32_t p_base = smem_addr(smem + C::P_OFF + (np & 1) * C::PB);
-                        const uint32_t o_hi = tmem + C::O_COL + (np & 1) * 32;
+                        const uint32_t o_col = tmem + C::O_COL + (np & 1) * 16;
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
                             // A = V^T, MN-major: the 128 dims of a token are one swizzled
-                            // row; 32 tokens per step, 8-token groups 1024 B apart
+                            // row; 32 tokens per step, 8-token groups 1024 B apart.
+                            // B = P^T, both terms of every head (N = 16).
                             const uint64_t a = sw128_desc(v_base + kk * 32 * C::ROW, 16, 1024);
-                            const uint64_t bh = sw128_desc(p_base + kk * 32, 16, 1024);
-                            const uint64_t bl = sw128_desc(p_base + C::PTERM + kk * 32, 16, 1024);
-                            mma_kind_f8f6f4(o_hi, a, bh, C::IDESC_PV, kk > 0);
-                            mma_kind_f8f6f4(o_hi + 16, a, bl, C::IDESC_PV, kk > 0);
+                            const uint64_t b = sw128_desc(p_base + kk * 32, 16, 1024);
+                            mma_kind_f8f6f4(o_col, a, b, C::IDESC_PV, kk > 0);
                         }
                         mma_commit(&o_full[np & 1]);
                         mma_commit(&empty[st]);
@@ -481,14 +437,20 @@ __global__ void __launch_bounds__(192, TcFp8Cfg<BS, G>::CTAS_PER_SM)
         for (int h = 0; h < G; ++h) {
             m_run[h] = -INFINITY;
             l_run[h] = 0.f;
-            acc[h] = 0.f;
             alpha_prev[h] = 1.f;
         }
+#pragma unroll
+        for (int h = 0; h < G; ++h) acc[h] = 0.f;
         auto fold = [&](int cc, const float* alpha) -> bool {
             if (!wait_all(&o_full[cc & 1], (cc >> 1) & 1)) return false;
             tc_fence_after();
-            float oh[G], ol[G];
-            tmem_ld_hi_lo<G>(lane_addr + C::O_COL + (cc & 1) * 32, oh, ol);
+            float ov[2 * G], oh[G], ol[G];
+            tmem_ld_first<2 * G>(lane_addr + C::O_COL + (cc & 1) * 16, ov);
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                oh[h] = ov[2 * h];
+                ol[h] = ov[2 * h + 1];
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&o_free[cc & 1]);
@@ -538,7 +500,7 @@ __global__ void __launch_bounds__(192, TcFp8Cfg<BS, G>::CTAS_PER_SM)
                 pr[h] = valid ? exp2f(x[h] - m_new) * 256.f : 0.f;
             }
             if constexpr (GP > G) pr[G] = 0.f;
-            // 256 p = hi + lo / 16, both e4m3; P^T rows are heads, K-major over tokens
+            // 256 p = hi + lo / 16, both e4m3; P^T rows 2h, 2h + 1, K-major over tokens
             unsigned char* pbuf = smem + C::P_OFF + (c & 1) * C::PB;
 #pragma unroll
             for (int h = 0; h < GP; h += 2) {
@@ -552,9 +514,9 @@ __global__ void __launch_bounds__(192, TcFp8Cfg<BS, G>::CTAS_PER_SM)
                     if (hh >= G) break;
                     const float rep = (u ? fmaf(lv.y, 0.0625f, hv.y) : fmaf(lv.x, 0.0625f, hv.x)) * 0.00390625f;
                     l_run[hh] = fmaf(l_run[hh], alpha[hh], rep);
-                    const int off = hh * C::ROW + (((r >> 4) ^ (hh & 7)) << 4) + (r & 15);
-                    pbuf[off] = (unsigned char)(hc >> (8 * u));
-                    pbuf[C::PTERM + off] = (unsigned char)(lc >> (8 * u));
+                    const int rh = 2 * hh, rl = 2 * hh + 1;  // P^T rows of the two terms
+                    pbuf[rh * C::ROW + (((r >> 4) ^ (rh & 7)) << 4) + (r & 15)] = (unsigned char)(hc >> (8 * u));
+                    pbuf[rl * C::ROW + (((r >> 4) ^ (rl & 7)) << 4) + (r & 15)] = (unsigned char)(lc >> (8 * u));
                 }
             }
             // the V tile must have landed; rows that are not valid tokens get
@@ -635,7 +597,8 @@ __global__ void __launch_bounds__(192, TcFp8Cfg<BS, G>::CTAS_PER_SM)
         __syncthreads();
         tc_fence_after();
         if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
-        abort_merge_turn<T, D, G>(p, s, g, part, nparts, last_flag);
+        abort_merge_turn<T, D, G>(p, s, g, (long long)s * p.num_heads + (long long)g * G, part,
+                                   nparts, last_flag);
         return;
     }
     tc_fence_after();

@@ -561,7 +561,11 @@ def set_tensor_core_gqa(enable: bool) -> bool:
     return bool(lib.pkv_set_tensor_core_gqa(1 if enable else 0))
 
 
-def set_longest_first(enable: bool) -> bool:
-    """Order the decode grid longest first (True, the default) or by index
-    (False); both give the same bits.  Returns the previous setting."""
-    return bool(lib.pkv_set_longest_first(1 if enable else 0))
+def set_longest_first(mode: int) -> int:
+    """Schedule of the decode grid: 1 (the default) longest first where it
+    pays, 2 always, 0 never; all give the same bits.  Returns the previous
+    mode."""
+    rc = int(lib.pkv_set_longest_first(int(mode)))
+    if rc < 0:
+        raise PagedKVError(rc, "pkv_set_longest_first")
+    return rc

@@ -4,10 +4,11 @@ a device sanitizer.
 
 On the CPU: it compiles for sm_100a, loads, exports every symbol the header
 declares, and says which build it is.  On the GPU: one step of every kernel
-family (CUDA-core decode at block sizes 8 / 16 / 32, the tensor-core decode
-over bf16 and fp8 caches, split-K with the fused merge, the longest-first
-schedule, the no-alloc entry, append and copy-on-write) runs through the
-debug library in a child process, matches the oracle, and no check fails.
+family (CUDA-core decode at block sizes 8 / 16 / 32 over fp32, bf16 and fp8
+caches, the tensor-core decode over bf16 and fp8 caches, split-K with the
+fused merge, the longest-first schedule, the no-alloc entry, append and
+copy-on-write) runs through the debug library in a child process, matches
+the oracle, and no check fails.
 """
 import ctypes
 import os
@@ -41,6 +42,7 @@ from paged_kv_cache_323_b200 import pagedkv as pk
 from paged_kv_cache_323_b200 import workload as wl
 from steps import gpu_step, oracle_step, assert_close, assert_pool_equal, to_device
 assert pk.DEBUG and pk.lib.pkv_debug_build() == 1
+pk.set_longest_first(2)  # plan every launch, so the schedule's checks run too
 cases = [
     ("cuda-core bs8 split-K", wl.mha(num_seqs=6, num_blocks=1200, heads=4, block_size=8), 256),
     ("cuda-core bs16", wl.mha(num_seqs=6, num_blocks=600, heads=4), 0),
@@ -51,6 +53,9 @@ cases = [
                                  block_size=16, dtype="fp8"), 512),
     ("cuda-core fp8 head_dim 64", wl.custom(6, [5, 77, 900], heads=4, kv_heads=2, head_dim=64,
                                            block_size=16, dtype="fp8"), 256),
+    ("cuda-core fp8 head_dim 64, 8 heads per kv head", wl.custom(8, [5, 77, 900], heads=16, kv_heads=2,
+                                                                 head_dim=64, block_size=16,
+                                                                 dtype="fp8"), 256),
 ]
 for name, w, pt in cases:
     ref, kref, vref = oracle_step(w)

@@ -45,6 +45,12 @@ def test_fp8_mha_full():
     full_size_check(wl.mha(device="cuda", dtype="fp8"))
 
 
+def test_fp8_head_dim_64_full():
+    """The batch-64 MHA step with head_dim 64 over an fp8 cache (the
+    CUDA-core kernel): every row."""
+    full_size_check(wl.mha(device="cuda", head_dim=64, dtype="fp8"))
+
+
 def test_fp8_saturates_large_values():
     """New tokens far beyond the e4m3 range store +-448 codes, as the oracle does."""
     w = wl.custom(5, [40, 17], heads=4, kv_heads=2, head_dim=128, block_size=16, dtype="fp8")

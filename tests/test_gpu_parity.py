@@ -134,8 +134,8 @@ def test_schedule_does_not_change_bits(make, pt):
     w = make()
     ref, _, _ = oracle_step(w)
     outs = []
-    for longest_first in (True, False):
-        prev = pk.set_longest_first(longest_first)
+    for mode in (2, 0):  # planned longest first, index order
+        prev = pk.set_longest_first(mode)
         try:
             out, _, _ = gpu_step(w, partition_tokens=pt)  # the step is idempotent on fresh copies
         finally:

@@ -127,3 +127,4 @@ def test_tc_fp8_group8_bs32_long_partitions(tc_mode, pt):
     out, kc, vc = gpu_step(w, partition_tokens=pt)
     assert_pool_equal(kc, kref, "k pool (codes)")
     assert_close(out, ref, "bf16")
+

@@ -41,10 +41,12 @@ def test_traffic_file_matches_current_kernel_sources(path):
         float(kv["dram_bytes_per_launch"])
 
 
-@pytest.mark.parametrize("heads,kv_heads,dtype,family", [
-    (32, 32, "bf16", "cuda_core"), (32, 8, "bf16", "tc_bf16"), (64, 8, "bf16", "tc_bf16"),
-    (32, 32, "fp8", "tc_fp8"), (32, 8, "fp8", "tc_fp8"), (8, 8, "f32", "cuda_core"),
+@pytest.mark.parametrize("heads,kv_heads,dtype,head_dim,family", [
+    (32, 32, "bf16", 128, "cuda_core"), (32, 8, "bf16", 128, "tc_bf16"), (64, 8, "bf16", 128, "tc_bf16"),
+    (32, 32, "fp8", 128, "tc_fp8"), (32, 8, "fp8", 128, "tc_fp8"), (8, 8, "f32", 128, "cuda_core"),
+    (32, 32, "fp8", 64, "cuda_core"), (32, 8, "bf16", 64, "cuda_core"),
 ])
-def test_kernel_family_by_shape(heads, kv_heads, dtype, family):
-    w = wl.custom(1, [40, 7], heads=heads, kv_heads=kv_heads, head_dim=128, block_size=16, dtype=dtype)
+def test_kernel_family_by_shape(heads, kv_heads, dtype, head_dim, family):
+    w = wl.custom(1, [40, 7], heads=heads, kv_heads=kv_heads, head_dim=head_dim, block_size=16,
+                  dtype=dtype)
     assert bench.decode_kernel_family(w) == family
