@@ -305,20 +305,24 @@ def test_launch_count_and_profiler():
     from paged_kv_cache_323_b200 import pagedkv as pk
 
     w = wl.mha(num_seqs=4, num_blocks=600, heads=4, ctx_range=(600, 2048))
-    t = to_device(w)
-    pk.profile_reset()
-    pk.profile_enable(True)
-    n0 = pk.launch_count()
-    gpu_step(w, t)
-    pk.profile_enable(False)
-    # append, then the decode's longest-first schedule and the decode itself
-    # (split-K merge fused); the profiler counts the last two as one decode
-    assert pk.launch_count() - n0 == 3
-    n, ms = pk.profile_read(pk.KERNEL_DECODE)
-    assert n == 1 and ms > 0
-    n, _ = pk.profile_read(pk.KERNEL_APPEND)
-    assert n == 1
-    pk.profile_reset()
+    # the default schedule leaves this CUDA-core launch unplanned: append,
+    # decode (split-K merge fused); planned, the schedule kernel comes first
+    # and the profiler counts it with the decode as one decode launch
+    for mode, kernels in ((1, 2), (2, 3)):
+        prev = pk.set_longest_first(mode)
+        t = to_device(w)
+        pk.profile_reset()
+        pk.profile_enable(True)
+        n0 = pk.launch_count()
+        gpu_step(w, t)
+        pk.profile_enable(False)
+        pk.set_longest_first(prev)
+        assert pk.launch_count() - n0 == kernels, mode
+        n, ms = pk.profile_read(pk.KERNEL_DECODE)
+        assert n == 1 and ms > 0
+        n, _ = pk.profile_read(pk.KERNEL_APPEND)
+        assert n == 1
+        pk.profile_reset()
 
 
 def test_bounded_wait_runs_out_without_fault():

@@ -17,6 +17,7 @@ FAMILY = {
     "mha": "cuda_core", "gqa_sampling": "tc_bf16", "long_context": "tc_bf16",
     "prefix_bs8": "tc_bf16", "prefix_bs16": "tc_bf16", "prefix_bs32": "tc_bf16",
     "mha_fp8": "tc_fp8", "gqa_sampling_fp8": "tc_fp8", "long_context_fp8": "tc_fp8",
+    "mha_d64_fp8": "cuda_core",
 }
 
 
