@@ -124,7 +124,8 @@ def committed_traffic(kernel: str, workload: str, source_sha: str):
 KERNEL_SOURCES = {
     "cuda_core": ("common.cuh", "decode_common.cuh", "decode_attn.cuh", "decode_launch.cuh"),
     "tc_bf16": ("common.cuh", "decode_common.cuh", "decode_tc.cuh", "decode_tc.cu"),
-    "tc_fp8": ("common.cuh", "decode_common.cuh", "decode_tc.cuh", "decode_tc_fp8.cuh", "decode_tc_fp8.cu"),
+    "tc_fp8": ("common.cuh", "decode_common.cuh", "decode_tc.cuh", "decode_tc_fp8.cuh", "decode_tc_fp8p.cuh",
+               "decode_tc_fp8p.cu", "plan.cuh"),
 }
 
 

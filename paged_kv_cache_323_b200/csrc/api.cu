@@ -45,6 +45,8 @@ std::atomic<int> g_tc_gqa{1};  // tensor-core kernel for grouped-query heads whe
 // Longest-first schedule of the decode grid: 0 never, 1 where it pays (the
 // tensor-core kernels with 2 to 4 partitions per sequence), 2 always.
 std::atomic<int> g_longest_first{1};
+// fp8 tensor-core decode in persistent form where a workspace holds its queue
+std::atomic<int> g_fp8_persistent{1};
 std::atomic<unsigned long long> g_launches{0};
 std::atomic<unsigned long long> g_wait_ns{pkv::kWaitTimeoutNs};  // decode pipeline wait limit
 
@@ -137,30 +139,33 @@ bool decode_shape_supported(int head_dim, int block_size, int group) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Decode workspace.  First the split-K merge counters, one int per
-// (sequence, kv head), in a region of at least kFixedCounterSlots slots at
-// offset 0 that nothing else is ever written to; then the longest-first
-// schedule of the launch ([B * P] int2); then, when sequences are split, the
-// fp32 partial outputs [B][H][P][D] and the (m, l) pairs [B][H][P]; each
-// region 256-byte aligned.  Every launch, complete or stopped by a timeout,
-// leaves the counters it used at zero, so the first kFixedCounterSlots
-// counters are zero between calls whatever shape each call has.  A batch
-// with more (sequence, kv head) units than that uses counters past the fixed
-// region, where an earlier call may have left other data: decode_impl clears
-// that part on every such call.
+// Decode workspace.  First the counters, in a region that nothing else is
+// ever written to: the persistent kernels' work queue (16 ints at offset 0)
+// and the split-K merge counters, one int per (sequence, kv head), in at
+// least kFixedCounterSlots slots; then the longest-first schedule of the
+// launch ([B * P] int2); then, when sequences are split, the fp32 partial
+// outputs [B][H][P][D] and the (m, l) pairs [B][H][P]; each region 256-byte
+// aligned.  Every launch, complete or stopped by a timeout, leaves the
+// counters it used at zero, so the fixed region is zero between calls
+// whatever shape each call has.  A batch with more (sequence, kv head)
+// units than kFixedCounterSlots also uses counters past the fixed region,
+// where an earlier call may have left other data: decode_impl clears that
+// part on every such call.
 constexpr long long kFixedCounterSlots = 65536;
+constexpr size_t kWorkBytes = 64;  // the work queue's counters
 
 struct WorkspaceLayout {
-    size_t cnt_off, plan_off, o_off, ml_off, total;
+    size_t work_off, cnt_off, plan_off, o_off, ml_off, total;
 };
 
 WorkspaceLayout workspace_layout(long long num_seqs, long long num_heads, long long parts, long long D) {
-    WorkspaceLayout w{0, 0, 0, 0, 0};
+    WorkspaceLayout w{0, 0, 0, 0, 0, 0};
     if (num_seqs <= 0 || parts <= 0) return w;
     const long long slots = num_seqs * num_heads > kFixedCounterSlots ? num_seqs * num_heads
                                                                       : kFixedCounterSlots;
-    w.cnt_off = 0;
-    w.plan_off = align256(size_t(slots) * sizeof(int));
+    w.work_off = 0;
+    w.cnt_off = kWorkBytes;
+    w.plan_off = align256(kWorkBytes + size_t(slots) * sizeof(int));
     w.o_off = w.plan_off + align256(size_t(num_seqs) * parts * sizeof(int2));
     w.ml_off = w.o_off;
     w.total = w.o_off;
@@ -220,9 +225,18 @@ int resolve_partition_tokens(int num_seqs, int num_heads, int num_kv_heads, int 
                              int block_size, long long max_ctx, int dtype, int partition_tokens) {
     if (partition_tokens != 0) return partition_tokens;
     const int group = num_kv_heads > 0 ? num_heads / num_kv_heads : 1;
-    return auto_partition_tokens(num_seqs, num_kv_heads, max_ctx,
-                                 tc_shape(dtype, head_dim, block_size, group),
-                                 dtype == PKV_FP8_E4M3);
+    const bool tc = tc_shape(dtype, head_dim, block_size, group);
+    const bool fp8 = dtype == PKV_FP8_E4M3;
+    int pt = auto_partition_tokens(num_seqs, num_kv_heads, max_ctx, tc, fp8);
+    // the persistent fp8 tensor-core kernel holds two tables of at most 128
+    // blocks per CTA: 2048 tokens at block size 16 (batch-64 MHA 106.5 us at
+    // 2048 against 112.1 us at 1024; the parallel-sampling batch 125.3 / 144.1)
+    if (tc && fp8 && g_fp8_persistent.load() != 0 &&
+        pkv::decode_tc_fp8_persistent_supported(block_size, group, 128)) {
+        const int cap = pkv::decode_tc_fp8_persistent_max_tokens(block_size);
+        if (pt > cap) pt = cap;
+    }
+    return pt;
 }
 
 }  // namespace
@@ -243,9 +257,9 @@ extern "C" void pkv_internal_decode_scratch(int num_seqs, int num_heads, int num
     const long long parts = (max_ctx + pt - 1) / pt;
     const WorkspaceLayout w = workspace_layout(num_seqs, num_heads, parts, head_dim);
     *total = w.total;
-    if (w.total > 0 && parts > 1) {
-        *cnt_off = w.cnt_off;
-        *cnt_bytes = size_t(num_seqs) * num_kv_heads * sizeof(int);
+    if (w.total > 0) {  // the work queue and the merge counters this batch uses
+        *cnt_off = w.work_off;
+        *cnt_bytes = w.cnt_off + size_t(num_seqs) * num_kv_heads * sizeof(int);
     }
 }
 
@@ -338,18 +352,23 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     p.ws_o = split ? reinterpret_cast<float*>(wsb + wl.o_off) : nullptr;
     p.ws_ml = split ? reinterpret_cast<float2*>(wsb + wl.ml_off) : nullptr;
     p.counters = split ? reinterpret_cast<int*>(wsb + wl.cnt_off) : nullptr;
+    p.work = workspace != nullptr ? reinterpret_cast<int*>(wsb + wl.work_off) : nullptr;
     // The schedule pays where index order leaves the longest work for last:
     // the tensor-core kernels run 2 to 4 partitions per sequence
     // partition-major, so the later partitions, which only the longest
     // sequences have, come at the end of the launch (parallel-sampling batch:
-    // 257 -> 250 us bf16, 154 -> 145 us fp8).  Elsewhere it does not: with
-    // one partition per sequence and nearly equal lengths (a shared-prefix
-    // batch) longest first starts the CTAs in synchronised waves that read
-    // the shared blocks in step (+4 %), and the planning kernel itself costs
-    // about 4 us per launch.
+    // 257 -> 250 us bf16), and the persistent fp8 kernel takes its units in
+    // queue order, so a long unit taken last runs alone (parallel-sampling
+    // batch 136.2 -> 125.3 us, batch-64 MHA 109.6 -> 106.5 us).  Elsewhere it
+    // does not: with one partition per sequence and nearly equal lengths (a
+    // shared-prefix batch) longest first starts the CTAs in synchronised
+    // waves that read the shared blocks in step (+4 %), and the planning
+    // kernel itself costs about 4 us per launch.
+    const bool persistent = use_tc && fp8 && workspace != nullptr && g_fp8_persistent.load() != 0 &&
+                            pkv::decode_tc_fp8_persistent_supported(block_size, group, pt);
     const int sched = g_longest_first.load();
     const bool plan = workspace != nullptr &&
-                      (sched == 2 || (sched == 1 && use_tc && parts >= 2 && parts <= 4));
+                      (sched == 2 || (sched == 1 && (persistent || (use_tc && parts >= 2 && parts <= 4))));
     int2* order = plan ? reinterpret_cast<int2*>(wsb + wl.plan_off) : nullptr;
     p.order = order;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -382,7 +401,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
             const cudaError_t e = cudaGetLastError();
             if (e != cudaSuccess) return e;
         }
-        if (use_tc) return pkv::launch_decode_tc(p, kv_dtype, block_size, group, grid, st);
+        if (use_tc) return pkv::launch_decode_tc(p, kv_dtype, block_size, group, grid, persistent, st);
         if (fp8) return pkv::launch_decode_partition_fp8(p, head_dim, block_size, group, grid, st);
         return dtype == PKV_F32 ? pkv::launch_decode_partition_f32(p, head_dim, block_size, group, grid, st)
                                 : pkv::launch_decode_partition_bf16(p, head_dim, block_size, group, grid, st);
@@ -750,6 +769,10 @@ int pkv_set_wait_limit_us(int microseconds) {
 int pkv_set_longest_first(int mode) {
     if (mode < 0 || mode > 2) return PKV_ERR_INVALID;
     return g_longest_first.exchange(mode);
+}
+
+PKV_API int pkv_internal_set_fp8_persistent(int enable) {
+    return g_fp8_persistent.exchange(enable != 0 ? 1 : 0);
 }
 
 int pkv_set_tensor_core_gqa(int enable) {

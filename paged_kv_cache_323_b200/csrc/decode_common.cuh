@@ -22,6 +22,9 @@ struct DecodeParams {
     float* ws_o;    // [B][H][P][D] unnormalised partial outputs
     float2* ws_ml;  // [B][H][P] (running max in log2 units, running sum)
     int* counters;  // [B][Hkv] partitions finished, zero between launches
+    // persistent kernels' work queue: [0] next unit, [1] CTAs done; zero
+    // between launches (the last CTA of a launch resets both)
+    int* work;
     // longest-first schedule written by plan_kernel just before this launch
     // ([B * P] entries {s * P + part, context length of s}), or null for
     // index order
@@ -115,15 +118,19 @@ constexpr int merge_scratch_bytes() {
     return ((2 * G + 3) / 4) * 16 + (NTHREADS > G * D / 4 ? NTHREADS : G * D / 4) * 16;
 }
 
-template <typename T, int D, int G, int NTHREADS>
-__device__ __forceinline__ void fused_merge(const DecodeParams& p, int s, int g, int nparts,
-                                            long long sh0, float* scratch, int* last_flag) {
-    const int tid = threadIdx.x;
+// The merge itself, for the NTHREADS threads that call it: tid is the
+// caller's index among them and sync() a barrier over exactly those threads,
+// which returns false when it could not complete (a bounded wait that ran
+// out); the merge then returns false too.
+template <typename T, int D, int G, int NTHREADS, class Sync>
+__device__ __forceinline__ bool fused_merge_with(const DecodeParams& p, int s, int g, int nparts,
+                                                 long long sh0, float* scratch, int* last_flag,
+                                                 int tid, Sync&& sync) {
     const int warp = tid >> 5;
     const int lane = tid & 31;
     const int P = p.num_partitions;
     __threadfence();
-    __syncthreads();
+    if (!sync()) return false;
     if (tid == 0) {
         *last_flag = 0;
         if (PKV_DCHECK(p.err, nparts <= P && (long long)s * p.num_kv_heads + g <
@@ -134,8 +141,8 @@ __device__ __forceinline__ void fused_merge(const DecodeParams& p, int s, int g,
             *last_flag = old == (unsigned)(nparts - 1);
         }
     }
-    __syncthreads();
-    if (!*last_flag) return;
+    if (!sync()) return false;
+    if (!*last_flag) return true;
     __threadfence();
 
     // per head: M = max_i m_i, L = sum_i 2^(m_i - M) l_i (one warp per head)
@@ -160,7 +167,7 @@ __device__ __forceinline__ void fused_merge(const DecodeParams& p, int s, int g,
             red[2 * hg + 1] = L;
         }
     }
-    __syncthreads();
+    if (!sync()) return false;
     // out = sum_i 2^(m_i - M) o_i / L, partitions split over thread groups
     constexpr int COLS = D / 4;
     constexpr int UNITS = G * COLS;
@@ -188,7 +195,7 @@ __device__ __forceinline__ void fused_merge(const DecodeParams& p, int s, int g,
         }
         acc_s[grp * UNITS + unit] = a;
     }
-    __syncthreads();
+    if (!sync()) return false;
     for (int unit = tid; unit < UNITS; unit += NTHREADS) {
         const int hg = unit / COLS;
         const int col = unit % COLS;
@@ -209,6 +216,18 @@ __device__ __forceinline__ void fused_merge(const DecodeParams& p, int s, int g,
         Elem<T>::store(dst + 2, t.z * inv);
         Elem<T>::store(dst + 3, t.w * inv);
     }
+    return true;
+}
+
+// The fused merge for a whole CTA (all NTHREADS threads, __syncthreads).
+template <typename T, int D, int G, int NTHREADS>
+__device__ __forceinline__ void fused_merge(const DecodeParams& p, int s, int g, int nparts,
+                                            long long sh0, float* scratch, int* last_flag) {
+    fused_merge_with<T, D, G, NTHREADS>(p, s, g, nparts, sh0, scratch, last_flag, (int)threadIdx.x,
+                                        [] {
+                                            __syncthreads();
+                                            return true;
+                                        });
 }
 
 // Zero the G output rows of D values from query head row sh0 (= s * H + the

@@ -91,14 +91,16 @@ bool decode_tc_supported(int kv_dtype, int D, int BS, int G, int partition_token
 }
 
 cudaError_t launch_decode_tc(const DecodeParams& p, int kv_dtype, int BS, int G, long long grid,
-                             cudaStream_t st) {
+                             bool persistent, cudaStream_t st) {
     const int eb = kv_dtype == PKV_FP8_E4M3 ? 1 : 2;
     CUtensorMap mk, mv;
     cudaError_t e = make_tc_pool_map(&mk, p.k_cache, p.num_kv_heads, BS, p.num_blocks, eb);
     if (e != cudaSuccess) return e;
     e = make_tc_pool_map(&mv, p.v_cache, p.num_kv_heads, BS, p.num_blocks, eb);
     if (e != cudaSuccess) return e;
-    if (kv_dtype == PKV_FP8_E4M3) return launch_decode_tc_fp8(p, mk, mv, BS, G, grid, st);
+    if (kv_dtype == PKV_FP8_E4M3)
+        return persistent ? launch_decode_tc_fp8_persistent(p, mk, mv, BS, G, grid, st)
+                          : launch_decode_tc_fp8(p, mk, mv, BS, G, grid, st);
     switch (BS) {
         case 8: return launch_group<8>(p, G, mk, mv, grid, st);
         case 16: return launch_group<16>(p, G, mk, mv, grid, st);

@@ -20,12 +20,21 @@ cudaError_t launch_decode_partition_fp8(const DecodeParams& p, int D, int BS, in
 // tokens: bf16 caches with groups of 2, 4 or 8 query heads, fp8 (e4m3)
 // caches with groups of 1, 2, 4 or 8.
 bool decode_tc_supported(int kv_dtype, int D, int BS, int G, int partition_tokens);
+// persistent: the fp8 kernel that takes its units from the work queue in
+// p.work, in the order of the schedule p.order when there is one (needs a
+// workspace and decode_tc_fp8_persistent_supported: 1, 2 or 4 query heads per
+// kv head, partitions of at most decode_tc_fp8_persistent_max_tokens(BS))
 cudaError_t launch_decode_tc(const DecodeParams& p, int kv_dtype, int BS, int G, long long grid,
-                             cudaStream_t st);
+                             bool persistent, cudaStream_t st);
+bool decode_tc_fp8_persistent_supported(int BS, int G, int partition_tokens);
+int decode_tc_fp8_persistent_max_tokens(int BS);
 // internal to the tensor-core translation units
 cudaError_t make_tc_pool_map(CUtensorMap* map, const void* pool, int Hkv, int BS, int num_blocks,
                              int elem_bytes);
 cudaError_t launch_decode_tc_fp8(const DecodeParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
                                  int BS, int G, long long grid, cudaStream_t st);
+cudaError_t launch_decode_tc_fp8_persistent(const DecodeParams& p, const CUtensorMap& mk,
+                                            const CUtensorMap& mv, int BS, int G, long long units,
+                                            cudaStream_t st);
 
 }  // namespace pkv

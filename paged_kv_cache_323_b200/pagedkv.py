@@ -93,6 +93,9 @@ for _name, (_res, _args) in SIGNATURES.items():
     _fn = getattr(lib, _name)
     _fn.restype = _res
     _fn.argtypes = _args
+# not in the header: selects the fp8 tensor-core decode's persistent form
+lib.pkv_internal_set_fp8_persistent.restype = _I
+lib.pkv_internal_set_fp8_persistent.argtypes = [_I]
 
 
 class PagedKVError(RuntimeError):
@@ -559,6 +562,15 @@ def set_tensor_core_gqa(enable: bool) -> bool:
     where a tensor-core one applies (bf16 caches with grouped query heads,
     fp8 caches); returns the previous setting."""
     return bool(lib.pkv_set_tensor_core_gqa(1 if enable else 0))
+
+
+def _set_fp8_persistent(enable: bool) -> bool:
+    """The fp8 tensor-core decode in persistent form (the default: one CTA
+    per resident slot taking units from a queue in the workspace, longest
+    first) where it applies -- a workspace is given and partitions are at
+    most 128 blocks -- or one CTA per unit (False).  Returns the previous
+    setting."""
+    return bool(lib.pkv_internal_set_fp8_persistent(1 if enable else 0))
 
 
 def set_longest_first(mode: int) -> int:

@@ -138,9 +138,17 @@ def test_partition_tokens(pk):
     assert pt(256, 32, 8, 128, 16, 8256, bf, 0) == 4096
     assert pt(8, 64, 8, 128, 32, 131072, bf, 0) == 4096  # 2048 CTAs: still 4 waves
     assert pt(1, 32, 8, 128, 16, 1024, bf, 0) == 512
-    f8 = pk.PKV_FP8_E4M3  # fp8 caches: the tensor-core kernel for MHA too
-    assert pt(64, 32, 32, 128, 16, 2048, f8, 0) == 4096
+    # fp8 caches: the tensor-core kernel for MHA too, in persistent form, whose
+    # partitions hold at most 128 blocks
+    f8 = pk.PKV_FP8_E4M3
+    assert pt(64, 32, 32, 128, 16, 2048, f8, 0) == 2048
     assert pt(8, 64, 8, 128, 32, 131072, f8, 0) == 4096
+    assert pt(64, 32, 32, 128, 8, 2048, f8, 0) == 1024
+    prev = pk._set_fp8_persistent(False)
+    try:
+        assert pt(64, 32, 32, 128, 16, 2048, f8, 0) == 4096  # one CTA per unit
+    finally:
+        pk._set_fp8_persistent(prev)
     prev = pk.set_tensor_core_gqa(False)
     try:
         big = pt(8, 64, 8, 128, 32, 131072, bf, 0)  # CUDA-core kernel: fewer, larger partitions

@@ -6,7 +6,8 @@ On the CPU: it compiles for sm_100a, loads, exports every symbol the header
 declares, and says which build it is.  On the GPU: one step of every kernel
 family (CUDA-core decode at block sizes 8 / 16 / 32 over fp32, bf16 and fp8
 caches, the tensor-core decode over bf16 and fp8 caches, split-K with the
-fused merge, the longest-first schedule, the no-alloc entry, append and
+fused merge, the longest-first schedule, the fp8 tensor-core kernel in both
+forms, the no-alloc entry, append and
 copy-on-write) runs through the debug library in a child process, matches
 the oracle, and no check fails.
 """
@@ -49,8 +50,8 @@ cases = [
     ("cuda-core bs32 fp32", wl.custom(3, [1, 31, 33, 700], heads=4, kv_heads=2, head_dim=64,
                                      block_size=32, dtype="f32"), 128),
     ("tensor-core bf16 copy-on-write", wl.gqa_sampling(groups=3, prompt_median=300, prompt_max=1500), 256),
-    ("tensor-core fp8", wl.custom(5, [1, 129, 640, 3000], heads=16, kv_heads=2, head_dim=128,
-                                 block_size=16, dtype="fp8"), 512),
+    ("tensor-core fp8 (persistent)", wl.custom(5, [1, 129, 640, 3000], heads=16, kv_heads=2,
+                                              head_dim=128, block_size=16, dtype="fp8"), 512),
     ("cuda-core fp8 head_dim 64", wl.custom(6, [5, 77, 900], heads=4, kv_heads=2, head_dim=64,
                                            block_size=16, dtype="fp8"), 256),
     ("cuda-core fp8 head_dim 64, 8 heads per kv head", wl.custom(8, [5, 77, 900], heads=16, kv_heads=2,
@@ -64,6 +65,13 @@ for name, w, pt in cases:
     assert_close(out, ref, "bf16" if w.dtype == "fp8" else w.dtype, name)
     line = pk.debug_failed_line()
     assert line == 0, f"{name}: index check failed at line {line}"
+pk._set_fp8_persistent(False)  # the fp8 tensor-core kernel with one CTA per unit
+name, w, pt = cases[4]
+ref, kref, vref = oracle_step(w)
+out, kc, vc = gpu_step(w, partition_tokens=pt)
+assert_close(out, ref, "bf16", name + ", one CTA per unit")
+assert pk.debug_failed_line() == 0, "one CTA per unit: index check failed"
+pk._set_fp8_persistent(True)
 w = wl.mha(num_seqs=8, num_blocks=2048)
 ref, _, _ = oracle_step(w)
 t = to_device(w)

@@ -18,12 +18,17 @@ from steps import assert_close, assert_pool_equal, full_size_check, gpu_step, or
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture
-def tc_mode():
+@pytest.fixture(params=[False, True], ids=["per_unit", "persistent"])
+def tc_mode(request):
+    """The tensor-core fp8 kernel in both forms: one CTA per unit, and the
+    persistent one (used wherever a workspace is given and partitions are at
+    most 2048 tokens)."""
     from paged_kv_cache_323_b200 import pagedkv as pk
 
     prev = pk.set_tensor_core_gqa(True)
+    prev_p = pk._set_fp8_persistent(request.param)
     yield pk
+    pk._set_fp8_persistent(prev_p)
     pk.set_tensor_core_gqa(prev)
 
 
@@ -128,3 +133,45 @@ def test_tc_fp8_group8_bs32_long_partitions(tc_mode, pt):
     assert_pool_equal(kc, kref, "k pool (codes)")
     assert_close(out, ref, "bf16")
 
+
+
+@pytest.mark.parametrize("bs,pt", [(16, 128), (16, 1024), (16, 2048), (8, 1024), (32, 4096)])
+def test_tc_fp8_persistent_same_bits(bs, pt):
+    """The persistent form computes every unit with the same arithmetic in
+    the same order as the one-CTA-per-unit kernel, so the outputs are
+    identical bit for bit under every schedule, launch after launch on one
+    workspace (the queue is back at zero after each launch)."""
+    from paged_kv_cache_323_b200 import pagedkv as pk
+
+    w = wl.custom(71, [1, 130, 700, 2049, 4500, 0, 3000, 129], heads=16, kv_heads=4, head_dim=128,
+                  block_size=bs, dtype="fp8")
+    ref, _, _ = oracle_step(w)
+    t = to_device(w)
+    ks = torch.from_numpy(w.k_scales).cuda()
+    vs = torch.from_numpy(w.v_scales).cuda()
+    pk.kv_cache_append_fp8(t["k_cache"], t["v_cache"], ks, vs, t["k_new"], t["v_new"], t["slot_mapping"])
+    need = pk.paged_attention_workspace_size(w.num_seqs, w.num_heads,
+                                             w.max_blocks_per_seq * w.block_size, w.head_dim, pt)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    outs = []
+    prev = pk._set_fp8_persistent(False)
+    prev_sched = pk.set_longest_first(1)
+    try:
+        for persistent, sched in ((False, 1), (True, 0), (True, 1), (True, 2), (True, 1), (False, 2),
+                                  (False, 0), (True, 0)):
+            pk._set_fp8_persistent(persistent)
+            pk.set_longest_first(sched)
+            t["out"].fill_(float("nan"))
+            pk.paged_attention_decode_fp8(t["out"], t["q"], t["k_cache"], t["v_cache"], ks, vs,
+                                          t["block_tables"], t["context_lens"], w.scale,
+                                          num_blocks=w.num_blocks, partition_tokens=pt, workspace=ws)
+            torch.cuda.synchronize()
+            assert pk.get_device_error() == 0
+            outs.append(t["out"].clone())
+    finally:
+        pk._set_fp8_persistent(prev)
+        pk.set_longest_first(prev_sched)
+    assert_close(outs[0], ref, "bf16")
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
+    assert int(ws[:8].view(torch.int32).abs().sum()) == 0  # queue counters back at zero

@@ -23,8 +23,10 @@ KERNELS = {
     "cuda_core": (lambda: wl.mha(num_seqs=8, num_blocks=2048), 512),
     # grouped-query heads on the tensor-core kernel, several partitions
     "tensor_core": (lambda: wl.gqa_sampling(groups=4, prompt_median=600, prompt_max=3000), 256),
-    # fp8 cache on the tensor-core fp8 kernel
+    # fp8 cache on the tensor-core fp8 kernel, one CTA per unit
     "tensor_core_fp8": (lambda: wl.mha(num_seqs=8, num_blocks=2048, dtype="fp8"), 512),
+    # the same in persistent form: a stopped CTA also drains the work queue
+    "tensor_core_fp8_persistent": (lambda: wl.mha(num_seqs=8, num_blocks=2048, dtype="fp8"), 512),
 }
 
 
@@ -82,7 +84,14 @@ def test_timeout_then_parity_on_the_same_workspace(kernel):
     from paged_kv_cache_323_b200 import pagedkv as pk
 
     make, pt = KERNELS[kernel]
-    w = make()
+    prev = pk._set_fp8_persistent(kernel != "tensor_core_fp8")
+    try:
+        _timeout_then_parity(pk, make(), pt)
+    finally:
+        pk._set_fp8_persistent(prev)
+
+
+def _timeout_then_parity(pk, w, pt):
     ref, _, _ = oracle_step(w)
     t = _appended(pk, w)
     need = pk.paged_attention_workspace_size(w.num_seqs, w.num_heads,
