@@ -126,6 +126,8 @@ KERNEL_SOURCES = {
     "tc_bf16": ("common.cuh", "decode_common.cuh", "decode_tc.cuh", "decode_tc.cu"),
     "tc_fp8": ("common.cuh", "decode_common.cuh", "decode_tc.cuh", "decode_tc_fp8.cuh", "decode_tc_fp8p.cuh",
                "decode_tc_fp8p.cu", "plan.cuh"),
+    "tc_fp8_d64": ("common.cuh", "decode_common.cuh", "decode_tc.cuh", "decode_tc_fp8.cuh", "decode_tc_fp8_d64.cuh",
+                   "decode_tc_fp8_d64.cu", "plan.cuh"),
 }
 
 
@@ -135,6 +137,8 @@ def decode_kernel_family(w) -> str:
     group = w.num_heads // w.num_kv_heads
     if w.head_dim == 128 and w.dtype == "fp8" and group in (1, 2, 4, 8):
         return "tc_fp8"
+    if w.head_dim == 64 and w.dtype == "fp8" and group in (1, 2, 4) and w.num_kv_heads % 2 == 0:
+        return "tc_fp8_d64"
     if w.head_dim == 128 and w.dtype == "bf16" and group in (2, 4, 8):
         return "tc_bf16"
     return "cuda_core"

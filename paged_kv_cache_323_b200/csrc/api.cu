@@ -217,21 +217,24 @@ int auto_partition_tokens(long long num_seqs, long long num_kv_heads, long long 
 
 // Whether the tensor-core kernel serves this shape (any partition size that
 // is a multiple of 128 tokens).
-bool tc_shape(int dtype, int head_dim, int block_size, int group) {
-    return g_tc_gqa.load() != 0 && pkv::decode_tc_supported(dtype, head_dim, block_size, group, 128);
+bool tc_shape(int dtype, int head_dim, int block_size, int group, int num_kv_heads) {
+    return g_tc_gqa.load() != 0 &&
+           pkv::decode_tc_supported(dtype, head_dim, block_size, group, num_kv_heads, 128);
 }
 
 int resolve_partition_tokens(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                              int block_size, long long max_ctx, int dtype, int partition_tokens) {
     if (partition_tokens != 0) return partition_tokens;
     const int group = num_kv_heads > 0 ? num_heads / num_kv_heads : 1;
-    const bool tc = tc_shape(dtype, head_dim, block_size, group);
+    const bool tc = tc_shape(dtype, head_dim, block_size, group, num_kv_heads);
     const bool fp8 = dtype == PKV_FP8_E4M3;
-    int pt = auto_partition_tokens(num_seqs, num_kv_heads, max_ctx, tc, fp8);
+    // the head_dim-64 tensor-core kernel runs one CTA per pair of kv heads
+    const int head_units = tc && head_dim == 64 ? num_kv_heads / 2 : num_kv_heads;
+    int pt = auto_partition_tokens(num_seqs, head_units, max_ctx, tc, fp8);
     // the persistent fp8 tensor-core kernel holds two tables of at most 128
     // blocks per CTA: 2048 tokens at block size 16 (batch-64 MHA 106.5 us at
     // 2048 against 112.1 us at 1024; the parallel-sampling batch 125.3 / 144.1)
-    if (tc && fp8 && g_fp8_persistent.load() != 0 &&
+    if (tc && fp8 && head_dim == 128 && g_fp8_persistent.load() != 0 &&
         pkv::decode_tc_fp8_persistent_supported(block_size, group, 128)) {
         const int cap = pkv::decode_tc_fp8_persistent_max_tokens(block_size);
         if (pt > cap) pt = cap;
@@ -323,7 +326,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
                                             block_size, max_ctx, kv_dtype, partition_tokens);
     const long long parts = (max_ctx + pt - 1) / pt;
     const bool use_tc = g_tc_gqa.load() != 0 &&
-                        pkv::decode_tc_supported(kv_dtype, head_dim, block_size, group, pt);
+                        pkv::decode_tc_supported(kv_dtype, head_dim, block_size, group, num_kv_heads, pt);
     const long long grid = parts * num_kv_heads * (long long)num_seqs;
     if (grid > INT_MAX || (long long)num_seqs * num_heads > INT_MAX) return PKV_ERR_INVALID;
     const size_t need = workspace_bytes_for(num_seqs, num_heads, parts, head_dim);
@@ -364,7 +367,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     // shared-prefix batch) longest first starts the CTAs in synchronised
     // waves that read the shared blocks in step (+4 %), and the planning
     // kernel itself costs about 4 us per launch.
-    const bool persistent = use_tc && fp8 && workspace != nullptr && g_fp8_persistent.load() != 0 &&
+    const bool persistent = use_tc && fp8 && head_dim == 128 && workspace != nullptr &&
+                            g_fp8_persistent.load() != 0 &&
                             pkv::decode_tc_fp8_persistent_supported(block_size, group, pt);
     const int sched = g_longest_first.load();
     const bool plan = workspace != nullptr &&
@@ -401,7 +405,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
             const cudaError_t e = cudaGetLastError();
             if (e != cudaSuccess) return e;
         }
-        if (use_tc) return pkv::launch_decode_tc(p, kv_dtype, block_size, group, grid, persistent, st);
+        if (use_tc)
+            return pkv::launch_decode_tc(p, kv_dtype, head_dim, block_size, group, grid, persistent, st);
         if (fp8) return pkv::launch_decode_partition_fp8(p, head_dim, block_size, group, grid, st);
         return dtype == PKV_F32 ? pkv::launch_decode_partition_f32(p, head_dim, block_size, group, grid, st)
                                 : pkv::launch_decode_partition_bf16(p, head_dim, block_size, group, grid, st);

@@ -75,9 +75,10 @@ struct Unit {
     int s, g, part, ctx;  // ctx: the sequence's context length
 };
 
-__device__ __forceinline__ Unit decode_unit(const DecodeParams& p, bool partition_major) {
+// `Hkv` is the number of head units per sequence: the kv heads, or the kv
+// head pairs of the head_dim-64 tensor-core kernel (unit g = pair g).
+__device__ __forceinline__ Unit decode_unit(const DecodeParams& p, bool partition_major, int Hkv) {
     const int P = p.num_partitions;
-    const int Hkv = p.num_kv_heads;
     const long long bid = blockIdx.x;
     Unit u;
     if (p.order != nullptr) {
@@ -103,6 +104,10 @@ __device__ __forceinline__ Unit decode_unit(const DecodeParams& p, bool partitio
     else if (p.order == nullptr)
         u.ctx = p.context_lens[u.s];
     return u;
+}
+
+__device__ __forceinline__ Unit decode_unit(const DecodeParams& p, bool partition_major) {
+    return decode_unit(p, partition_major, p.num_kv_heads);
 }
 
 // Split-K merge, fused into the decode kernels: called by every thread of a

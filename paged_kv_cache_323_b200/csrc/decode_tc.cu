@@ -30,6 +30,8 @@ EncodeTiledFn encoder() {
 
 }  // namespace
 
+void* tc_tensor_map_encoder() { return reinterpret_cast<void*>(encoder()); }
+
 // The pool [num_blocks][Hkv][bs][128] as a 4-D tensor (dims innermost first:
 // dim, slot, kv head, block); boxes of one 128-byte row span (64 bf16 dims or
 // 128 e4m3 codes) x bs slots of one (block, kv head), 128-byte swizzle.
@@ -83,15 +85,19 @@ cudaError_t launch_group(const DecodeParams& p, int G, const CUtensorMap& mk, co
 
 }  // namespace
 
-bool decode_tc_supported(int kv_dtype, int D, int BS, int G, int partition_tokens) {
-    const bool shape = D == 128 && (BS == 8 || BS == 16 || BS == 32) && partition_tokens % 128 == 0;
-    if (kv_dtype == PKV_BF16) return shape && (G == 2 || G == 4 || G == 8);
-    if (kv_dtype == PKV_FP8_E4M3) return shape && (G == 1 || G == 2 || G == 4 || G == 8);
+bool decode_tc_supported(int kv_dtype, int D, int BS, int G, int Hkv, int partition_tokens) {
+    const bool bs = (BS == 8 || BS == 16 || BS == 32) && partition_tokens % 128 == 0;
+    if (kv_dtype == PKV_BF16) return bs && D == 128 && (G == 2 || G == 4 || G == 8);
+    if (kv_dtype == PKV_FP8_E4M3) {
+        if (D == 64) return bs && Hkv % 2 == 0 && (G == 1 || G == 2 || G == 4);  // kv head pairs
+        return bs && D == 128 && (G == 1 || G == 2 || G == 4 || G == 8);
+    }
     return false;
 }
 
-cudaError_t launch_decode_tc(const DecodeParams& p, int kv_dtype, int BS, int G, long long grid,
+cudaError_t launch_decode_tc(const DecodeParams& p, int kv_dtype, int D, int BS, int G, long long grid,
                              bool persistent, cudaStream_t st) {
+    if (kv_dtype == PKV_FP8_E4M3 && D == 64) return launch_decode_tc_fp8_d64(p, BS, G, st);
     const int eb = kv_dtype == PKV_FP8_E4M3 ? 1 : 2;
     CUtensorMap mk, mv;
     cudaError_t e = make_tc_pool_map(&mk, p.k_cache, p.num_kv_heads, BS, p.num_blocks, eb);

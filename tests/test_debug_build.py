@@ -52,11 +52,15 @@ cases = [
     ("tensor-core bf16 copy-on-write", wl.gqa_sampling(groups=3, prompt_median=300, prompt_max=1500), 256),
     ("tensor-core fp8 (persistent)", wl.custom(5, [1, 129, 640, 3000], heads=16, kv_heads=2,
                                               head_dim=128, block_size=16, dtype="fp8"), 512),
-    ("cuda-core fp8 head_dim 64", wl.custom(6, [5, 77, 900], heads=4, kv_heads=2, head_dim=64,
-                                           block_size=16, dtype="fp8"), 256),
+    ("tensor-core fp8 head_dim 64 (kv head pairs)", wl.custom(6, [5, 77, 900], heads=4, kv_heads=2,
+                                                              head_dim=64, block_size=16, dtype="fp8"), 256),
+    ("tensor-core fp8 head_dim 64, 4 heads per kv head, block size 32",
+     wl.custom(7, [5, 77, 900], heads=16, kv_heads=4, head_dim=64, block_size=32, dtype="fp8"), 256),
     ("cuda-core fp8 head_dim 64, 8 heads per kv head", wl.custom(8, [5, 77, 900], heads=16, kv_heads=2,
                                                                  head_dim=64, block_size=16,
                                                                  dtype="fp8"), 256),
+    ("cuda-core fp8 head_dim 64, odd kv heads", wl.custom(9, [5, 77, 900], heads=3, kv_heads=3,
+                                                          head_dim=64, block_size=16, dtype="fp8"), 256),
 ]
 for name, w, pt in cases:
     ref, kref, vref = oracle_step(w)
@@ -66,7 +70,7 @@ for name, w, pt in cases:
     line = pk.debug_failed_line()
     assert line == 0, f"{name}: index check failed at line {line}"
 pk._set_fp8_persistent(False)  # the fp8 tensor-core kernel with one CTA per unit
-name, w, pt = cases[4]
+name, w, pt = cases[4]  # the head_dim-128 fp8 case
 ref, kref, vref = oracle_step(w)
 out, kc, vc = gpu_step(w, partition_tokens=pt)
 assert_close(out, ref, "bf16", name + ", one CTA per unit")

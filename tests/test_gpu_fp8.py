@@ -47,7 +47,7 @@ def test_fp8_mha_full():
 
 def test_fp8_head_dim_64_full():
     """The batch-64 MHA step with head_dim 64 over an fp8 cache (the
-    CUDA-core kernel): every row."""
+    tensor-core kernel on kv head pairs): every row."""
     full_size_check(wl.mha(device="cuda", head_dim=64, dtype="fp8"))
 
 

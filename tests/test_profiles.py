@@ -17,7 +17,7 @@ FAMILY = {
     "mha": "cuda_core", "gqa_sampling": "tc_bf16", "long_context": "tc_bf16",
     "prefix_bs8": "tc_bf16", "prefix_bs16": "tc_bf16", "prefix_bs32": "tc_bf16",
     "mha_fp8": "tc_fp8", "gqa_sampling_fp8": "tc_fp8", "long_context_fp8": "tc_fp8",
-    "mha_d64_fp8": "cuda_core",
+    "mha_d64_fp8": "tc_fp8_d64",
 }
 
 
@@ -45,7 +45,8 @@ def test_traffic_file_matches_current_kernel_sources(path):
 @pytest.mark.parametrize("heads,kv_heads,dtype,head_dim,family", [
     (32, 32, "bf16", 128, "cuda_core"), (32, 8, "bf16", 128, "tc_bf16"), (64, 8, "bf16", 128, "tc_bf16"),
     (32, 32, "fp8", 128, "tc_fp8"), (32, 8, "fp8", 128, "tc_fp8"), (8, 8, "f32", 128, "cuda_core"),
-    (32, 32, "fp8", 64, "cuda_core"), (32, 8, "bf16", 64, "cuda_core"),
+    (32, 32, "fp8", 64, "tc_fp8_d64"), (32, 8, "fp8", 64, "tc_fp8_d64"), (6, 3, "fp8", 64, "cuda_core"),
+    (64, 8, "fp8", 64, "cuda_core"), (32, 8, "bf16", 64, "cuda_core"),
 ])
 def test_kernel_family_by_shape(heads, kv_heads, dtype, head_dim, family):
     w = wl.custom(1, [40, 7], heads=heads, kv_heads=kv_heads, head_dim=head_dim, block_size=16,
