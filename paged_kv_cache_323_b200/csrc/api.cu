@@ -186,12 +186,12 @@ size_t workspace_bytes_for(long long num_seqs, long long num_heads, long long pa
 //    of the maximum length would still be split into more than 64 partitions
 //    and the grid keeps at least four waves of 3 CTAs per SM.
 //  * Tensor-core kernels: 4096 tokens, halved (down to 512) while the grid
-//    would have fewer than 4 × 148 × 2 CTAs.  Their CTAs carry a
+//    would have fewer than min_ctas CTAs (4 × 148 × 2 unless given).  Their CTAs carry a
 //    fixed set-up and drain cost, so long partitions pay: on B200 the
 //    parallel-sampling GQA batch ran at 0.75 / 0.88 / 0.97 of peak with
 //    1024 / 2048 / 4096-token partitions.
 int auto_partition_tokens(long long num_seqs, long long num_kv_heads, long long max_ctx, bool tc,
-                          bool fp8 = false) {
+                          bool fp8 = false, long long min_ctas = 4LL * 148 * 2) {
     if (tc) {
         // The tensor-core kernels run 2 to 4 CTAs per SM, and a CTA's start
         // (table and q fetch, first TMA round trip) and merge are a fixed
@@ -200,7 +200,6 @@ int auto_partition_tokens(long long num_seqs, long long num_kv_heads, long long 
         // at 2048; the fp8 parallel-sampling batch at 4 CTAs per SM: 153 /
         // 171 / 209 us at 4096 / 2048 / 1024).
         long long pt = kMaxPartitionTokens;
-        const long long min_ctas = 4LL * 148 * 2;
         while (pt > kMinPartitionTokens && num_seqs * num_kv_heads * ((max_ctx + pt - 1) / pt) < min_ctas)
             pt /= 2;
         return (int)pt;
@@ -208,9 +207,9 @@ int auto_partition_tokens(long long num_seqs, long long num_kv_heads, long long 
     // fp8 caches carry half the bytes per token, so a CTA's fixed cost weighs
     // twice as much: 2048 tokens (on batch-64 MHA 154 us at 1024, 139 us at 2048)
     long long pt = fp8 ? 2 * kAutoPartitionTokens : kAutoPartitionTokens;
-    const long long min_ctas = 4LL * 148 * 3;
+    const long long min_cc_ctas = 4LL * 148 * 3;
     while (pt < kMaxPartitionTokens && (max_ctx + pt - 1) / pt > 64 &&
-           num_seqs * num_kv_heads * ((max_ctx + 2 * pt - 1) / (2 * pt)) >= min_ctas)
+           num_seqs * num_kv_heads * ((max_ctx + 2 * pt - 1) / (2 * pt)) >= min_cc_ctas)
         pt *= 2;
     return (int)pt;
 }
@@ -228,9 +227,14 @@ int resolve_partition_tokens(int num_seqs, int num_heads, int num_kv_heads, int 
     const int group = num_kv_heads > 0 ? num_heads / num_kv_heads : 1;
     const bool tc = tc_shape(dtype, head_dim, block_size, group, num_kv_heads);
     const bool fp8 = dtype == PKV_FP8_E4M3;
-    // the head_dim-64 tensor-core kernel runs one CTA per pair of kv heads
-    const int head_units = tc && head_dim == 64 ? num_kv_heads / 2 : num_kv_heads;
-    int pt = auto_partition_tokens(num_seqs, head_units, max_ctx, tc, fp8);
+    // The head_dim-64 tensor-core kernel runs one CTA per pair of kv heads,
+    // always in longest-first order, where the last CTAs to start are the
+    // shortest: its partitions stay long while the grid fills one wave of 5
+    // CTAs per SM (batch-64 MHA: 59.3 us at 2048 tokens, 68.4 at 1024, 76.1
+    // at 512).
+    const bool pairs = tc && head_dim == 64;
+    int pt = pairs ? auto_partition_tokens(num_seqs, num_kv_heads / 2, max_ctx, tc, fp8, 148LL * 5)
+                   : auto_partition_tokens(num_seqs, num_kv_heads, max_ctx, tc, fp8);
     // the persistent fp8 tensor-core kernel holds two tables of at most 128
     // blocks per CTA: 2048 tokens at block size 16 (batch-64 MHA 106.5 us at
     // 2048 against 112.1 us at 1024; the parallel-sampling batch 125.3 / 144.1)
@@ -371,8 +375,10 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
                             g_fp8_persistent.load() != 0 &&
                             pkv::decode_tc_fp8_persistent_supported(block_size, group, pt);
     const int sched = g_longest_first.load();
+    const bool pairs = use_tc && head_dim == 64;  // head_dim-64 kernel (batch-64 MHA 67.2 -> 59.3 us)
     const bool plan = workspace != nullptr &&
-                      (sched == 2 || (sched == 1 && (persistent || (use_tc && parts >= 2 && parts <= 4))));
+                      (sched == 2 ||
+                       (sched == 1 && (persistent || pairs || (use_tc && parts >= 2 && parts <= 4))));
     int2* order = plan ? reinterpret_cast<int2*>(wsb + wl.plan_off) : nullptr;
     p.order = order;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -39,6 +39,20 @@ cudaError_t make_tc_pool_map(CUtensorMap* map, const void* pool, int Hkv, int BS
                              int elem_bytes) {
     EncodeTiledFn fn = encoder();
     if (fn == nullptr) return cudaErrorNotSupported;
+    if (elem_bytes == 2 && BS == 8) {
+        // bf16, block size 8: one box per block, both 64-dim halves: dims
+        // (64 values, 8 slots at 256 B, 2 halves at 128 B, kv head, block),
+        // box (64, 8, 2, 1, 1) -> the block's 8 rows of the first half, then
+        // its 8 rows of the second
+        const cuuint64_t dims[5] = {64, 8, 2, (cuuint64_t)Hkv, (cuuint64_t)num_blocks};
+        const cuuint64_t strides[4] = {256, 128, 8 * 256, (cuuint64_t)Hkv * 8 * 256};
+        const cuuint32_t box[5] = {64, 8, 2, 1, 1};
+        const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+        const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(pool), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+    }
     const cuuint64_t eb = (cuuint64_t)elem_bytes;
     const cuuint64_t dims[4] = {128, (cuuint64_t)BS, (cuuint64_t)Hkv, (cuuint64_t)num_blocks};
     const cuuint64_t strides[3] = {128 * eb, (cuuint64_t)BS * 128 * eb, (cuuint64_t)Hkv * BS * 128 * eb};

@@ -55,6 +55,16 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
+__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                            int c3, int c4, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4),
+        "r"(smem_addr(bar))
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(dst)),
@@ -167,6 +177,16 @@ struct TcCfg {
     static constexpr int ROW = 128;          // bytes of one swizzled row (64 bf16)
     static constexpr int HALF = TILE * ROW;  // one 64-dim half of a K or V tile
     static constexpr int SLOT = 2 * HALF;    // one K or V tile (32 KB)
+    // Tile layout.  Block sizes 16 and 32: the first 64-dim half of all 128
+    // tokens, then the second (two copies per block, one per half).  Block
+    // size 8: one copy per block lands its 8 rows of the first half and then
+    // its 8 rows of the second (2 KB), so a chunk is 16 such pairs -- half
+    // the copies, which at 1 KB each had set the pace (~45 SM cycles per
+    // copy).  Either way token r's half h sits at
+    // (r / 8) * GSTRIDE + h * HSTEP + (r % 8) * ROW.
+    static constexpr bool IL = BS == 8;
+    static constexpr int HSTEP = IL ? 8 * ROW : HALF;        // offset of the second half
+    static constexpr int GSTRIDE = IL ? 16 * ROW : 8 * ROW;  // stride of 8-token groups
     static constexpr int NSLOT = 3;
     static constexpr int QB = 2 * NPAD * ROW;  // Q operand: 2 dim halves x 16 rows
     static constexpr int PB = 2 * NPAD * ROW;  // one P operand: 2 token halves x 16 rows
@@ -356,9 +376,13 @@ __global__ void __launch_bounds__(192, 2)
             }
             __syncwarp();  // the expected byte count is registered before any copy lands
             if (load) {
-                unsigned char* dst = smem + st * C::SLOT + lane * BS * C::ROW;
-                tma_load_4d(dst, map, 0, 0, g, e, &full[st]);
-                tma_load_4d(dst + C::HALF, map, 64, 0, g, e, &full[st]);
+                if constexpr (C::IL) {
+                    tma_load_5d(smem + st * C::SLOT + lane * 2 * BS * C::ROW, map, 0, 0, 0, g, e, &full[st]);
+                } else {
+                    unsigned char* dst = smem + st * C::SLOT + lane * BS * C::ROW;
+                    tma_load_4d(dst, map, 0, 0, g, e, &full[st]);
+                    tma_load_4d(dst + C::HALF, map, 64, 0, g, e, &full[st]);
+                }
             }
             issued = li + 1;
         }
@@ -380,7 +404,7 @@ __global__ void __launch_bounds__(192, 2)
                 const uint32_t k_base = smem_addr(smem + st * C::SLOT);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t a = sw128_desc(k_base + (kk >> 2) * C::HALF + (kk & 3) * 32, 16, 1024);
+                    const uint64_t a = sw128_desc(k_base + (kk >> 2) * C::HSTEP + (kk & 3) * 32, 16, C::GSTRIDE);
                     const uint64_t b = sw128_desc(q_base + (kk >> 2) * (C::NPAD * C::ROW) + (kk & 3) * 32, 16, 1024);
                     mma_kind_f16(tmem + C::S_COL + (c & 1) * 16, a, b, C::IDESC_QK, kk > 0);
                 }
@@ -399,8 +423,9 @@ __global__ void __launch_bounds__(192, 2)
                 const uint32_t p_base = smem_addr(smem + C::P_OFF + (c & 1) * C::PB);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    // A = V^T, MN-major: 64-dim halves C::HALF apart, 8-token groups 1024 B apart
-                    const uint64_t a = sw128_desc(v_base + kk * 16 * C::ROW, C::HALF, 1024);
+                    // A = V^T, MN-major: 64-dim halves HSTEP apart, 8-token groups
+                    // GSTRIDE apart, 16 tokens (two groups) per step
+                    const uint64_t a = sw128_desc(v_base + kk * 2 * C::GSTRIDE, C::HSTEP, C::GSTRIDE);
                     const uint64_t b = sw128_desc(p_base + (kk >> 2) * (C::NPAD * C::ROW) + (kk & 3) * 32, 16, 1024);
                     mma_kind_f16(tmem + C::O_COL + (c & 1) * 16, a, b, C::IDESC_PV, kk > 0);
                 }
@@ -499,8 +524,9 @@ __global__ void __launch_bounds__(192, 2)
                     break;
                 }
                 if (!valid) {
-                    uint4* row0 = reinterpret_cast<uint4*>(smem + st * C::SLOT + r * C::ROW);
-                    uint4* row1 = reinterpret_cast<uint4*>(smem + st * C::SLOT + C::HALF + r * C::ROW);
+                    unsigned char* row = smem + st * C::SLOT + (r >> 3) * C::GSTRIDE + (r & 7) * C::ROW;
+                    uint4* row0 = reinterpret_cast<uint4*>(row);
+                    uint4* row1 = reinterpret_cast<uint4*>(row + C::HSTEP);
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         row0[k] = make_uint4(0u, 0u, 0u, 0u);

@@ -100,16 +100,6 @@ __device__ __forceinline__ uint64_t sw64_desc(uint32_t saddr, uint32_t lbo, uint
     return d;
 }
 
-__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
-                                            int c3, int c4, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_addr(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4),
-        "r"(smem_addr(bar))
-        : "memory");
-}
-
 template <int BS, int G>
 __global__ void __launch_bounds__(192, TcFp8D64Cfg<BS, G>::CTAS_PER_SM)
     decode_tc_fp8_d64_kernel(const __grid_constant__ DecodeParams p,

@@ -144,8 +144,9 @@ def test_partition_tokens(pk):
     assert pt(64, 32, 32, 128, 16, 2048, f8, 0) == 2048
     assert pt(8, 64, 8, 128, 32, 131072, f8, 0) == 4096
     assert pt(64, 32, 32, 128, 8, 2048, f8, 0) == 1024
-    # head_dim 64: one CTA per pair of kv heads, partitions halved until 4 waves
-    assert pt(64, 32, 32, 64, 16, 2048, f8, 0) == 1024
+    # head_dim 64: one CTA per pair of kv heads, partitions halved until one wave
+    assert pt(64, 32, 32, 64, 16, 2048, f8, 0) == 4096
+    assert pt(8, 32, 32, 64, 16, 2048, f8, 0) == 512
     prev = pk._set_fp8_persistent(False)
     try:
         assert pt(64, 32, 32, 128, 16, 2048, f8, 0) == 4096  # one CTA per unit
