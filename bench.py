@@ -125,7 +125,7 @@ KERNEL_SOURCES = {
     "cuda_core": ("common.cuh", "decode_common.cuh", "decode_attn.cuh", "decode_launch.cuh"),
     "tc_bf16": ("common.cuh", "decode_common.cuh", "decode_tc.cuh", "decode_tc.cu"),
     "tc_fp8": ("common.cuh", "decode_common.cuh", "decode_tc.cuh", "decode_tc_fp8.cuh", "decode_tc_fp8p.cuh",
-               "decode_tc_fp8p.cu", "plan.cuh"),
+               "decode_tc_fp8p.cu", "persist.cuh", "plan.cuh"),
     "tc_fp8_d64": ("common.cuh", "decode_common.cuh", "decode_tc.cuh", "decode_tc_fp8.cuh", "decode_tc_fp8_d64.cuh",
                    "decode_tc_fp8_d64.cu", "plan.cuh"),
 }
