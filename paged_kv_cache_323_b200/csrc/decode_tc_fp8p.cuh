@@ -212,8 +212,6 @@ __global__ void __launch_bounds__(192, TcFp8PCfg<BS, G>::CTAS_PER_SM)
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    // a schedule is written by the planning grid this launch follows
-    if (p.order != nullptr) asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (tid == 0) {
         for (int i = 0; i < C::NSLOT; ++i) {
@@ -266,6 +264,9 @@ __global__ void __launch_bounds__(192, TcFp8PCfg<BS, G>::CTAS_PER_SM)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
+        // The queue follows the schedule the planning grid writes; only this
+        // warp reads it (the others' set-up above overlaps the plan).
+        if (p.order != nullptr) asm volatile("griddepcontrol.wait;" ::: "memory");
         for (int k = 0;; ++k) {
             const int rec = k & 1;
             // the next unit with work; units with nothing to attend are settled here
@@ -660,6 +661,7 @@ __global__ void __launch_bounds__(192, TcFp8PCfg<BS, G>::CTAS_PER_SM)
     if (aborted) {
         // every unit this CTA took and did not finish, then every unit left in
         // the queue, takes its turn on its merge counter with an empty partial
+        if (p.order != nullptr) asm volatile("griddepcontrol.wait;" ::: "memory");
         const int first = *units_done, published = *units_published;
         const int orphan = *fetched_unit;
         __syncthreads();
