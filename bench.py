@@ -431,7 +431,9 @@ def run_reference(args, world, rank):
 # Configurations measured beside the headline in the default run: the
 # parallel-sampling GQA batch, the long-context split-K batch and the
 # prefix-sharing block-size sweep.
-DEFAULT_CONFIGS = ("gqa_sampling", "long_context", "prefix_bs8", "prefix_bs16", "prefix_bs32")
+# configs 3-5, then the block-size-8 MHA step and the fp8-cache rows (the quantised cache)
+DEFAULT_CONFIGS = ("gqa_sampling", "long_context", "prefix_bs8", "prefix_bs16", "prefix_bs32", "mha_bs8",
+                   "mha_fp8", "gqa_sampling_fp8", "mha_d64_fp8")
 L2_FLUSH_BYTES = 512 << 20  # written before each cold step: four times the 126 MB L2
 
 

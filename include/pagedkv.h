@@ -130,9 +130,11 @@ PKV_API int paged_attention_decode(void* out, const void* q, const void* k_cache
  *                     paged_attention_workspace_size(num_seqs, num_heads,
  *                     max_blocks_per_seq*block_size, head_dim, partition_tokens)
  *                     bytes, 256-byte aligned, owned by the caller.  It holds
- *                     one split-K merge counter per (sequence, kv head) at its
- *                     start, in a region nothing else uses, then the launch's
- *                     schedule, then the partial results of split sequences.
+ *                     at its start, in a region nothing else uses, the work
+ *                     queue of the persistent fp8 kernel (64 bytes) and one
+ *                     split-K merge counter per (sequence, kv head); then the
+ *                     launch's schedule, then the partial results of split
+ *                     sequences.
  *                     The schedule, where one is planned (see
  *                     pkv_set_longest_first), orders the grid's (sequence,
  *                     partition) units longest first; a one-CTA planning
@@ -141,14 +143,16 @@ PKV_API int paged_attention_decode(void* out, const void* q, const void* k_cache
  *                     a unit and when, never the arithmetic, so outputs are
  *                     the same bits with or without it.  Zero-fill the workspace (e.g.
  *                     cudaMemset) once before its first use.  Every call
- *                     leaves the counters it used at zero again -- a call
+ *                     leaves the queue and the counters it used at zero
+ *                     again -- a call
  *                     whose kernel stopped on PKV_ERR_TIMEOUT too -- so the
  *                     same buffer serves later calls of any shape without
  *                     clearing.  (A batch of more than 65536 (sequence, kv
  *                     head) units also uses counters past that region; the
  *                     call clears those itself, on `stream`, before its
  *                     kernel.)  When no sequence is split, workspace may be
- *                     NULL: the grid then runs in index order, unplanned.  Two
+ *                     NULL: the grid then runs in index order, unplanned, one
+ *                     CTA per (sequence, kv head, partition).  Two
  *                     calls in flight at once must not share a workspace.
  */
 PKV_API int paged_attention_decode_ex(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -160,7 +164,8 @@ PKV_API int paged_attention_decode_ex(void* out, const void* q, const void* k_ca
 
 /* Partition size (tokens per CTA) paged_attention_decode_ex uses for these
  * arguments: partition_tokens itself, or the automatic choice when it is 0
- * (which depends on the kernel that serves the shape).  0 on bad sizes. */
+ * (which depends on the kernel that serves the shape, and is at most 128
+ * blocks where the persistent fp8 kernel serves it).  0 on bad sizes. */
 PKV_API int paged_attention_partition_tokens(int num_seqs, int num_heads, int num_kv_heads,
                                              int head_dim, int block_size, int max_context,
                                              int dtype, int partition_tokens);
@@ -172,12 +177,17 @@ PKV_API int paged_attention_partition_tokens(int num_seqs, int num_heads, int nu
  * pools hold fp8 e4m3 codes; one float scale per kv head (device arrays
  * k_scales, v_scales [num_kv_heads]) gives the stored value code * scale.  q
  * and out are bf16.  Otherwise exactly paged_attention_decode_ex (same
- * workspace, partitions, faults).  With head_dim 128 and 1, 2, 4 or 8 query
- * heads per kv head (and partitions a multiple of 128 tokens) the tensor-core
- * kernel serves it: both products on e4m3 tensor cores over the codes as
- * they land, q and the probabilities each split into two e4m3 terms that
- * keep 8 significant bits; otherwise the CUDA-core kernel, widening each
- * code.  Either reads half the bytes of a bf16 cache per token.
+ * workspace, partitions, faults).  Tensor-core kernels serve it (both
+ * products on e4m3 tensor cores over the codes as they land, q and the
+ * probabilities each split into two e4m3 terms that keep 8 significant bits;
+ * partitions a multiple of 128 tokens) with head_dim 128 and 1, 2, 4 or 8
+ * query heads per kv head -- with a workspace and up to 4 heads in
+ * persistent form (one CTA per SM slot taking units from the workspace's
+ * queue, longest first; partitions of at most 128 blocks) -- and with
+ * head_dim 64, 1, 2 or 4 query heads per kv head and an even number of kv
+ * heads (one CTA per pair of kv heads).  Other shapes run on the CUDA-core
+ * kernel, widening each code.  Every kernel reads half the bytes of a bf16
+ * cache per token.
  */
 PKV_API int paged_attention_decode_fp8(void* out, const void* q, const void* k_cache,
                                        const void* v_cache, const float* k_scales,
@@ -335,9 +345,10 @@ PKV_API int pkv_profile_enable(int on);
 PKV_API int pkv_profile_read(int kind, long long* launches, double* total_ms);
 PKV_API int pkv_profile_reset(void);
 
-/* Choose the decode kernel where a tensor-core one applies (head_dim 128,
- * partitions a multiple of 128 tokens; bf16 caches with 2, 4 or 8 query heads
- * per kv head, fp8 caches with 1, 2, 4 or 8): 1 (default) runs the
+/* Choose the decode kernel where a tensor-core one applies (partitions a
+ * multiple of 128 tokens; head_dim 128 with bf16 caches and 2, 4 or 8 query
+ * heads per kv head, or fp8 caches and 1, 2, 4 or 8; head_dim 64 with fp8
+ * caches, 1, 2 or 4 and an even number of kv heads): 1 (default) runs the
  * tensor-core kernel (tcgen05 MMAs into tensor memory), 0 the CUDA-core
  * kernel that serves every other shape.  Both compute the same attention;
  * returns the previous setting.  Process-wide. */
@@ -347,7 +358,9 @@ PKV_API int pkv_set_tensor_core_gqa(int enable);
  * paged_attention_decode_ex): 1 (default) plans longest first where that
  * pays -- the tensor-core kernels with 2 to 4 partitions per sequence, whose
  * index order would leave the partitions only long sequences have for the
- * end of the launch -- and runs every other launch in index order; 2 plans
+ * end of the launch, the persistent fp8 kernel, whose queue then hands out
+ * the shortest units last, and the head_dim-64 fp8 kernel -- and runs every
+ * other launch in index order; 2 plans
  * every launch; 0 none.  All give the same bits; only the time differs.
  * Process-wide; returns the previous mode, or PKV_ERR_INVALID. */
 PKV_API int pkv_set_longest_first(int mode);
