@@ -118,9 +118,14 @@ __device__ __forceinline__ Unit decode_unit(const DecodeParams& p, bool partitio
 // partitions in partition order:
 //     M = max_i m_i,  L = sum_i 2^(m_i - M) l_i,  out = sum_i 2^(m_i - M) o_i / L.
 // `scratch` is shared memory of at least merge_scratch_bytes<G, D, NTHREADS>().
+// The partitions are split over thread groups of a fixed 128-thread budget
+// (kMergeLanes), whatever the caller's thread count, so every kernel -- one
+// CTA per unit or persistent -- sums them in the same order and gives the
+// same bits.
+constexpr int kMergeLanes = 128;
 template <int G, int D, int NTHREADS>
 constexpr int merge_scratch_bytes() {
-    return ((2 * G + 3) / 4) * 16 + (NTHREADS > G * D / 4 ? NTHREADS : G * D / 4) * 16;
+    return ((2 * G + 3) / 4) * 16 + (kMergeLanes > G * D / 4 ? kMergeLanes : G * D / 4) * 16;
 }
 
 // The merge itself, for the NTHREADS threads that call it: tid is the
@@ -176,7 +181,7 @@ __device__ __forceinline__ bool fused_merge_with(const DecodeParams& p, int s, i
     // out = sum_i 2^(m_i - M) o_i / L, partitions split over thread groups
     constexpr int COLS = D / 4;
     constexpr int UNITS = G * COLS;
-    constexpr int GROUPS = NTHREADS / UNITS > 0 ? NTHREADS / UNITS : 1;
+    constexpr int GROUPS = kMergeLanes / UNITS > 0 ? kMergeLanes / UNITS : 1;
     float4* acc_s = reinterpret_cast<float4*>(scratch + ((2 * G + 3) / 4) * 4);  // [GROUPS][UNITS]
     for (int u = tid; u < GROUPS * UNITS; u += NTHREADS) {
         const int unit = u % UNITS;

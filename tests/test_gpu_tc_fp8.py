@@ -135,15 +135,18 @@ def test_tc_fp8_group8_bs32_long_partitions(tc_mode, pt):
 
 
 
-@pytest.mark.parametrize("bs,pt", [(16, 128), (16, 1024), (16, 2048), (8, 1024), (32, 4096)])
-def test_tc_fp8_persistent_same_bits(bs, pt):
+@pytest.mark.parametrize("G,bs,pt", [(4, 16, 128), (4, 16, 1024), (4, 16, 2048), (4, 8, 1024), (4, 32, 4096),
+                                     (1, 16, 256), (2, 16, 512)])
+def test_tc_fp8_persistent_same_bits(G, bs, pt):
     """The persistent form computes every unit with the same arithmetic in
-    the same order as the one-CTA-per-unit kernel, so the outputs are
-    identical bit for bit under every schedule, launch after launch on one
-    workspace (the queue is back at zero after each launch)."""
+    the same order as the one-CTA-per-unit kernel -- the split-K merge's
+    partition order included, which does not depend on how many threads run
+    it -- so the outputs are identical bit for bit under every schedule,
+    launch after launch on one workspace (the queue is back at zero after
+    each launch)."""
     from paged_kv_cache_323_b200 import pagedkv as pk
 
-    w = wl.custom(71, [1, 130, 700, 2049, 4500, 0, 3000, 129], heads=16, kv_heads=4, head_dim=128,
+    w = wl.custom(71, [1, 130, 700, 2049, 4500, 0, 3000, 129], heads=4 * G, kv_heads=4, head_dim=128,
                   block_size=bs, dtype="fp8")
     ref, _, _ = oracle_step(w)
     t = to_device(w)
