@@ -9,11 +9,11 @@
 namespace pkv {
 namespace {
 
-template <int BS, int G>
-cudaError_t launch_inst(const DecodeParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
-                        long long units, cudaStream_t st) {
+template <int BS, int G, bool FW>
+cudaError_t launch_fw(const DecodeParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
+                      long long units, cudaStream_t st) {
     using C = tc::TcFp8PCfg<BS, G>;
-    auto kern = tc::decode_tc_fp8_persistent_kernel<BS, G>;
+    auto kern = tc::decode_tc_fp8_persistent_kernel<BS, G, FW>;
     static std::atomic<unsigned long long> configured{0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -33,6 +33,15 @@ cudaError_t launch_inst(const DecodeParams& p, const CUtensorMap& mk, const CUte
     const long long grid = units < slots ? units : slots;
     return launch_decode_kernel(kern, static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, st,
                                 p.order != nullptr, p, mk, mv);
+}
+
+// Launches whose sequences each fit one partition start a first wave in
+// index order without waiting for the schedule (decode_tc_fp8p.cuh).
+template <int BS, int G>
+cudaError_t launch_inst(const DecodeParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
+                        long long units, cudaStream_t st) {
+    return p.num_partitions == 1 ? launch_fw<BS, G, true>(p, mk, mv, units, st)
+                                 : launch_fw<BS, G, false>(p, mk, mv, units, st);
 }
 
 template <int BS>

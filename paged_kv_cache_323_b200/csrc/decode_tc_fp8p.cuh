@@ -169,7 +169,8 @@ __device__ __forceinline__ void build_q_warp(const DecodeParams& p, int s, int g
     }
 }
 
-template <int BS, int G>
+// FIRST_WAVE: the launch's sequences each fit one partition (see the producer)
+template <int BS, int G, bool FIRST_WAVE>
 __global__ void __launch_bounds__(192, TcFp8PCfg<BS, G>::CTAS_PER_SM)
     decode_tc_fp8_persistent_kernel(const __grid_constant__ DecodeParams p,
                                     const __grid_constant__ CUtensorMap tmk,
@@ -184,6 +185,7 @@ __global__ void __launch_bounds__(192, TcFp8PCfg<BS, G>::CTAS_PER_SM)
     const int PTOK = p.partition_tokens;
     const int max_ctx = p.max_blocks_per_seq * BS;
     const int num_units = p.num_seqs * p.num_kv_heads * P;
+    constexpr bool first_wave = FIRST_WAVE;  // see the producer
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
     uint64_t* full = bars;
@@ -264,19 +266,41 @@ __global__ void __launch_bounds__(192, TcFp8PCfg<BS, G>::CTAS_PER_SM)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        // The queue follows the schedule the planning grid writes; only this
-        // warp reads it (the others' set-up above overlaps the plan).
-        if (p.order != nullptr) asm volatile("griddepcontrol.wait;" ::: "memory");
+        // The first wave (launches where every sequence fits one partition):
+        // CTA b's first unit is unit b in index order, taken at once.  Every
+        // later unit comes from the queue, which follows the schedule the
+        // planning grid writes (longest first) and skips the first wave's
+        // units; so the plan runs while the first wave streams, and the units
+        // handed out last are still the shortest (batch-64 MHA: 106.5 ->
+        // 101.7 us).  With several partitions per sequence the index order
+        // would start the short last partitions ahead of long ones (the
+        // parallel-sampling batch lost 2 %): there every unit comes from the
+        // queue.  Only this warp reads the schedule.
+        bool first_pending = first_wave, plan_seen = false;
         for (int k = 0;; ++k) {
             const int rec = k & 1;
-            // the next unit with work; units with nothing to attend are settled here
+            // the next unit with work (its index-order id); units with nothing
+            // to attend are settled here
             int u = -1, s = 0, g = 0, part = 0, ctx = 0, nparts = 0;
             for (;;) {
-                int cand = 0;
-                if (lane == 0) cand = atomicAdd(p.work, 1);
-                cand = __shfl_sync(0xffffffffu, cand, 0);
-                if (cand >= num_units) break;
-                if (!queue_unit(p, cand, s, g, part)) continue;
+                int idx;
+                if (first_pending) {
+                    first_pending = false;
+                    idx = (int)blockIdx.x;  // the grid never has more CTAs than units
+                    index_unit(p, idx, s, g, part);
+                } else {
+                    if (!plan_seen) {
+                        if (p.order != nullptr) asm volatile("griddepcontrol.wait;" ::: "memory");
+                        plan_seen = true;
+                    }
+                    int cand = 0;
+                    if (lane == 0) cand = atomicAdd(p.work, 1);
+                    cand = __shfl_sync(0xffffffffu, cand, 0);
+                    if (cand >= num_units) break;
+                    if (!queue_unit(p, cand, s, g, part)) continue;
+                    idx = unit_index(p, s, g, part);
+                    if (first_wave && idx < (int)gridDim.x) continue;  // a first-wave unit: its CTA has it
+                }
                 ctx = p.context_lens[s];
                 if (ctx < 0 || ctx > max_ctx) {
                     if (part == 0) {
@@ -291,7 +315,7 @@ __global__ void __launch_bounds__(192, TcFp8PCfg<BS, G>::CTAS_PER_SM)
                         zero_rows_warp<G>(p, (long long)s * p.num_heads + (long long)g * G, lane);
                     continue;
                 }
-                u = cand;
+                u = idx;
                 break;
             }
             if (lane == 0) *fetched_unit = u;
@@ -663,16 +687,26 @@ __global__ void __launch_bounds__(192, TcFp8PCfg<BS, G>::CTAS_PER_SM)
         // the queue, takes its turn on its merge counter with an empty partial
         if (p.order != nullptr) asm volatile("griddepcontrol.wait;" ::: "memory");
         const int first = *units_done, published = *units_published;
-        const int orphan = *fetched_unit;
+        const int orphan = *fetched_unit;  // index-order id, or -1
         __syncthreads();
         for (int k = first; k < published; ++k) {
             const int* R = recs + (k & 1) * C::REC_INTS;
             abort_merge_turn<T, D, G>(p, R[1], R[2], (long long)R[1] * p.num_heads + (long long)R[2] * G,
                                       R[3], R[4], last_flag);
         }
-        for (int u = orphan;;) {
-            int s, g, part;
-            if (u >= 0 && u < num_units && queue_unit(p, u, s, g, part)) {
+        // first the unit taken and not published, then the queue's entries
+        // (whose first-wave units their own CTAs settle)
+        for (int u = orphan, from_queue = 0;;) {
+            int s = 0, g = 0, part = 0;
+            bool take = false;
+            if (from_queue) {
+                take = u < num_units && queue_unit(p, u, s, g, part) &&
+                       !(first_wave && unit_index(p, s, g, part) < (int)gridDim.x);
+            } else if (u >= 0 && u < num_units) {
+                index_unit(p, u, s, g, part);
+                take = true;
+            }
+            if (take) {
                 const int ctx = p.context_lens[s];
                 const bool bad = ctx < 0 || ctx > max_ctx;
                 const int nparts = bad ? 0 : (ctx + PTOK - 1) / PTOK;
@@ -686,6 +720,7 @@ __global__ void __launch_bounds__(192, TcFp8PCfg<BS, G>::CTAS_PER_SM)
             if (tid == 0) *queue_entry = atomicAdd(p.work, 1);
             __syncthreads();
             u = *queue_entry;
+            from_queue = 1;
             if (u >= num_units) break;
         }
     }

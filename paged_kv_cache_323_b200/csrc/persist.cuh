@@ -27,6 +27,18 @@ __device__ __forceinline__ bool queue_unit(const DecodeParams& p, int u, int& s,
     return PKV_DCHECK(p.err, s >= 0 && s < p.num_seqs && part >= 0 && part < P);
 }
 
+// A unit's index in index order (partition fastest), and back.
+__device__ __forceinline__ int unit_index(const DecodeParams& p, int s, int g, int part) {
+    return (s * p.num_kv_heads + g) * p.num_partitions + part;
+}
+
+__device__ __forceinline__ void index_unit(const DecodeParams& p, int idx, int& s, int& g, int& part) {
+    const int P = p.num_partitions;
+    part = idx % P;
+    g = (idx / P) % p.num_kv_heads;
+    s = idx / (P * p.num_kv_heads);
+}
+
 // Zero G output rows from row sh0 with the lanes of one warp.
 template <int G>
 __device__ __forceinline__ void zero_rows_warp(const DecodeParams& p, long long sh0, int lane) {

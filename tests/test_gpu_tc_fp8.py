@@ -135,9 +135,14 @@ def test_tc_fp8_group8_bs32_long_partitions(tc_mode, pt):
 
 
 
-@pytest.mark.parametrize("G,bs,pt", [(4, 16, 128), (4, 16, 1024), (4, 16, 2048), (4, 8, 1024), (4, 32, 4096),
-                                     (1, 16, 256), (2, 16, 512)])
-def test_tc_fp8_persistent_same_bits(G, bs, pt):
+@pytest.mark.parametrize("G,bs,pt,lens", [
+    (4, 16, 128, None), (4, 16, 1024, None), (4, 16, 2048, None), (4, 8, 1024, None), (4, 32, 4096, None),
+    (1, 16, 256, None), (2, 16, 512, None),
+    # every sequence in one partition: the first wave takes units in index order, the queue the rest
+    (1, 16, 2048, [1, 130, 700, 2048, 1500, 0, 2000, 129] * 40),
+    (4, 16, 2048, [1, 130, 700, 2048, 1500, 0, 2000, 129] * 3),
+])
+def test_tc_fp8_persistent_same_bits(G, bs, pt, lens):
     """The persistent form computes every unit with the same arithmetic in
     the same order as the one-CTA-per-unit kernel -- the split-K merge's
     partition order included, which does not depend on how many threads run
@@ -146,8 +151,12 @@ def test_tc_fp8_persistent_same_bits(G, bs, pt):
     each launch)."""
     from paged_kv_cache_323_b200 import pagedkv as pk
 
-    w = wl.custom(71, [1, 130, 700, 2049, 4500, 0, 3000, 129], heads=4 * G, kv_heads=4, head_dim=128,
-                  block_size=bs, dtype="fp8")
+    if lens is None:
+        w = wl.custom(71, [1, 130, 700, 2049, 4500, 0, 3000, 129], heads=4 * G, kv_heads=4, head_dim=128,
+                      block_size=bs, dtype="fp8")
+    else:
+        w = wl.custom(71, lens, heads=4 * G, kv_heads=4, head_dim=128, block_size=bs, dtype="fp8",
+                      maxb=pt // bs)
     ref, _, _ = oracle_step(w)
     t = to_device(w)
     ks = torch.from_numpy(w.k_scales).cuda()

@@ -27,6 +27,9 @@ KERNELS = {
     "tensor_core_fp8": (lambda: wl.mha(num_seqs=8, num_blocks=2048, dtype="fp8"), 512),
     # the same in persistent form: a stopped CTA also drains the work queue
     "tensor_core_fp8_persistent": (lambda: wl.mha(num_seqs=8, num_blocks=2048, dtype="fp8"), 512),
+    # persistent, one partition per sequence: first-wave units in index order, the rest queued
+    "tensor_core_fp8_persistent_one_partition": (lambda: wl.mha(num_seqs=64, num_blocks=16384, dtype="fp8"),
+                                                 2048),
     # head_dim 64 over an fp8 cache: one CTA per pair of kv heads
     "tensor_core_fp8_d64": (lambda: wl.mha(num_seqs=8, num_blocks=2048, head_dim=64, dtype="fp8"), 512),
 }
