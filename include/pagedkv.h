@@ -221,7 +221,11 @@ PKV_API size_t paged_attention_workspace_size(int num_seqs, int num_heads, int m
  * for every kv head g.  k and v are [num_tokens][num_kv_heads][head_dim];
  * slot_mapping is int64 [num_tokens]; -1 means "skip".  The copy is bit-exact.
  * Slots >= num_blocks*bs are device faults (not written).  Two tokens must not
- * name the same slot.
+ * name the same slot.  The append's kernel releases a kernel launched next
+ * as a programmatic dependent at once (this library's decode kernels are
+ * launched so, and wait for the append to finish before they read
+ * anything); a caller's own kernel launched that way after it must likewise
+ * wait (griddepcontrol.wait) before it reads the pools.
  */
 PKV_API int kv_cache_append(void* k_cache, void* v_cache, const void* k, const void* v,
                     const int64_t* slot_mapping, int num_tokens, int num_kv_heads, int head_dim,

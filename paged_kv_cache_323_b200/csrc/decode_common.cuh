@@ -45,13 +45,13 @@ struct DecodeParams {
     unsigned long long wait_ns;
 };
 
-// Launch a decode kernel.  When the launch follows a planning grid
-// (p.order set), it is a programmatic dependent launch: its CTAs may start
-// while the plan still runs and wait for it in decode_unit.
+// Launch a decode kernel, as a programmatic dependent launch when `pdl`: its
+// CTAs may start while the preceding grid (the planning grid, or the append
+// of the same step, which releases its dependents at once) still runs, and
+// wait for it (griddepcontrol.wait) before they read anything.
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_decode_kernel(void (*kern)(KArgs...), unsigned grid, unsigned threads,
-                                        size_t smem, cudaStream_t st, bool after_plan,
-                                        Args&&... args) {
+                                        size_t smem, cudaStream_t st, bool pdl, Args&&... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(threads);
@@ -61,14 +61,14 @@ inline cudaError_t launch_decode_kernel(void (*kern)(KArgs...), unsigned grid, u
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = after_plan ? 1 : 0;
+    cfg.numAttrs = pdl ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
-// Which (sequence, kv head, partition) this CTA runs.  With a schedule
-// (p.order) the CTA first waits for the planning grid that wrote it (a no-op
-// without one in flight), then takes pair order[b / Hkv] and kv head
-// b % Hkv.  Without one: partition fastest, or, when `partition_major` (the
+// Which (sequence, kv head, partition) this CTA runs.  The CTA first waits
+// for the grid its launch depends on (the planning grid or the step's
+// append; a no-op when the launch depends on none), then, with a schedule
+// (p.order), takes pair order[b / Hkv] and kv head b % Hkv.  Without one: partition fastest, or, when `partition_major` (the
 // tensor-core kernels with at most 4 partitions per sequence), all first
 // partitions, then all second ones, and so on.
 struct Unit {
@@ -81,8 +81,8 @@ __device__ __forceinline__ Unit decode_unit(const DecodeParams& p, bool partitio
     const int P = p.num_partitions;
     const long long bid = blockIdx.x;
     Unit u;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (p.order != nullptr) {
-        asm volatile("griddepcontrol.wait;" ::: "memory");
         const int2 e = p.order[bid / Hkv];
         u.g = (int)(bid % Hkv);
         u.s = e.x / P;

@@ -25,8 +25,8 @@ cudaError_t launch_partition_inst(const DecodeParams& p, long long grid, cudaStr
         if (e != cudaSuccess) return e;
         configured.fetch_or(bit);
     }
-    return launch_decode_kernel(kern, static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, st,
-                                p.order != nullptr, p);
+    // every CTA waits for the preceding grid in decode_unit
+    return launch_decode_kernel(kern, static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, st, true, p);
 }
 
 template <typename T, typename TKV, int D, int BS>

@@ -23,8 +23,9 @@ cudaError_t launch_inst(const DecodeParams& p, const CUtensorMap& mk, const CUte
         if (e != cudaSuccess) return e;
         configured.fetch_or(bit);
     }
-    return launch_decode_kernel(kern, static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, st,
-                                p.order != nullptr, p, mk, mv);
+    // one CTA per unit: every CTA waits for the preceding grid in decode_unit
+    return launch_decode_kernel(kern, static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, st, true, p,
+                                mk, mv);
 }
 
 template <int BS>

@@ -36,6 +36,9 @@ struct AppendParams {
 // rows, one thread per 16-byte chunk.  The new token's K and V chunks are
 // loaded before the slot is known, so the only dependent step is the store.
 __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
+    // a decode launched next as a programmatic dependent may start now; it
+    // waits for this grid to finish before it reads the pools
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int cpr = p.chunks_per_row;
     const int rows_per_cta = blockDim.x / cpr;
     const int r_in = threadIdx.x / cpr;
@@ -109,6 +112,7 @@ __device__ __forceinline__ uint4 quantise16(const uint4 a, const uint4 b, float 
 }
 
 __global__ void __launch_bounds__(256) kv_append_fp8_kernel(const AppendFp8Params p) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // as in kv_append_kernel
     const int cpr = p.chunks_per_row;
     const int rows_per_cta = blockDim.x / cpr;
     const int r_in = threadIdx.x / cpr;
