@@ -187,3 +187,51 @@ def test_tc_fp8_persistent_same_bits(G, bs, pt, lens):
     for o in outs[1:]:
         assert torch.equal(o, outs[0])
     assert int(ws[:8].view(torch.int32).abs().sum()) == 0  # queue counters back at zero
+
+
+def test_tc_fp8_bad_context_zero_rows(tc_mode):
+    """A context length past the table: that sequence's rows are zero and
+    the error word says so; every other row still matches the oracle (in
+    the persistent form the producer settles such units from the queue)."""
+    pk = tc_mode
+    w = wl.custom(91, [300, 700, 129, 1000, 64], heads=8, kv_heads=4, head_dim=128, block_size=16,
+                  dtype="fp8")
+    ref, _, _ = oracle_step(w)
+    t = to_device(w)
+    t["context_lens"][2] = w.max_blocks_per_seq * w.block_size + 1
+    out, _, _ = gpu_step(w, t, partition_tokens=256, check_error=False)
+    assert pk.get_device_error() == pk.PKV_ERR_DEVICE_BOUNDS
+    assert torch.count_nonzero(out[2]) == 0
+    keep = [0, 1, 3, 4]
+    assert_close(out[keep], ref[keep], "bf16")
+
+
+def test_tc_fp8_many_units_twice(tc_mode):
+    """More (sequence, kv head) units than the workspace's fixed counter
+    region holds (65536), split into partitions, twice on one workspace:
+    the counters past the region are cleared per call and both calls match
+    the oracle."""
+    pk = tc_mode
+    rng = np.random.default_rng(5)
+    # mostly short sequences (the pool stays near 1 GB), a fifth long enough to split
+    lens = np.where(rng.random(2100) < 0.8, rng.integers(1, 65, size=2100),
+                    rng.integers(129, 300, size=2100)).tolist()
+    w = wl.custom(93, lens, heads=32, kv_heads=32, head_dim=128, block_size=16, dtype="fp8")
+    assert w.num_seqs * w.num_kv_heads > 65536
+    ref, _, _ = oracle_step(w)
+    t = to_device(w)
+    ks = torch.from_numpy(w.k_scales).cuda()
+    vs = torch.from_numpy(w.v_scales).cuda()
+    pk.kv_cache_append_fp8(t["k_cache"], t["v_cache"], ks, vs, t["k_new"], t["v_new"], t["slot_mapping"])
+    pt = 128
+    need = pk.paged_attention_workspace_size(w.num_seqs, w.num_heads, w.max_blocks_per_seq * w.block_size,
+                                             w.head_dim, pt)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        t["out"].fill_(float("nan"))
+        pk.paged_attention_decode_fp8(t["out"], t["q"], t["k_cache"], t["v_cache"], ks, vs,
+                                      t["block_tables"], t["context_lens"], w.scale,
+                                      num_blocks=w.num_blocks, partition_tokens=pt, workspace=ws)
+        torch.cuda.synchronize()
+        assert pk.get_device_error() == 0
+        assert_close(t["out"], ref, "bf16")
