@@ -128,6 +128,7 @@ KERNEL_SOURCES = {
                "decode_tc_fp8p.cu", "persist.cuh", "plan.cuh"),
     "tc_fp8_d64": ("common.cuh", "decode_common.cuh", "decode_tc.cuh", "decode_tc_fp8.cuh", "decode_tc_fp8_d64.cuh",
                    "decode_tc_fp8_d64.cu", "plan.cuh"),
+    "reg": ("common.cuh", "decode_common.cuh", "decode_attn.cuh", "decode_reg.cuh", "decode_reg.cu"),
 }
 
 
@@ -141,6 +142,8 @@ def decode_kernel_family(w) -> str:
         return "tc_fp8_d64"
     if w.head_dim == 128 and w.dtype == "bf16" and group in (2, 4, 8):
         return "tc_bf16"
+    if w.head_dim == 128 and w.dtype == "bf16" and group == 1 and w.block_size == 8:
+        return "reg"
     return "cuda_core"
 
 

@@ -22,7 +22,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpagedkv.so")
 LIB_DEBUG = os.path.join(PKG, "libpagedkv_debug.so")
 SOURCES = ["api.cu", "decode_f32.cu", "decode_bf16.cu", "decode_fp8.cu", "decode_tc.cu", "decode_tc_fp8.cu",
-           "decode_tc_fp8p.cu", "decode_tc_fp8_d64.cu",
+           "decode_tc_fp8p.cu", "decode_tc_fp8_d64.cu", "decode_reg.cu",
            "noalloc.cu",
            "block_manager.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -47,6 +47,8 @@ std::atomic<int> g_tc_gqa{1};  // tensor-core kernel for grouped-query heads whe
 std::atomic<int> g_longest_first{1};
 // fp8 tensor-core decode in persistent form where a workspace holds its queue
 std::atomic<int> g_fp8_persistent{1};
+// register-streamed kernel for bf16 MHA over 8-token blocks (else the staged one)
+std::atomic<int> g_reg_stream{1};
 std::atomic<unsigned long long> g_launches{0};
 std::atomic<unsigned long long> g_wait_ns{pkv::kWaitTimeoutNs};  // decode pipeline wait limit
 
@@ -331,6 +333,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     const long long parts = (max_ctx + pt - 1) / pt;
     const bool use_tc = g_tc_gqa.load() != 0 &&
                         pkv::decode_tc_supported(kv_dtype, head_dim, block_size, group, num_kv_heads, pt);
+    const bool use_reg = !use_tc && g_reg_stream.load() != 0 &&
+                         pkv::decode_reg_supported(kv_dtype, head_dim, block_size, group);
     const long long grid = parts * num_kv_heads * (long long)num_seqs;
     if (grid > INT_MAX || (long long)num_seqs * num_heads > INT_MAX) return PKV_ERR_INVALID;
     const size_t need = workspace_bytes_for(num_seqs, num_heads, parts, head_dim);
@@ -413,6 +417,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
         }
         if (use_tc)
             return pkv::launch_decode_tc(p, kv_dtype, head_dim, block_size, group, grid, persistent, st);
+        if (use_reg) return pkv::launch_decode_reg(p, head_dim, block_size, group, grid, st);
         if (fp8) return pkv::launch_decode_partition_fp8(p, head_dim, block_size, group, grid, st);
         return dtype == PKV_F32 ? pkv::launch_decode_partition_f32(p, head_dim, block_size, group, grid, st)
                                 : pkv::launch_decode_partition_bf16(p, head_dim, block_size, group, grid, st);
@@ -784,6 +789,10 @@ int pkv_set_longest_first(int mode) {
 
 PKV_API int pkv_internal_set_fp8_persistent(int enable) {
     return g_fp8_persistent.exchange(enable != 0 ? 1 : 0);
+}
+
+PKV_API int pkv_internal_set_reg_stream(int enable) {
+    return g_reg_stream.exchange(enable != 0 ? 1 : 0);
 }
 
 int pkv_set_tensor_core_gqa(int enable) {

@@ -16,6 +16,11 @@ cudaError_t launch_decode_partition_bf16(const DecodeParams& p, int D, int BS, i
 cudaError_t launch_decode_partition_fp8(const DecodeParams& p, int D, int BS, int G,
                                         long long grid, cudaStream_t st);
 
+// bf16 MHA over 8-token blocks, head_dim 128: K and V streamed through
+// registers with plain loads instead of staged copies
+bool decode_reg_supported(int kv_dtype, int D, int BS, int G);
+cudaError_t launch_decode_reg(const DecodeParams& p, int D, int BS, int G, long long grid, cudaStream_t st);
+
 // Tensor-core (tcgen05) kernels, partitions a multiple of 128 tokens: bf16
 // caches with head_dim 128 and groups of 2, 4 or 8 query heads; fp8 (e4m3)
 // caches with head_dim 128 and groups of 1, 2, 4 or 8, or head_dim 64, an

@@ -96,6 +96,8 @@ for _name, (_res, _args) in SIGNATURES.items():
 # not in the header: selects the fp8 tensor-core decode's persistent form
 lib.pkv_internal_set_fp8_persistent.restype = _I
 lib.pkv_internal_set_fp8_persistent.argtypes = [_I]
+lib.pkv_internal_set_reg_stream.restype = _I
+lib.pkv_internal_set_reg_stream.argtypes = [_I]
 
 
 class PagedKVError(RuntimeError):
@@ -571,6 +573,13 @@ def _set_fp8_persistent(enable: bool) -> bool:
     most 128 blocks -- or one CTA per unit (False).  Returns the previous
     setting."""
     return bool(lib.pkv_internal_set_fp8_persistent(1 if enable else 0))
+
+
+def _set_reg_stream(enable: bool) -> bool:
+    """bf16 MHA decode over 8-token blocks with K and V streamed through
+    registers (the default) or staged in shared memory by bulk copies
+    (False).  Returns the previous setting."""
+    return bool(lib.pkv_internal_set_reg_stream(1 if enable else 0))
 
 
 def set_longest_first(mode: int) -> int:

@@ -52,3 +52,9 @@ def test_kernel_family_by_shape(heads, kv_heads, dtype, head_dim, family):
     w = wl.custom(1, [40, 7], heads=heads, kv_heads=kv_heads, head_dim=head_dim, block_size=16,
                   dtype=dtype)
     assert bench.decode_kernel_family(w) == family
+
+
+@pytest.mark.parametrize("bs,family", [(8, "reg"), (16, "cuda_core"), (32, "cuda_core")])
+def test_kernel_family_bf16_mha_by_block_size(bs, family):
+    w = wl.custom(1, [40, 7], heads=8, kv_heads=8, head_dim=128, block_size=bs, dtype="bf16")
+    assert bench.decode_kernel_family(w) == family
