@@ -132,18 +132,20 @@ KERNEL_SOURCES = {
 }
 
 
-def decode_kernel_family(w) -> str:
+def decode_kernel_family(w, tensor_cores: bool = True) -> str:
     """Which decode kernel the library runs for this workload (tensor-core
-    kernels on, as by default)."""
+    kernels on, as by default, or off)."""
     group = w.num_heads // w.num_kv_heads
+    if w.head_dim == 128 and w.dtype == "bf16" and group == 1:
+        return "reg"
+    if not tensor_cores:
+        return "cuda_core"
     if w.head_dim == 128 and w.dtype == "fp8" and group in (1, 2, 4, 8):
         return "tc_fp8"
     if w.head_dim == 64 and w.dtype == "fp8" and group in (1, 2, 4) and w.num_kv_heads % 2 == 0:
         return "tc_fp8_d64"
     if w.head_dim == 128 and w.dtype == "bf16" and group in (2, 4, 8):
         return "tc_bf16"
-    if w.head_dim == 128 and w.dtype == "bf16" and group == 1 and w.block_size == 8:
-        return "reg"
     return "cuda_core"
 
 
@@ -745,7 +747,8 @@ def run_gpu(args, world, rank, local):
     roofline = None
     if part:
         achieved = kv_bytes / (part["avg_us"] * 1e-6) / 1e9
-        traffic = committed_traffic("decode", args.workload, kernel_source_sha(decode_kernel_family(w)))
+        fam = decode_kernel_family(w, not args.cuda_cores)
+        traffic = committed_traffic("decode", args.workload, kernel_source_sha(fam))
         roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                     "frac": achieved / peak, "traffic": traffic,
                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
@@ -763,7 +766,7 @@ def run_gpu(args, world, rank, local):
                    "accumulate": "f32",
                    "schedule": {0: "index order", 1: "longest first where it pays",
                                 2: "longest first"}[args.schedule],
-                   "kernel": "cuda_core" if args.cuda_cores else decode_kernel_family(w),
+                   "kernel": decode_kernel_family(w, not args.cuda_cores),
                    "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush; "
                          "step_us_cold_l2 flushes L2 before each step",
                    "parallelism": f"{world} independent batches, one per GPU"},

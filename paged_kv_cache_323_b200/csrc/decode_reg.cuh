@@ -4,22 +4,24 @@
 // Same computation as decode_attn.cuh ("PagedAttention Explained: Virtual
 // Memory for the KV Cache", section "How PagedAttention works", item 5: the
 // kernel follows the block table and gathers each block's keys and values),
-// for one query head per kv head, bf16 caches and 8-token blocks:
+// for one query head per kv head and bf16 caches:
 //     out[s][h] = softmax(scale * q[s][h] . K_s^T) V_s
 //
 // Why a second form: at block size 8 a (block, kv head) slice of K is 2 KB.
 // Staging such slices through shared memory costs one asynchronous copy each
 // (bulk copy, or sixteen 16-byte cp.async per warp), and at that size the
 // per-copy cost, not HBM, set the pace of the staged kernel.  Here each warp
-// reads its blocks with plain 16-byte loads straight into registers:
+// reads the cache with plain 16-byte loads straight into registers:
 //  * One CTA per (sequence, kv head, partition), NW warps.  The partition's
 //    table entries are read once into shared memory and range-checked.
-//  * Warp w takes the partition's blocks w, w + NW, w + 2 NW, ...  A block's
-//    K (and V) slice is BS rows of D values; lane l loads the 16-byte chunk
+//  * The partition is cut into chunks of 8 tokens (a whole block at block
+//    size 8, an 8-row-aligned run of a larger block: 2 KB of K and
+//    2 KB of V, contiguous in the [block][kv head][slot][dim] pool).  Warp w
+//    takes chunks w, w + NW, w + 2 NW, ...; lane l loads the 16-byte piece
 //    l % 16 of rows l / 16, l / 16 + 2, ... (one warp-wide load covers 512
-//    contiguous bytes).  The next block's K and V loads are issued before the
-//    current block is computed (two register buffers), so every warp keeps a
-//    whole block in flight while it works.
+//    contiguous bytes).  The next chunk's K and V loads are issued before the
+//    current chunk is computed (two register buffers), so every warp keeps a
+//    whole chunk in flight while it works.
 //  * Partial dot products over a lane's 8 dims are reduced by the transposing
 //    butterfly of decode_attn.cuh; online softmax in base 2 with fp32 running
 //    max and sum; PV into fp32 registers (8 dims per lane).  Unused slots of
@@ -40,9 +42,11 @@ namespace pkv {
 
 template <int D, int BS, int NW>
 struct RegCfg {
-    static constexpr int CPR = D / 8;        // 16-byte chunks (8 bf16) per row
+    static constexpr int CPR = D / 8;        // 16-byte pieces (8 bf16) per row
     static constexpr int RPI = 32 / CPR;     // rows covered by one warp-wide load
-    static constexpr int RPL = BS / RPI;     // rows per lane per block
+    static constexpr int RW = 8;             // rows (tokens) per chunk
+    static constexpr int CPB = BS / RW;      // chunks per block
+    static constexpr int RPL = RW / RPI;     // rows per lane per chunk
     static constexpr int THREADS = NW * 32;
     static constexpr int ROWB = D * 2;       // bytes of one token row
     static constexpr int SLICE = BS * ROWB;  // bytes of one (block, kv head)
@@ -51,7 +55,7 @@ struct RegCfg {
     static constexpr int SCRATCH_FLOATS = merge_scratch_bytes<1, D, THREADS>() / 4;
 
     static_assert(D % 8 == 0 && CPR <= 32 && 32 % CPR == 0, "head_dim chunking");
-    static_assert(BS % RPI == 0 && RPL >= 1 && RPL <= CPR, "rows per lane");
+    static_assert(BS % RW == 0 && RW % RPI == 0 && RPL >= 1 && RPL <= CPR, "rows per lane");
 };
 
 // 16 bytes of the cache, read once: no L1 allocation.
@@ -94,6 +98,7 @@ __global__ void __launch_bounds__(NW * 32, MINB) decode_reg_kernel(const DecodeP
     const int tok0 = part * PT;
     const int tok1 = min(ctx, tok0 + PT);
     const int nblk = (tok1 - tok0 + BS - 1) / BS;
+    const int nchk = (tok1 - tok0 + C::RW - 1) / C::RW;
     const int blk0 = tok0 / BS;
 
     const int tid = threadIdx.x;
@@ -109,8 +114,8 @@ __global__ void __launch_bounds__(NW * 32, MINB) decode_reg_kernel(const DecodeP
         phys[j] = e;
     }
 
-    const int c = lane % C::CPR;  // this lane's 16-byte chunk of a row
-    const int r0 = lane / C::CPR;  // its first row of a block
+    const int c = lane % C::CPR;  // this lane's 16-byte piece of a row
+    const int r0 = lane / C::CPR;  // its first row of a chunk
     float qf[8];
     {
         const uint4 qr = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) + sh0 * D + c * 8);
@@ -127,11 +132,11 @@ __global__ void __launch_bounds__(NW * 32, MINB) decode_reg_kernel(const DecodeP
     const long long pool_bytes = (long long)p.num_blocks * slice_stride;  // debug checks
     (void)pool_bytes;
 
-    // block j of the partition into registers (zeros for a skipped block)
-    auto load = [&](int j, uint4 (&kr)[C::RPL], uint4 (&vr)[C::RPL]) {
-        const int e = j < nblk ? phys[j] : -1;
-        const long long off = (long long)e * slice_stride;
-        if (e >= 0 && PKV_DCHECK(p.err, off + (long long)g * C::SLICE + C::SLICE <= pool_bytes)) {
+    // chunk q of the partition into registers (zeros for a skipped block)
+    auto load = [&](int q, uint4 (&kr)[C::RPL], uint4 (&vr)[C::RPL]) {
+        const int e = q < nchk ? phys[q / C::CPB] : -1;
+        const long long off = (long long)e * slice_stride + (q % C::CPB) * (C::RW * C::ROWB);
+        if (e >= 0 && PKV_DCHECK(p.err, off + (long long)g * C::SLICE + C::RW * C::ROWB <= pool_bytes)) {
 #pragma unroll
             for (int k = 0; k < C::RPL; ++k) {
                 kr[k] = ld_kv_stream(kbase + off + k * C::RPI * C::ROWB);
@@ -152,9 +157,9 @@ __global__ void __launch_bounds__(NW * 32, MINB) decode_reg_kernel(const DecodeP
     const int vi = c / SPREAD;
     const bool l_owner = c % SPREAD == 0;
 
-    auto compute = [&](int j, const uint4 (&kr)[C::RPL], const uint4 (&vr)[C::RPL]) {
-        if (phys[j] < 0) return;  // out-of-range entry: skipped, error already set
-        const int nvalid = min(BS, tok1 - (tok0 + j * BS));
+    auto compute = [&](int q, const uint4 (&kr)[C::RPL], const uint4 (&vr)[C::RPL]) {
+        if (phys[q / C::CPB] < 0) return;  // out-of-range entry: skipped, error already set
+        const int nvalid = min(C::RW, tok1 - (tok0 + q * C::RW));
         float sc[C::RPL];
 #pragma unroll
         for (int k = 0; k < C::RPL; ++k) {
@@ -191,16 +196,16 @@ __global__ void __launch_bounds__(NW * 32, MINB) decode_reg_kernel(const DecodeP
 
     {
         uint4 ka[C::RPL], va[C::RPL], kb[C::RPL], vb[C::RPL];
-        int j = warp;
-        load(j, ka, va);
-        while (j < nblk) {
-            load(j + NW, kb, vb);
-            compute(j, ka, va);
-            j += NW;
-            if (j >= nblk) break;
-            load(j + NW, ka, va);
-            compute(j, kb, vb);
-            j += NW;
+        int q = warp;
+        load(q, ka, va);
+        while (q < nchk) {
+            load(q + NW, kb, vb);
+            compute(q, ka, va);
+            q += NW;
+            if (q >= nchk) break;
+            load(q + NW, ka, va);
+            compute(q, kb, vb);
+            q += NW;
         }
     }
 

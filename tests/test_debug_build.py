@@ -4,8 +4,9 @@ a device sanitizer.
 
 On the CPU: it compiles for sm_100a, loads, exports every symbol the header
 declares, and says which build it is.  On the GPU: one step of every kernel
-family (CUDA-core decode at block sizes 8 / 16 / 32 over fp32, bf16 and fp8
-caches, the tensor-core decode over bf16 and fp8 caches, split-K with the
+family (the register-streamed bf16 MHA decode, the staged CUDA-core decode at
+block sizes 8 / 16 / 32 over fp32, bf16 and fp8 caches, the tensor-core
+decode over bf16 and fp8 caches, split-K with the
 fused merge, the longest-first schedule, the fp8 tensor-core kernel in both
 forms, the no-alloc entry, append and
 copy-on-write) runs through the debug library in a child process, matches
@@ -45,8 +46,8 @@ from steps import gpu_step, oracle_step, assert_close, assert_pool_equal, to_dev
 assert pk.DEBUG and pk.lib.pkv_debug_build() == 1
 pk.set_longest_first(2)  # plan every launch, so the schedule's checks run too
 cases = [
-    ("cuda-core bs8 split-K", wl.mha(num_seqs=6, num_blocks=1200, heads=4, block_size=8), 256),
-    ("cuda-core bs16", wl.mha(num_seqs=6, num_blocks=600, heads=4), 0),
+    ("register-streamed bs8 split-K", wl.mha(num_seqs=6, num_blocks=1200, heads=4, block_size=8), 256),
+    ("register-streamed bs16", wl.mha(num_seqs=6, num_blocks=600, heads=4), 0),
     ("cuda-core bs32 fp32", wl.custom(3, [1, 31, 33, 700], heads=4, kv_heads=2, head_dim=64,
                                      block_size=32, dtype="f32"), 128),
     ("tensor-core bf16 copy-on-write", wl.gqa_sampling(groups=3, prompt_median=300, prompt_max=1500), 256),
@@ -76,6 +77,13 @@ out, kc, vc = gpu_step(w, partition_tokens=pt)
 assert_close(out, ref, "bf16", name + ", one CTA per unit")
 assert pk.debug_failed_line() == 0, "one CTA per unit: index check failed"
 pk._set_fp8_persistent(True)
+pk._set_reg_stream(False)  # bf16 MHA on the staged kernel (bulk copies into shared memory)
+for name, w, pt in cases[:2]:
+    ref, _, _ = oracle_step(w)
+    out, _, _ = gpu_step(w, partition_tokens=pt)
+    assert_close(out, ref, w.dtype, name + ", staged")
+    assert pk.debug_failed_line() == 0, name + ", staged: index check failed"
+pk._set_reg_stream(True)
 w = wl.mha(num_seqs=8, num_blocks=2048)
 ref, _, _ = oracle_step(w)
 t = to_device(w)

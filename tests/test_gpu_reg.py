@@ -1,6 +1,6 @@
-"""The register-streamed decode kernel (bf16 MHA over 8-token blocks, head_dim
-128) against the oracle, and the staged kernel it replaces on the same
-inputs ("How PagedAttention works", items 2-5: the kernel walks the block
+"""The register-streamed decode kernel (bf16 MHA, head_dim 128, blocks of 8,
+16 or 32 tokens read in 8-token chunks) against the oracle, and the staged
+kernel on the same inputs ("How PagedAttention works", items 2-5: the kernel walks the block
 table and gathers each block's keys and values wherever they sit).
 
 Both forms meet the bf16 bar on every case; the register form is the
@@ -29,14 +29,16 @@ def form(request):
     pk._set_reg_stream(prev)
 
 
-@pytest.mark.parametrize("pt", [0, 8, 24, 64, 256, 4096])
-def test_edge_lengths(form, pt):
+@pytest.mark.parametrize("bs,pt", [(8, 0), (8, 8), (8, 24), (8, 64), (8, 256), (8, 4096),
+                                   (16, 0), (16, 16), (16, 48), (16, 4096), (32, 0), (32, 32), (32, 96)])
+def test_edge_lengths(form, bs, pt):
     """Empty (zero row), one token, one short of / exactly / one past a
-    block, ragged tails, the table's maximum context; partitions from one
-    block (8 tokens) to the 4096-token maximum."""
-    maxb = 160
-    lens = [0, 1, 7, 8, 9, 15, 16, 17, 100, 1000, maxb * 8, 5, 1279, 63]
-    w = wl.custom(21, lens, heads=4, kv_heads=4, head_dim=128, block_size=8, dtype="bf16", maxb=maxb)
+    chunk and a block, ragged tails, the table's maximum context; partitions
+    from one block to the 4096-token maximum."""
+    maxb = 1280 // bs
+    lens = [0, 1, 7, 8, 9, 15, 16, 17, 31, 33, 100, 1000, maxb * bs, 5, 1279, 63]
+    w = wl.custom(21 + bs, lens, heads=4, kv_heads=4, head_dim=128, block_size=bs, dtype="bf16",
+                  maxb=maxb)
     ref, kref, vref = oracle_step(w)
     out, kc, vc = gpu_step(w, partition_tokens=pt)
     assert_pool_equal(kc, kref, "k pool")
@@ -45,20 +47,22 @@ def test_edge_lengths(form, pt):
     assert torch.count_nonzero(out[0]) == 0
 
 
-def test_reduced_batch(form):
+@pytest.mark.parametrize("bs", [8, 16, 32])
+def test_reduced_batch(form, bs):
     """A batch-64-like MHA batch cut to 8 sequences, several partitions."""
-    w = wl.mha(num_seqs=8, num_blocks=4096, heads=8, block_size=8)
+    w = wl.mha(num_seqs=8, num_blocks=32768 // bs, heads=8, block_size=bs)
     ref, _, _ = oracle_step(w)
     for pt in (0, 128, 512):
         out, _, _ = gpu_step(w, partition_tokens=pt)
         assert_close(out, ref, "bf16", what=f"partition {pt}")
 
 
-def test_nan_poisoned_unused_slots(form):
+@pytest.mark.parametrize("bs", [8, 16, 32])
+def test_nan_poisoned_unused_slots(form, bs):
     """Unused slots and blocks past each context hold NaN: outputs stay
     finite and match the oracle, so nothing outside the context is read
     into the result."""
-    w = wl.mha(num_seqs=6, num_blocks=1800, heads=4, block_size=8, ctx_range=(1, 700))
+    w = wl.mha(num_seqs=6, num_blocks=14400 // bs, heads=4, block_size=bs, ctx_range=(1, 700))
     bs = w.block_size
     used = np.zeros((w.num_blocks, bs), dtype=bool)
     for s in range(w.num_seqs):
@@ -77,10 +81,11 @@ def test_nan_poisoned_unused_slots(form):
         assert_close(out, ref, "bf16", what=f"partition {pt}")
 
 
-def test_permutation_bit_identical(form):
+@pytest.mark.parametrize("bs", [8, 16])
+def test_permutation_bit_identical(form, bs):
     """Moving blocks (data and table together) leaves the output
     bit-identical: the reduction order is logical."""
-    w = wl.mha(num_seqs=6, num_blocks=1200, heads=8, block_size=8)
+    w = wl.mha(num_seqs=6, num_blocks=9600 // bs, heads=8, block_size=bs)
     out1, _, _ = gpu_step(w, partition_tokens=256)
     perm = np.random.default_rng(9).permutation(w.num_blocks)
     w2 = wl.Workload(**{**w.__dict__})
@@ -111,21 +116,22 @@ def test_schedule_does_not_change_bits(form):
     assert torch.equal(outs[0], outs[1])
 
 
-def test_bad_table_entry_sets_error(form):
+@pytest.mark.parametrize("bs", [8, 32])
+def test_bad_table_entry_sets_error(form, bs):
     """An entry past the pool sets the error word; its block is skipped and
     the outputs stay finite."""
     from paged_kv_cache_323_b200 import pagedkv as pk
 
-    w = wl.mha(num_seqs=3, num_blocks=800, heads=4, block_size=8)
+    w = wl.mha(num_seqs=3, num_blocks=6400 // bs, heads=4, block_size=bs)
     w.block_tables[1, 2] = w.num_blocks + 7
     out, _, _ = gpu_step(w, check_error=False)
     assert pk.get_device_error() == pk.PKV_ERR_DEVICE_BOUNDS
     assert torch.isfinite(out.float()).all()
 
 
-@pytest.mark.parametrize("contiguous", [False, True], ids=["paged", "contiguous"])
-def test_full_size(form, contiguous):
-    """Batch-64 MHA at block size 8 (32 = 32 heads, contexts U[128, 2048],
-    pool of 32768 blocks): all 64 x 32 rows, paged and contiguous
-    placement."""
-    full_size_check(wl.mha(block_size=8, contiguous=contiguous, device="cuda"))
+@pytest.mark.parametrize("bs,contiguous", [(8, False), (8, True), (16, False), (32, False)],
+                         ids=["bs8", "bs8_contiguous", "bs16", "bs32"])
+def test_full_size(form, bs, contiguous):
+    """Batch-64 MHA (32 = 32 heads, contexts U[128, 2048], a pool of 256 Ki
+    tokens): all 64 x 32 rows, paged and contiguous placement."""
+    full_size_check(wl.mha(block_size=bs, contiguous=contiguous, device="cuda"))

@@ -19,7 +19,9 @@ from steps import assert_close, oracle_step, to_device
 pytestmark = pytest.mark.gpu
 
 KERNELS = {
-    # batch-64-like MHA on the CUDA-core kernel, 4 partitions per long sequence
+    # batch-64-like MHA on the staged CUDA-core kernel (bulk copies and
+    # mbarrier waits; the register-streamed kernel that serves this shape by
+    # default has no waits), 4 partitions per long sequence
     "cuda_core": (lambda: wl.mha(num_seqs=8, num_blocks=2048), 512),
     # grouped-query heads on the tensor-core kernel, several partitions
     "tensor_core": (lambda: wl.gqa_sampling(groups=4, prompt_median=600, prompt_max=3000), 256),
@@ -90,10 +92,12 @@ def test_timeout_then_parity_on_the_same_workspace(kernel):
 
     make, pt = KERNELS[kernel]
     prev = pk._set_fp8_persistent(kernel != "tensor_core_fp8")
+    prev_reg = pk._set_reg_stream(False)
     try:
         _timeout_then_parity(pk, make(), pt)
     finally:
         pk._set_fp8_persistent(prev)
+        pk._set_reg_stream(prev_reg)
 
 
 def _timeout_then_parity(pk, w, pt):
@@ -126,16 +130,45 @@ def test_timeout_then_parity_library_workspace():
         pk.paged_attention_decode(t["out"], t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
                                   t["context_lens"], w.scale)
 
-    plain()  # the library's workspace for this stream exists before the timeout
-    torch.cuda.synchronize()
-    assert pk.get_device_error() == 0
-    _time_out(pk, plain)
-    for _ in range(2):
-        t["out"].fill_(float("nan"))
-        plain()
+    prev_reg = pk._set_reg_stream(False)  # the staged kernel, which waits on its copies
+    try:
+        plain()  # the library's workspace for this stream exists before the timeout
         torch.cuda.synchronize()
         assert pk.get_device_error() == 0
-        assert_close(t["out"], ref, w.dtype)
+        _time_out(pk, plain)
+        for _ in range(2):
+            t["out"].fill_(float("nan"))
+            plain()
+            torch.cuda.synchronize()
+            assert pk.get_device_error() == 0
+            assert_close(t["out"], ref, w.dtype)
+    finally:
+        pk._set_reg_stream(prev_reg)
+
+
+def test_register_kernel_has_no_waits():
+    """The register-streamed kernel (bf16 MHA) loads straight into registers
+    and waits on nothing: with the 1 us limit its launches never report a
+    timeout and still match the oracle."""
+    from paged_kv_cache_323_b200 import pagedkv as pk
+
+    w = wl.mha(num_seqs=8, num_blocks=2048)
+    ref, _, _ = oracle_step(w)
+    t = _appended(pk, w)
+    need = pk.paged_attention_workspace_size(w.num_seqs, w.num_heads,
+                                             w.max_blocks_per_seq * w.block_size, w.head_dim, 512)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    assert pk.get_device_error() == 0
+    prev = pk.set_wait_limit_us(1)
+    try:
+        for _ in range(3):
+            t["out"].fill_(float("nan"))
+            _decode(pk, w, t, 512, ws)
+            torch.cuda.synchronize()
+            assert pk.get_device_error() == 0
+            assert_close(t["out"], ref, w.dtype)
+    finally:
+        pk.set_wait_limit_us(0)
 
 
 def _shapes():

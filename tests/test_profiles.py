@@ -14,10 +14,10 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 # which decode kernel serves each bench workload (by shape and cache type)
 FAMILY = {
-    "mha": "cuda_core", "gqa_sampling": "tc_bf16", "long_context": "tc_bf16",
+    "mha": "reg", "gqa_sampling": "tc_bf16", "long_context": "tc_bf16",
     "prefix_bs8": "tc_bf16", "prefix_bs16": "tc_bf16", "prefix_bs32": "tc_bf16",
     "mha_fp8": "tc_fp8", "gqa_sampling_fp8": "tc_fp8", "long_context_fp8": "tc_fp8",
-    "mha_d64_fp8": "tc_fp8_d64",
+    "mha_d64_fp8": "tc_fp8_d64", "mha_bs8": "reg",
 }
 
 
@@ -43,7 +43,7 @@ def test_traffic_file_matches_current_kernel_sources(path):
 
 
 @pytest.mark.parametrize("heads,kv_heads,dtype,head_dim,family", [
-    (32, 32, "bf16", 128, "cuda_core"), (32, 8, "bf16", 128, "tc_bf16"), (64, 8, "bf16", 128, "tc_bf16"),
+    (32, 32, "bf16", 128, "reg"), (32, 8, "bf16", 128, "tc_bf16"), (64, 8, "bf16", 128, "tc_bf16"),
     (32, 32, "fp8", 128, "tc_fp8"), (32, 8, "fp8", 128, "tc_fp8"), (8, 8, "f32", 128, "cuda_core"),
     (32, 32, "fp8", 64, "tc_fp8_d64"), (32, 8, "fp8", 64, "tc_fp8_d64"), (6, 3, "fp8", 64, "cuda_core"),
     (64, 8, "fp8", 64, "cuda_core"), (32, 8, "bf16", 64, "cuda_core"),
@@ -54,7 +54,9 @@ def test_kernel_family_by_shape(heads, kv_heads, dtype, head_dim, family):
     assert bench.decode_kernel_family(w) == family
 
 
-@pytest.mark.parametrize("bs,family", [(8, "reg"), (16, "cuda_core"), (32, "cuda_core")])
-def test_kernel_family_bf16_mha_by_block_size(bs, family):
-    w = wl.custom(1, [40, 7], heads=8, kv_heads=8, head_dim=128, block_size=bs, dtype="bf16")
+@pytest.mark.parametrize("bs,D,dtype,family", [(8, 128, "bf16", "reg"), (16, 128, "bf16", "reg"),
+                                              (32, 128, "bf16", "reg"), (16, 64, "bf16", "cuda_core"),
+                                              (8, 128, "f32", "cuda_core")])
+def test_kernel_family_mha_by_block_size(bs, D, dtype, family):
+    w = wl.custom(1, [40, 7], heads=8, kv_heads=8, head_dim=D, block_size=bs, dtype=dtype)
     assert bench.decode_kernel_family(w) == family
