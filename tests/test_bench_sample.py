@@ -58,7 +58,8 @@ def test_pick_sample_bounds_the_work():
 
 
 def test_rows_match_bar():
-    """The bench's per-row parity verdict applies the spec bars."""
+    """The bench's per-row parity verdict applies the parity bars: bf16
+    2e-2 + 1e-2 |ref| elementwise, fp32 1e-5 absolute, never a NaN."""
     import torch
 
     ref = np.zeros((2, 3, 4))
