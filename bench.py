@@ -70,7 +70,10 @@ WORKLOADS = {
                          lambda dev, seed: wl.gqa_sampling(seed=seed, device=dev, dtype="fp8")),
     "long_context_fp8": ("long_context_b8_h64_kv8_d128_bs32_ctxU32768-131072_fp8e4m3_cache",
                          lambda dev, seed: wl.long_context(seed=seed, device=dev, dtype="fp8")),
-    # head_dim 64 over an fp8 cache (the CUDA-core kernel)
+    # head_dim 64, bf16 cache (the register-streamed kernel)
+    "mha_d64": ("mha_decode_b64_h32_kv32_d64_bs16_ctxU128-2048_bf16",
+                lambda dev, seed: wl.mha(seed=seed, device=dev, head_dim=64)),
+    # head_dim 64 over an fp8 cache (the tensor-core kernel on kv head pairs)
     "mha_d64_fp8": ("mha_decode_b64_h32_kv32_d64_bs16_ctxU128-2048_fp8e4m3_cache",
                     lambda dev, seed: wl.mha(seed=seed, device=dev, head_dim=64, dtype="fp8")),
     "mha_d64_fp8_small": ("mha_decode_b16_h32_kv32_d64_bs16_ctxU128-2048_fp8e4m3_cache_pool4096",
@@ -87,7 +90,7 @@ DEFAULT_SEED = {"mha": 2, "gqa_sampling": 3, "long_context": 4, "prefix_bs8": 5,
                 "prefix_bs32": 5, "tiny": 1, "mha_small": 2, "mha_bs8": 2, "mha_bs32": 2,
                 "mha_contig_bs8": 2, "mha_contig_bs16": 2, "mha_contig_bs32": 2, "mha_fp8": 2,
                 "mha_fp8_small": 2, "mha_bs8_small": 2, "gqa_sampling_fp8": 3, "long_context_fp8": 4,
-                "mha_d64_fp8": 2, "mha_d64_fp8_small": 2}
+                "mha_d64_fp8": 2, "mha_d64_fp8_small": 2, "mha_d64": 2}
 
 
 def measured_peak():
@@ -136,7 +139,7 @@ def decode_kernel_family(w, tensor_cores: bool = True) -> str:
     """Which decode kernel the library runs for this workload (tensor-core
     kernels on, as by default, or off)."""
     group = w.num_heads // w.num_kv_heads
-    if w.head_dim == 128 and w.dtype == "bf16" and group == 1:
+    if w.head_dim in (64, 128) and w.dtype == "bf16" and group == 1:
         return "reg"
     if not tensor_cores:
         return "cuda_core"

@@ -355,8 +355,8 @@ PKV_API int pkv_profile_reset(void);
  * caches, 1, 2 or 4 and an even number of kv heads): 1 (default) runs the
  * tensor-core kernel (tcgen05 MMAs into tensor memory), 0 the CUDA-core
  * kernels that serve every other shape (bf16 caches with one query head per
- * kv head and head_dim 128 stream K and V through registers; the rest stage
- * them in shared memory).  All compute the same attention; returns the
+ * kv head and head_dim 64 or 128 stream K and V through registers; the rest
+ * stage them in shared memory).  All compute the same attention; returns the
  * previous setting.  Process-wide. */
 PKV_API int pkv_set_tensor_core_gqa(int enable);
 

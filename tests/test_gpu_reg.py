@@ -1,5 +1,5 @@
-"""The register-streamed decode kernel (bf16 MHA, head_dim 128, blocks of 8,
-16 or 32 tokens read in 8-token chunks) against the oracle, and the staged
+"""The register-streamed decode kernel (bf16 MHA, head_dim 64 or 128, blocks
+of 8, 16 or 32 tokens read in 8-token chunks) against the oracle, and the staged
 kernel on the same inputs ("How PagedAttention works", items 2-5: the kernel walks the block
 table and gathers each block's keys and values wherever they sit).
 
@@ -43,6 +43,20 @@ def test_edge_lengths(form, bs, pt):
     out, kc, vc = gpu_step(w, partition_tokens=pt)
     assert_pool_equal(kc, kref, "k pool")
     assert_pool_equal(vc, vref, "v pool")
+    assert_close(out, ref, "bf16")
+    assert torch.count_nonzero(out[0]) == 0
+
+
+@pytest.mark.parametrize("bs,pt", [(8, 0), (8, 24), (16, 0), (16, 64), (32, 96)])
+def test_head_dim_64(form, bs, pt):
+    """head_dim 64: a chunk is 8 rows of 128 bytes, 4 rows per warp-wide
+    load; the same edge lengths and partitions as at head_dim 128."""
+    maxb = 1280 // bs
+    lens = [0, 1, 7, 8, 9, 15, 16, 17, 31, 33, 100, 1000, maxb * bs, 5, 1279, 63]
+    w = wl.custom(41 + bs, lens, heads=4, kv_heads=4, head_dim=64, block_size=bs, dtype="bf16", maxb=maxb)
+    ref, kref, _ = oracle_step(w)
+    out, kc, _ = gpu_step(w, partition_tokens=pt)
+    assert_pool_equal(kc, kref, "k pool")
     assert_close(out, ref, "bf16")
     assert torch.count_nonzero(out[0]) == 0
 
@@ -129,9 +143,11 @@ def test_bad_table_entry_sets_error(form, bs):
     assert torch.isfinite(out.float()).all()
 
 
-@pytest.mark.parametrize("bs,contiguous", [(8, False), (8, True), (16, False), (32, False)],
-                         ids=["bs8", "bs8_contiguous", "bs16", "bs32"])
-def test_full_size(form, bs, contiguous):
+@pytest.mark.parametrize("bs,contiguous,D", [(8, False, 128), (8, True, 128), (16, False, 128), (32, False, 128),
+                                            (16, False, 64)],
+                         ids=["bs8", "bs8_contiguous", "bs16", "bs32", "bs16_d64"])
+def test_full_size(form, bs, contiguous, D):
     """Batch-64 MHA (32 = 32 heads, contexts U[128, 2048], a pool of 256 Ki
-    tokens): all 64 x 32 rows, paged and contiguous placement."""
-    full_size_check(wl.mha(block_size=bs, contiguous=contiguous, device="cuda"))
+    tokens): all 64 x 32 rows, paged and contiguous placement, head_dim 128
+    and 64."""
+    full_size_check(wl.mha(block_size=bs, contiguous=contiguous, head_dim=D, device="cuda"))

@@ -17,7 +17,7 @@ FAMILY = {
     "mha": "reg", "gqa_sampling": "tc_bf16", "long_context": "tc_bf16",
     "prefix_bs8": "tc_bf16", "prefix_bs16": "tc_bf16", "prefix_bs32": "tc_bf16",
     "mha_fp8": "tc_fp8", "gqa_sampling_fp8": "tc_fp8", "long_context_fp8": "tc_fp8",
-    "mha_d64_fp8": "tc_fp8_d64", "mha_bs8": "reg",
+    "mha_d64_fp8": "tc_fp8_d64", "mha_bs8": "reg", "mha_d64": "reg",
 }
 
 
@@ -55,7 +55,7 @@ def test_kernel_family_by_shape(heads, kv_heads, dtype, head_dim, family):
 
 
 @pytest.mark.parametrize("bs,D,dtype,family", [(8, 128, "bf16", "reg"), (16, 128, "bf16", "reg"),
-                                              (32, 128, "bf16", "reg"), (16, 64, "bf16", "cuda_core"),
+                                              (32, 128, "bf16", "reg"), (16, 64, "bf16", "reg"),
                                               (8, 128, "f32", "cuda_core")])
 def test_kernel_family_mha_by_block_size(bs, D, dtype, family):
     w = wl.custom(1, [40, 7], heads=8, kv_heads=8, head_dim=D, block_size=bs, dtype=dtype)
