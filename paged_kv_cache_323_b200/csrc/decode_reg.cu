@@ -8,20 +8,21 @@ namespace pkv {
 
 namespace {
 constexpr int kRegWarps = 4;  // warps per CTA
-// CTAs per SM the registers are budgeted for: head_dim 128 holds 4 x 16
-// bytes per lane per chunk (126 registers, 4 CTAs); head_dim 64 half that
-// (80 registers, 6 CTAs), so more warps keep its 2 KB chunks in flight
-template <int D>
+// CTAs per SM the registers are budgeted for: a chunk of 2 KB of K and V
+// holds 4 x 16 bytes of each per lane (about 126 registers, 4 CTAs); the
+// 1 KB chunks of head_dim 64 at block size 8 hold half that (80 registers,
+// 6 CTAs), so more warps keep them in flight
+template <int D, int BS>
 constexpr int reg_min_blocks() {
-    return D == 64 ? 6 : 4;
+    return RegCfg<D, BS, kRegWarps>::RPL >= 4 ? 4 : 6;
 }
 
 template <int D>
 void (*reg_kernel(int BS))(const DecodeParams) {
     switch (BS) {
-        case 8: return decode_reg_kernel<D, 8, kRegWarps, reg_min_blocks<D>()>;
-        case 16: return decode_reg_kernel<D, 16, kRegWarps, reg_min_blocks<D>()>;
-        case 32: return decode_reg_kernel<D, 32, kRegWarps, reg_min_blocks<D>()>;
+        case 8: return decode_reg_kernel<D, 8, kRegWarps, reg_min_blocks<D, 8>()>;
+        case 16: return decode_reg_kernel<D, 16, kRegWarps, reg_min_blocks<D, 16>()>;
+        case 32: return decode_reg_kernel<D, 32, kRegWarps, reg_min_blocks<D, 32>()>;
         default: return nullptr;
     }
 }

@@ -14,12 +14,13 @@
 // reads the cache with plain 16-byte loads straight into registers:
 //  * One CTA per (sequence, kv head, partition), NW warps.  The partition's
 //    table entries are read once into shared memory and range-checked.
-//  * The partition is cut into chunks of 8 tokens (a whole block at block
-//    size 8, an 8-row-aligned run of a larger block: 2 KB of K and
-//    2 KB of V, contiguous in the [block][kv head][slot][dim] pool).  Warp w
-//    takes chunks w, w + NW, w + 2 NW, ...; lane l loads the 16-byte piece
-//    l % 16 of rows l / 16, l / 16 + 2, ... (one warp-wide load covers 512
-//    contiguous bytes).  The next chunk's K and V loads are issued before the
+//  * The partition is cut into chunks of 2 KB of K and 2 KB of V, each
+//    contiguous in the [block][kv head][slot][dim] pool: 8 tokens at head_dim
+//    128, 16 at head_dim 64 (8 when the block holds only 8), a whole block or
+//    an aligned run of rows of a larger one.  Warp w takes chunks w, w + NW,
+//    w + 2 NW, ...; lane l loads the 16-byte piece l % (D / 8) of rows
+//    l / (D / 8), and every 32 / (D / 8) rows after it (one warp-wide load
+//    covers 512 contiguous bytes).  The next chunk's K and V loads are issued before the
 //    current chunk is computed (two register buffers), so every warp keeps a
 //    whole chunk in flight while it works.
 //  * Partial dot products over a lane's 8 dims are reduced by the transposing
@@ -44,11 +45,13 @@ template <int D, int BS, int NW>
 struct RegCfg {
     static constexpr int CPR = D / 8;        // 16-byte pieces (8 bf16) per row
     static constexpr int RPI = 32 / CPR;     // rows covered by one warp-wide load
-    static constexpr int RW = 8;             // rows (tokens) per chunk
+    static constexpr int ROWB = D * 2;       // bytes of one token row
+    // rows (tokens) per chunk: 2 KB of K (8 rows at head_dim 128, 16 at 64),
+    // at most one block
+    static constexpr int RW = BS < 2048 / ROWB ? BS : 2048 / ROWB;
     static constexpr int CPB = BS / RW;      // chunks per block
     static constexpr int RPL = RW / RPI;     // rows per lane per chunk
     static constexpr int THREADS = NW * 32;
-    static constexpr int ROWB = D * 2;       // bytes of one token row
     static constexpr int SLICE = BS * ROWB;  // bytes of one (block, kv head)
     static constexpr int MAX_PART_TOKENS = 4096;
     static constexpr int MAX_PART_BLOCKS = MAX_PART_TOKENS / BS;

@@ -1,6 +1,7 @@
 """The register-streamed decode kernel's lane arithmetic, checked on the CPU.
 
-A 32-lane model of one warp working on one 8-token chunk, with the index
+A 32-lane model of one warp working on one chunk (2 KB of K: 8 tokens at
+head_dim 128, 16 at head_dim 64, at most one block), with the index
 formulas of decode_reg.cuh written out: which 16-byte piece of which row each
 lane loads, the transposing butterfly that turns the lanes' partial dot
 products into whole logits, the lane each row's probability is read from for
@@ -13,13 +14,15 @@ token's key is dotted with the query, then its value weighted).
 import numpy as np
 import pytest
 
-CHUNK_ROWS = 8  # tokens per chunk
+
+def chunk_rows(D, BS):
+    return min(BS, 2048 // (2 * D))
 
 
-def cfg(D):
-    cpr = D // 8             # 16-byte pieces (8 bf16) per row
-    rpi = 32 // cpr          # rows one warp-wide load covers
-    rpl = CHUNK_ROWS // rpi  # rows per lane per chunk
+def cfg(D, rows):
+    cpr = D // 8        # 16-byte pieces (8 bf16) per row
+    rpi = 32 // cpr     # rows one warp-wide load covers
+    rpl = rows // rpi   # rows per lane per chunk
     return cpr, rpi, rpl
 
 
@@ -51,30 +54,32 @@ def transpose_reduce(x, n, m):
 @pytest.mark.parametrize("D", [128, 64])
 @pytest.mark.parametrize("BS", [8, 16, 32])
 def test_chunk_loads_cover_each_byte_once(D, BS):
-    cpr, rpi, rpl = cfg(D)
+    rows = chunk_rows(D, BS)
+    cpr, rpi, rpl = cfg(D, rows)
     rowb = D * 2
     slice_bytes = BS * rowb
-    for q in range(BS // CHUNK_ROWS):  # every chunk of one block
+    assert BS % rows == 0 and rows * rowb <= 2048
+    for q in range(BS // rows):  # every chunk of one block
         seen = np.zeros(slice_bytes, dtype=int)
         for lane in range(32):
             c, r0 = lane % cpr, lane // cpr
             lane_off = r0 * rowb + c * 16  # within the (block, kv head) slice
             for k in range(rpl):
-                off = lane_off + (q % (BS // CHUNK_ROWS)) * CHUNK_ROWS * rowb + k * rpi * rowb
+                off = lane_off + (q % (BS // rows)) * rows * rowb + k * rpi * rowb
                 assert 0 <= off and off + 16 <= slice_bytes
                 seen[off:off + 16] += 1
-        chunk = slice(q * CHUNK_ROWS * rowb, (q + 1) * CHUNK_ROWS * rowb)
-        assert (seen[chunk] == 1).all() and seen.sum() == CHUNK_ROWS * rowb
+        chunk = slice(q * rows * rowb, (q + 1) * rows * rowb)
+        assert (seen[chunk] == 1).all() and seen.sum() == rows * rowb
 
 
-@pytest.mark.parametrize("D", [128, 64])
-def test_butterfly_logits_and_pv_sources(D):
-    cpr, rpi, rpl = cfg(D)
+@pytest.mark.parametrize("D,rows", [(128, 8), (64, 8), (64, 16)])
+def test_butterfly_logits_and_pv_sources(D, rows):
+    cpr, rpi, rpl = cfg(D, rows)
     spread = cpr // rpl  # lanes that end up holding one logit
     rng = np.random.default_rng(D)
     qv = rng.standard_normal(D)
-    K = rng.standard_normal((CHUNK_ROWS, D))
-    V = rng.standard_normal((CHUNK_ROWS, D))
+    K = rng.standard_normal((rows, D))
+    V = rng.standard_normal((rows, D))
     logits = K @ qv
 
     # partial dot products: lane (c, r0) over dims [8c, 8c + 8) of rows r0 + rpi k
@@ -120,5 +125,5 @@ def test_butterfly_logits_and_pv_sources(D):
 
     # the running sum: one owner lane per logit, summed over all 32 lanes
     owners = [lane for lane in range(32) if (lane % cpr) % spread == 0]
-    assert len(owners) == CHUNK_ROWS
+    assert len(owners) == rows
     assert np.isclose(sum(p[x] for x in owners), np.exp(logits - logits.max()).sum(), rtol=0, atol=1e-12)
