@@ -1,5 +1,5 @@
-// decode_reg.cuh -- paged decode attention for small blocks, streamed through
-// registers (sm_100a).
+// decode_reg.cuh -- paged decode attention with one query head per kv head,
+// the cache streamed through registers (sm_100a).
 //
 // Same computation as decode_attn.cuh ("PagedAttention Explained: Virtual
 // Memory for the KV Cache", section "How PagedAttention works", item 5: the
@@ -11,7 +11,8 @@
 // Staging such slices through shared memory costs one asynchronous copy each
 // (bulk copy, or sixteen 16-byte cp.async per warp), and at that size the
 // per-copy cost, not HBM, set the pace of the staged kernel.  Here each warp
-// reads the cache with plain 16-byte loads straight into registers:
+// reads the cache with plain 16-byte loads straight into registers, which
+// also beat the staged kernel at block sizes 16 and 32:
 //  * One CTA per (sequence, kv head, partition), NW warps.  The partition's
 //    table entries are read once into shared memory and range-checked.
 //  * The partition is cut into chunks of 2 KB of K and 2 KB of V, each
@@ -20,9 +21,9 @@
 //    an aligned run of rows of a larger one.  Warp w takes chunks w, w + NW,
 //    w + 2 NW, ...; lane l loads the 16-byte piece l % (D / 8) of rows
 //    l / (D / 8), and every 32 / (D / 8) rows after it (one warp-wide load
-//    covers 512 contiguous bytes).  The next chunk's K and V loads are issued before the
-//    current chunk is computed (two register buffers), so every warp keeps a
-//    whole chunk in flight while it works.
+//    covers 512 contiguous bytes).  The next chunk's K and V loads are
+//    issued before the current chunk is computed (two register buffers), so
+//    every warp keeps a whole chunk in flight while it works.
 //  * Partial dot products over a lane's 8 dims are reduced by the transposing
 //    butterfly of decode_attn.cuh; online softmax in base 2 with fp32 running
 //    max and sum; PV into fp32 registers (8 dims per lane).  Unused slots of
