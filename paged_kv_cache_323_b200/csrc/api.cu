@@ -183,8 +183,9 @@ size_t workspace_bytes_for(long long num_seqs, long long num_heads, long long pa
 }
 
 // Partition size when the caller passes 0.
-//  * CUDA-core kernel: 1024 tokens (fewer split-K merges than 512 at no loss
-//    of parallelism on batch-64 MHA), doubled (up to 4096) while a sequence
+//  * CUDA-core kernels: 1024 tokens (fewer split-K merges than 512 at no loss
+//    of parallelism on batch-64 MHA; 2048 for tokens of at most 256 bytes
+//    per kv head), doubled (up to 4096) while a sequence
 //    of the maximum length would still be split into more than 64 partitions
 //    and the grid keeps at least four waves of 3 CTAs per SM.
 //  * Tensor-core kernels: 4096 tokens, halved (down to 512) while the grid
@@ -193,7 +194,7 @@ size_t workspace_bytes_for(long long num_seqs, long long num_heads, long long pa
 //    parallel-sampling GQA batch ran at 0.75 / 0.88 / 0.97 of peak with
 //    1024 / 2048 / 4096-token partitions.
 int auto_partition_tokens(long long num_seqs, long long num_kv_heads, long long max_ctx, bool tc,
-                          bool fp8 = false, long long min_ctas = 4LL * 148 * 2) {
+                          bool short_tokens = false, long long min_ctas = 4LL * 148 * 2) {
     if (tc) {
         // The tensor-core kernels run 2 to 4 CTAs per SM, and a CTA's start
         // (table and q fetch, first TMA round trip) and merge are a fixed
@@ -206,9 +207,13 @@ int auto_partition_tokens(long long num_seqs, long long num_kv_heads, long long 
             pt /= 2;
         return (int)pt;
     }
-    // fp8 caches carry half the bytes per token, so a CTA's fixed cost weighs
-    // twice as much: 2048 tokens (on batch-64 MHA 154 us at 1024, 139 us at 2048)
-    long long pt = fp8 ? 2 * kAutoPartitionTokens : kAutoPartitionTokens;
+    // Where a token of one kv head carries at most 256 bytes of K and V (fp8
+    // caches, bf16 at head_dim 64) a CTA's fixed cost weighs twice as much
+    // per token: 2048 tokens (batch-64 MHA over fp8 on the staged kernel:
+    // 154 us at 1024, 139 us at 2048; bf16 at head_dim 64 on the
+    // register-streamed kernel: 104.7 / 102.4 us), against 1024 for 512-byte
+    // tokens (bf16 at head_dim 128: 194.3 us at 1024, 200.9 at 2048)
+    long long pt = short_tokens ? 2 * kAutoPartitionTokens : kAutoPartitionTokens;
     const long long min_cc_ctas = 4LL * 148 * 3;
     while (pt < kMaxPartitionTokens && (max_ctx + pt - 1) / pt > 64 &&
            num_seqs * num_kv_heads * ((max_ctx + 2 * pt - 1) / (2 * pt)) >= min_cc_ctas)
@@ -229,14 +234,16 @@ int resolve_partition_tokens(int num_seqs, int num_heads, int num_kv_heads, int 
     const int group = num_kv_heads > 0 ? num_heads / num_kv_heads : 1;
     const bool tc = tc_shape(dtype, head_dim, block_size, group, num_kv_heads);
     const bool fp8 = dtype == PKV_FP8_E4M3;
+    const int elt = dtype == PKV_F32 ? 4 : (dtype == PKV_BF16 ? 2 : 1);
+    const bool short_tokens = 2LL * head_dim * elt <= 256;  // K and V bytes of one token, one kv head
     // The head_dim-64 tensor-core kernel runs one CTA per pair of kv heads,
     // always in longest-first order, where the last CTAs to start are the
     // shortest: its partitions stay long while the grid fills one wave of 5
     // CTAs per SM (batch-64 MHA: 59.3 us at 2048 tokens, 68.4 at 1024, 76.1
     // at 512).
     const bool pairs = tc && head_dim == 64;
-    int pt = pairs ? auto_partition_tokens(num_seqs, num_kv_heads / 2, max_ctx, tc, fp8, 148LL * 5)
-                   : auto_partition_tokens(num_seqs, num_kv_heads, max_ctx, tc, fp8);
+    int pt = pairs ? auto_partition_tokens(num_seqs, num_kv_heads / 2, max_ctx, tc, short_tokens, 148LL * 5)
+                   : auto_partition_tokens(num_seqs, num_kv_heads, max_ctx, tc, short_tokens);
     // the persistent fp8 tensor-core kernel holds two tables of at most 128
     // blocks per CTA: 2048 tokens at block size 16 (batch-64 MHA 106.5 us at
     // 2048 against 112.1 us at 1024; the parallel-sampling batch 125.3 / 144.1)

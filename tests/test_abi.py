@@ -133,6 +133,9 @@ def test_partition_tokens(pk):
     pt = pk.paged_attention_partition_tokens
     bf = pk.PKV_BF16
     assert pt(64, 32, 32, 128, 16, 2048, bf, 0) == 1024  # batch-64 MHA, CUDA-core kernel
+    # tokens of at most 256 bytes per kv head (here bf16 at head_dim 64): twice as long
+    assert pt(64, 32, 32, 64, 16, 2048, bf, 0) == 2048
+    assert pt(4, 8, 8, 64, 16, 64, pk.PKV_F32, 0) == 1024  # fp32 at head_dim 64: 512-byte tokens
     assert pt(64, 32, 32, 128, 16, 2048, bf, 256) == 256  # explicit sizes pass through
     # grouped-query heads on the tensor-core kernel: long partitions unless the grid gets small
     assert pt(256, 32, 8, 128, 16, 8256, bf, 0) == 4096
