@@ -60,3 +60,15 @@ def test_kernel_family_by_shape(heads, kv_heads, dtype, head_dim, family):
 def test_kernel_family_mha_by_block_size(bs, D, dtype, family):
     w = wl.custom(1, [40, 7], heads=8, kv_heads=8, head_dim=D, block_size=bs, dtype=dtype)
     assert bench.decode_kernel_family(w) == family
+
+
+@pytest.mark.parametrize("heads,kv_heads,dtype,head_dim,family", [
+    (32, 32, "bf16", 128, "reg"), (32, 8, "bf16", 128, "cuda_core"), (32, 32, "fp8", 128, "cuda_core"),
+    (32, 32, "bf16", 64, "reg"), (32, 32, "fp8", 64, "cuda_core"),
+])
+def test_kernel_family_with_tensor_cores_off(heads, kv_heads, dtype, head_dim, family):
+    """bench.py --cuda-cores: bf16 MHA keeps the register-streamed kernel, the
+    rest falls to the staged CUDA-core kernel."""
+    w = wl.custom(1, [40, 7], heads=heads, kv_heads=kv_heads, head_dim=head_dim, block_size=16,
+                  dtype=dtype)
+    assert bench.decode_kernel_family(w, tensor_cores=False) == family
